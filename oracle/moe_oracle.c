@@ -1,0 +1,341 @@
+/*
+ * CPU oracle for the forward pass of one sparse Mixture-of-Experts FFN layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the slow, plain, obviously correct
+ * statement of what the layer computes.  Only the test suite, the smoke check
+ * and the benchmark's CPU-baseline leg may load it.  It shares no code, header,
+ * table or helper with the CUDA library, and it never reads a value that the
+ * CUDA library produced.
+ *
+ * Arithmetic: every sum is accumulated in double in ascending index order; the
+ * only roundings are the ones the definitions below state.  Inputs arrive as
+ * fp32 values or as raw bf16 bit patterns; a bf16 value is widened to fp32 and
+ * then to double exactly.
+ *
+ * Sources (page title, section):
+ *  - "From Switch Transformer to GLaM" (blog.euler0525.cn), sections
+ *    "Dense Scaling vs MoE" (FFN(x) = W2 s(W1 x); router h(x) = W_r x; softmax
+ *    p_i), "Switch Transformer: making MoE simple" (top-1 i* = argmax p,
+ *    y = p_{i*} E_{i*}(x)), "Load balancing" (f_i, P_i, L_aux = alpha N sum f_i
+ *    P_i, alpha = 1e-2), "Expert Capacity and Token Dropping" (C = T/N x cf;
+ *    an overflowing token skips the expert FFN and only the residual carries
+ *    it), "Why GLaM returns to top-2" (y = w1 E_{i1} + w2 E_{i2}).
+ *  - CMU 10-423 Lecture 16 "Mixture of Experts", section 2.3 (sparse gating
+ *    G(x) = softmax(topk(x W_g, k)), non-top-k entries set to -inf; the
+ *    Mixtral SwiGLU expert; a zero router picks the lowest indices on ties),
+ *    section 6.1 (capacity with the GShard rule: all tokens' first choices are
+ *    placed before any second choice), exercise 3 (C = cf k T / N = 320).
+ *  - CS25 Lecture 05 notes "Scaling Transformers through Sparsity", section
+ *    "Static compilation meets dynamic routing" (capacity-aware dispatch:
+ *    tokens claim slots in token order, a full expert skips the token).
+ *  - "Training Stability, Results & Limitations" (nano-ai.tech), section 2.1
+ *    Selective Precision (router in float32; bf16 rounding example).
+ *
+ * Readings taken where the pages are silent or garbled:
+ *  - top-k ties go to the lower expert index; the ranking uses the fp32 logits;
+ *  - C = floor(k T cf / N), computed exactly from the double cf;
+ *  - slot claim is rank-major (every rank-0 choice before any rank-1 choice),
+ *    then token order;
+ *  - gates are fixed before capacity: a surviving assignment keeps its gate;
+ *  - a token with no kept assignment gets a zero layer output;
+ *  - f_i counts the pre-capacity top-1 choice; P_i averages the full softmax;
+ *  - Swish uses beta = 1: silu(z) = z / (1 + exp(-z));
+ *  - biases are optional and are added inside the expert, before gating.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#include <string.h>
+
+#define ORACLE_F32 0
+#define ORACLE_BF16 1
+
+#define ORACLE_RELU 0
+#define ORACLE_SWIGLU 1
+
+/* ---- bf16 <-> fp32, written from the format's definition ----------------
+ * A bf16 value is the upper 16 bits of an IEEE-754 binary32 value.
+ * Widening appends 16 zero bits (exact).  Narrowing rounds to nearest, ties to
+ * even, on the 16 discarded bits; NaN stays NaN (quiet). */
+static float bf16_bits_to_float(uint16_t b) {
+    uint32_t u = ((uint32_t)b) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+uint16_t oracle_float_to_bf16_bits(float f) {
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu) != 0u) {
+        return (uint16_t)((u >> 16) | 0x0040u); /* quiet NaN */
+    }
+    uint32_t upper = u >> 16;
+    uint32_t lower = u & 0xFFFFu;
+    if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) {
+        upper += 1u; /* carries into the exponent correctly, up to infinity */
+    }
+    return (uint16_t)upper;
+}
+
+float oracle_bf16_round(float f) {
+    return bf16_bits_to_float(oracle_float_to_bf16_bits(f));
+}
+
+/* element i of an array that is fp32 or raw bf16, widened to double */
+static double load_elem(const void* base, int dtype, size_t i) {
+    if (dtype == ORACLE_BF16) {
+        return (double)bf16_bits_to_float(((const uint16_t*)base)[i]);
+    }
+    return (double)((const float*)base)[i];
+}
+
+/* ---- Router: logits, softmax, top-k, gate --------------------------------
+ * h_{t,i} = sum_j x_{t,j} W_r[i,j] (+ b_r[i]) in double, ascending j, then
+ * rounded once to fp32 (the router is an fp32 computation).
+ * p_{t,i} = exp(h_i - m) / sum_j exp(h_j - m), m = max_j h_j, in double,
+ * stored as fp32 (the shift by m leaves the softmax value unchanged).
+ * top-1: the largest h; on equal h the lower index.  top-2: the largest h
+ * among the other experts, same tie rule.
+ * gate, k = 1: p_{i*}.  k = 2: softmax over the two kept logits,
+ * g_r = exp(h_{i_r} - h_{i_1}) / (1 + exp(h_{i_2} - h_{i_1})).
+ *
+ * x: [T, d] (dtype x_dtype); w_r: [N, d] fp32; b_r: [N] fp32 or NULL.
+ * Outputs: logits [T, N] fp32 (nullable), probs [T, N] fp32 (nullable),
+ * idx [T, k] int32, gate [T, k] fp32. */
+void oracle_router(int64_t T, int32_t d, int32_t N, int32_t k,
+                   const void* x, int32_t x_dtype, const float* w_r, const float* b_r,
+                   float* logits, float* probs, int32_t* idx, float* gate) {
+    float h[1024];
+    double e[1024];
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t i = 0; i < N; ++i) {
+            double acc = 0.0;
+            for (int32_t j = 0; j < d; ++j) {
+                acc += load_elem(x, x_dtype, (size_t)t * d + j) * (double)w_r[(size_t)i * d + j];
+            }
+            if (b_r) acc += (double)b_r[i];
+            h[i] = (float)acc;
+        }
+        double m = (double)h[0];
+        for (int32_t i = 1; i < N; ++i) {
+            if ((double)h[i] > m) m = (double)h[i];
+        }
+        double s = 0.0;
+        for (int32_t i = 0; i < N; ++i) {
+            e[i] = exp((double)h[i] - m);
+            s += e[i];
+        }
+        for (int32_t i = 0; i < N; ++i) {
+            if (logits) logits[(size_t)t * N + i] = h[i];
+            if (probs) probs[(size_t)t * N + i] = (float)(e[i] / s);
+        }
+        int32_t i1 = 0;
+        for (int32_t i = 1; i < N; ++i) {
+            if (h[i] > h[i1]) i1 = i; /* strict: the lower index keeps a tie */
+        }
+        if (k == 1) {
+            idx[t] = i1;
+            gate[t] = (float)(e[i1] / s);
+        } else {
+            int32_t i2 = (i1 == 0) ? 1 : 0;
+            for (int32_t i = 0; i < N; ++i) {
+                if (i == i1) continue;
+                if (h[i] > h[i2]) i2 = i;
+            }
+            double r = exp((double)h[i2] - (double)h[i1]);
+            idx[t * 2 + 0] = i1;
+            idx[t * 2 + 1] = i2;
+            gate[t * 2 + 0] = (float)(1.0 / (1.0 + r));
+            gate[t * 2 + 1] = (float)(r / (1.0 + r));
+        }
+    }
+}
+
+/* ---- Load-balancing loss -------------------------------------------------
+ * f_i = #{t : top-1 choice of t is i} / T   (pre-capacity, argmax indicator)
+ * P_i = sum_t p_{t,i} / T
+ * aux = alpha * N * sum_i f_i P_i
+ * idx: [T, k]; its column 0 is the top-1 choice.  T = 0 gives all zeros. */
+void oracle_aux(int64_t T, int32_t N, int32_t k, const int32_t* idx, const float* probs,
+                double alpha, double* f, double* P, double* aux) {
+    for (int32_t i = 0; i < N; ++i) {
+        f[i] = 0.0;
+        P[i] = 0.0;
+    }
+    *aux = 0.0;
+    if (T <= 0) return;
+    for (int64_t t = 0; t < T; ++t) {
+        f[idx[t * k]] += 1.0;
+        for (int32_t i = 0; i < N; ++i) P[i] += (double)probs[(size_t)t * N + i];
+    }
+    double s = 0.0;
+    for (int32_t i = 0; i < N; ++i) {
+        f[i] /= (double)T;
+        P[i] /= (double)T;
+        s += f[i] * P[i];
+    }
+    *aux = alpha * (double)N * s;
+}
+
+/* ---- Capacity --------------------------------------------------------------
+ * C = floor(k * T * cf / N), exact.  cf is a binary double m * 2^e with m an
+ * odd-or-zero 53-bit integer, so k T cf / N = k T m / (N 2^-e) is a rational
+ * whose floor is taken with 128-bit integers.  Returns -1 when the inputs are
+ * out of range (T < 0, N < 1, k < 1, cf < 0 or not finite, result > 2^31-1). */
+int32_t oracle_capacity(int64_t T, int32_t N, int32_t k, double cf) {
+    if (T < 0 || N < 1 || k < 1 || !(cf >= 0.0) || isinf(cf)) return -1;
+    if (cf == 0.0 || T == 0) return 0;
+    int ex;
+    double fr = frexp(cf, &ex);           /* cf = fr * 2^ex, 0.5 <= fr < 1 */
+    int64_t m = (int64_t)ldexp(fr, 53);   /* exact: fr has 53 significant bits */
+    ex -= 53;                             /* cf = m * 2^ex */
+    while (m % 2 == 0 && ex < 0) {
+        m /= 2;
+        ex += 1;
+    }
+    __int128 num = (__int128)k * (__int128)T * (__int128)m;
+    __int128 den = (__int128)N;
+    if (ex >= 0) {
+        if (ex > 60) return -1;
+        num <<= ex;
+    } else {
+        if (-ex > 100) return 0;
+        den <<= -ex;
+    }
+    __int128 q = num / den;
+    if (q > (__int128)2147483647) return -1;
+    return (int32_t)q;
+}
+
+/* ---- Capacity-limited slot claim -------------------------------------------
+ * For r = 0..k-1, for t = 0..T-1 in order: e = idx[t, r]; the assignment takes
+ * claim number pos[t, r] = (claims on e so far); it is kept iff pos < C.
+ * counts[r, e] = claims of rank r on e (pre-capacity); kept[e] =
+ * min(sum_r counts[r, e], C); offsets[e] = sum_{e' < e} kept[e'], offsets[N] =
+ * total kept rows.  The compact expert-major row of a kept (t, r) is
+ * offsets[e] + pos[t, r]. */
+void oracle_dispatch(int64_t T, int32_t N, int32_t k, int32_t C, const int32_t* idx,
+                     int32_t* pos, uint8_t* drop, int32_t* counts, int32_t* kept,
+                     int32_t* offsets) {
+    int64_t claims[1024];
+    for (int32_t e = 0; e < N; ++e) claims[e] = 0;
+    for (int32_t r = 0; r < k; ++r) {
+        for (int32_t e = 0; e < N; ++e) counts[r * N + e] = 0;
+        for (int64_t t = 0; t < T; ++t) {
+            int32_t e = idx[t * k + r];
+            int64_t p = claims[e];
+            claims[e] = p + 1;
+            counts[r * N + e] += 1;
+            pos[t * k + r] = (int32_t)p;
+            drop[t * k + r] = (uint8_t)(p >= (int64_t)C);
+        }
+    }
+    int64_t acc = 0;
+    for (int32_t e = 0; e < N; ++e) {
+        int64_t total = claims[e];
+        kept[e] = (int32_t)(total < (int64_t)C ? total : (int64_t)C);
+        offsets[e] = (int32_t)acc;
+        acc += kept[e];
+    }
+    offsets[N] = (int32_t)acc;
+}
+
+/* ---- One expert on one token -----------------------------------------------
+ * ReLU expert:   u = W1 x + b1; a = max(u, 0); y = W2 a + b2.
+ * SwiGLU expert: u = W1 x + b1; v = W3 x + b3; a = silu(u) * v; y = W2 a + b2.
+ * W1, W3: [d_ff, d]; W2: [d, d_ff] (output-by-input, so W x is a row dot
+ * product); biases nullable.  All in double; a is NOT rounded.
+ * x: d values (dtype x_dtype); weights and biases: dtype w_dtype.  y: [d]. */
+void oracle_expert_ffn(int32_t d, int32_t d_ff, int32_t act,
+                       const void* x, int32_t x_dtype, size_t x_off,
+                       const void* w1, const void* b1, const void* w3, const void* b3,
+                       const void* w2, const void* b2, int32_t w_dtype,
+                       size_t w1_off, size_t b1_off, size_t w2_off, size_t b2_off,
+                       double* a_scratch, double* y) {
+    for (int32_t j = 0; j < d_ff; ++j) {
+        double u = 0.0;
+        for (int32_t i = 0; i < d; ++i) {
+            u += load_elem(w1, w_dtype, w1_off + (size_t)j * d + i) * load_elem(x, x_dtype, x_off + i);
+        }
+        if (b1) u += load_elem(b1, w_dtype, b1_off + j);
+        if (act == ORACLE_RELU) {
+            a_scratch[j] = u > 0.0 ? u : 0.0;
+        } else {
+            double v = 0.0;
+            for (int32_t i = 0; i < d; ++i) {
+                v += load_elem(w3, w_dtype, w1_off + (size_t)j * d + i) * load_elem(x, x_dtype, x_off + i);
+            }
+            if (b3) v += load_elem(b3, w_dtype, b1_off + j);
+            a_scratch[j] = (u / (1.0 + exp(-u))) * v;
+        }
+    }
+    for (int32_t n = 0; n < d; ++n) {
+        double acc = 0.0;
+        for (int32_t j = 0; j < d_ff; ++j) {
+            acc += load_elem(w2, w_dtype, w2_off + (size_t)n * d_ff + j) * a_scratch[j];
+        }
+        if (b2) acc += load_elem(b2, w_dtype, b2_off + n);
+        y[n] = acc;
+    }
+}
+
+/* ---- Layer output for a list of tokens --------------------------------------
+ * out_t = sum over kept r of g_{t,r} * E_{idx[t,r]}(x_t), in double; zero when
+ * no assignment of t is kept (the residual path outside the layer carries a
+ * dropped token).  out_exact gets the double value; out_rounded the value
+ * rounded once to the output dtype (fp32, or bf16 round-to-nearest-even).
+ *
+ * x: [T, d]; w1, w3: [N, d_ff, d]; w2: [N, d, d_ff]; b1, b3: [N, d_ff];
+ * b2: [N, d].  idx, gate, drop: [T, k] from oracle_router / oracle_dispatch.
+ * tokens: the n_tok token indices to evaluate; outputs are [n_tok, d].
+ * scratch: d_ff + d doubles. */
+void oracle_layer_tokens(int32_t d, int32_t d_ff, int32_t k, int32_t act,
+                         const void* x, int32_t x_dtype,
+                         const void* w1, const void* b1, const void* w3, const void* b3,
+                         const void* w2, const void* b2, int32_t w_dtype,
+                         const int32_t* idx, const float* gate, const uint8_t* drop,
+                         int64_t n_tok, const int64_t* tokens, int32_t out_dtype,
+                         double* scratch, double* out_exact, float* out_rounded) {
+    double* a = scratch;
+    double* y = scratch + d_ff;
+    for (int64_t q = 0; q < n_tok; ++q) {
+        int64_t t = tokens[q];
+        double* o = out_exact + (size_t)q * d;
+        for (int32_t n = 0; n < d; ++n) o[n] = 0.0;
+        for (int32_t r = 0; r < k; ++r) {
+            if (drop[t * k + r]) continue;
+            int32_t e = idx[t * k + r];
+            double g = (double)gate[t * k + r];
+            oracle_expert_ffn(d, d_ff, act, x, x_dtype, (size_t)t * d,
+                              w1, b1, w3, b3, w2, b2, w_dtype,
+                              (size_t)e * d_ff * d, (size_t)e * d_ff,
+                              (size_t)e * d * d_ff, (size_t)e * d, a, y);
+            for (int32_t n = 0; n < d; ++n) o[n] += g * y[n];
+        }
+        for (int32_t n = 0; n < d; ++n) {
+            float v = (float)o[n];
+            out_rounded[(size_t)q * d + n] = (out_dtype == ORACLE_BF16) ? oracle_bf16_round(v) : v;
+        }
+    }
+}
+
+/* ---- Un-gated expert outputs in compact expert-major order ------------------
+ * ye[row] = E_e(x_t) for each requested compact row, where row = offsets[e] +
+ * pos[t, r] for a kept (t, r).  rows_token / rows_expert give (t, e) for each
+ * requested row.  Output [n_rows, d] in double. */
+void oracle_expert_rows(int32_t d, int32_t d_ff, int32_t act,
+                        const void* x, int32_t x_dtype,
+                        const void* w1, const void* b1, const void* w3, const void* b3,
+                        const void* w2, const void* b2, int32_t w_dtype,
+                        int64_t n_rows, const int64_t* rows_token, const int32_t* rows_expert,
+                        double* scratch, double* ye) {
+    for (int64_t q = 0; q < n_rows; ++q) {
+        int64_t t = rows_token[q];
+        int32_t e = rows_expert[q];
+        oracle_expert_ffn(d, d_ff, act, x, x_dtype, (size_t)t * d,
+                          w1, b1, w3, b3, w2, b2, w_dtype,
+                          (size_t)e * d_ff * d, (size_t)e * d_ff,
+                          (size_t)e * d * d_ff, (size_t)e * d, scratch, ye + (size_t)q * d);
+    }
+}
