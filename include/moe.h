@@ -1,0 +1,199 @@
+/*
+ * moe.h -- C ABI of libmoe_b200.so: the forward pass of one sparse
+ * Mixture-of-Experts FFN layer (Switch / sparsely-gated MoE) on one B200.
+ *
+ * The layer, as the pages define it:
+ *   router      h = W_r x (+ b_r), fp32;  p = softmax(h)
+ *               ("From Switch Transformer to GLaM", section "Dense Scaling vs
+ *               MoE"; "Training Stability, Results & Limitations", section 2.1
+ *               Selective Precision: the router runs in float32)
+ *   top-k gate  k = 1: i* = argmax p, gate p_{i*}  (GLaM page, "Switch
+ *               Transformer: making MoE simple");  k = 2: the two largest
+ *               logits, gates = softmax over those two logits (CMU 10-423
+ *               Lecture 16, section 2.3; GLaM page, "Why GLaM returns to top-2")
+ *   capacity    C = floor(k T cf / N) slots per expert (GLaM page, "Expert
+ *               Capacity and Token Dropping"; Lecture 16, exercise 3); tokens
+ *               claim slots in token order, all first choices before any second
+ *               choice (CS25 Lecture 05 notes, capacity-aware dispatch; Lecture
+ *               16 section 6.1, GShard rule); an overflowing assignment is
+ *               dropped and a token with no kept assignment outputs zero (its
+ *               residual connection, outside this layer, carries it)
+ *   expert      ReLU: W2 relu(W1 x + b1) + b2 (GLaM page, FFN(x) = W2 s(W1 x));
+ *               SwiGLU: W2 (silu(W1 x + b1) * (W3 x + b3)) + b2 (Lecture 16,
+ *               section 2.3, Mixtral expert; silu(z) = z / (1 + e^-z))
+ *   combine     out_t = sum over kept r of gate_{t,r} * E_{idx[t,r]}(x_t)
+ *   aux loss    alpha N sum_i f_i P_i, f_i = fraction of tokens whose top-1
+ *               choice is i (before capacity), P_i = mean router probability
+ *               (GLaM page, section "Load balancing"; alpha = 1e-2)
+ *
+ * Conventions shared by every entry point
+ *   - All array pointers are DEVICE pointers unless stated; the caller owns
+ *     every buffer.  The library never allocates or frees memory.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream).  Only moe_read_device_status
+ *     synchronises.  Calls are stateless apart from the caller's workspace, so
+ *     distinct workspaces may be used from distinct threads.
+ *   - Layouts (row-major): x, out [T, d_model]; w_r [N, d_model] fp32; b_r [N]
+ *     fp32; w1, w3 [N, d_ff, d_model]; w2 [N, d_model, d_ff] ("output x input",
+ *     so every product is a row dot product); b1, b3 [N, d_ff]; b2 [N, d_model];
+ *     idx, gate, pos, drop [T, k]; counts [k, N]; kept [N]; offsets [N + 1].
+ *   - dtype MOE_BF16: x, out, weights and biases are bf16; MOE_F32: all fp32.
+ *     The router weights w_r, b_r and the gates are always fp32.
+ *   - The compact expert-major row of a kept assignment (t, r) is
+ *     offsets[idx[t,r]] + pos[t,r]; rows of expert e are
+ *     [offsets[e], offsets[e+1]), in claim order.
+ *   - Every pointer must be 16-byte aligned.  Nullable pointers say so.
+ *   - Errors come back as a moe_status; invalid arguments are rejected on the
+ *     host before anything is launched.  Device-side failures (a bounded wait
+ *     that ran out) are latched in the workspace and reported by
+ *     moe_read_device_status.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, negative size, bad enum */
+    MOE_ERR_UNSUPPORTED = 2,   /* valid but outside what the kernels handle */
+    MOE_ERR_WORKSPACE = 3,     /* workspace pointer null or smaller than required */
+    MOE_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed */
+    MOE_ERR_TIMEOUT = 5        /* a device-side bounded wait gave up (latched) */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1 } moe_dtype;
+typedef enum { MOE_RELU = 0, MOE_SWIGLU = 1 } moe_act;
+
+/* Layer shape.  Limits: 0 <= T < 2^28; 1 <= n_experts <= 128; top_k in {1, 2}
+ * with top_k <= n_experts; capacity >= 0 (the explicit C; see moe_capacity);
+ * d_model, d_ff >= 1; for MOE_BF16, d_model and d_ff multiples of 16. */
+typedef struct {
+    int32_t T;
+    int32_t d_model;
+    int32_t d_ff;
+    int32_t n_experts;
+    int32_t top_k;
+    int32_t capacity;
+    int32_t dtype;   /* moe_dtype */
+    int32_t act;     /* moe_act */
+    float alpha;     /* load-balancing loss weight */
+} moe_config;
+
+/* Expert capacity C = floor(k * T * cf / N), computed exactly from the binary
+ * value of cf (GLaM page, "Expert Capacity and Token Dropping"; CMU 10-423
+ * Lecture 16, exercise 3: 1.25 * 2 * 1024 / 8 = 320).  Host-only, no device
+ * work.  Returns -1 for T < 0, N < 1, k < 1, cf negative or not finite, or a
+ * result above 2^31 - 1. */
+int32_t moe_capacity(int64_t T, int32_t n_experts, int32_t top_k, double capacity_factor);
+
+/* Bytes of device workspace every entry point below needs for `cfg` (0 if the
+ * config is invalid).  One workspace serves all entry points; it must not be
+ * shared by calls that may run concurrently. */
+size_t moe_workspace_bytes(const moe_config* cfg);
+
+/* Prepare a workspace for first use: clears the latched device status (the
+ * first 256 bytes).  Call once after allocating a workspace, before any other
+ * entry point uses it; later calls keep it consistent by themselves.
+ * Asynchronous on `stream`. */
+int32_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Static description of a status code. */
+const char* moe_status_string(int32_t status);
+
+/* Router + load-balancing loss (rows A1, A2, A8 of the hot path).
+ * In:  x [T, d] (dtype), w_r [N, d] fp32, b_r [N] fp32 (nullable).
+ * Out: idx [T, k] int32 (experts, descending logit, ties to the lower index),
+ *      gate [T, k] fp32, probs [T, N] fp32 (nullable: full softmax),
+ *      f [N], P [N], aux [1] as fp64 (each nullable).
+ * ws: workspace of ws_bytes >= moe_workspace_bytes(cfg). */
+int32_t moe_route(const moe_config* cfg, const void* x, const float* w_r, const float* b_r,
+                  int32_t* idx, float* gate, float* probs,
+                  double* f, double* P, double* aux,
+                  void* ws, size_t ws_bytes, void* stream);
+
+/* Capacity-limited dispatch (row A3 and the gather of A4).
+ * In:  x [T, d] (dtype; nullable when xe is NULL), idx [T, k], gate [T, k].
+ * Out: pos [T, k] int32 (claim number of the assignment on its expert: all
+ *      rank-0 claims in token order, then the rank-1 claims), drop [T, k] uint8
+ *      (1 iff pos >= C), counts [k, N] (claims per rank before capacity),
+ *      kept [N] = min(sum_r counts[r][e], C), offsets [N + 1] (exclusive prefix
+ *      of kept), row_token [R] / row_gate [R] (token and gate of every compact
+ *      row, R = offsets[N]), xe [R, d] (dtype; the gathered rows; nullable).
+ *      The row_* and xe buffers must hold min(k T, N C) rows. */
+int32_t moe_dispatch(const moe_config* cfg, const void* x, const int32_t* idx, const float* gate,
+                     int32_t* pos, uint8_t* drop, int32_t* counts, int32_t* kept,
+                     int32_t* offsets, int32_t* row_token, float* row_gate, void* xe,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* Grouped expert FFN over the compact rows (rows A5, A6).
+ * In:  xe [R, d] (dtype) with R = offsets[N]; offsets [N + 1]; w1, w2 and
+ *      (SwiGLU) w3; b1, b3, b2 nullable.
+ * Out: ye [R, d] (dtype): the un-gated expert output of every row. */
+int32_t moe_expert_ffn(const moe_config* cfg, const void* xe, const int32_t* offsets,
+                       const void* w1, const void* b1, const void* w3, const void* b3,
+                       const void* w2, const void* b2, void* ye,
+                       void* ws, size_t ws_bytes, void* stream);
+
+/* Gate-scaled combine back to token order (row A7).
+ * out[t] = sum over r with drop[t,r] == 0 of gate[t,r] * ye[offsets[idx[t,r]] +
+ * pos[t,r]], accumulated in fp32 and rounded once; zero if every assignment of
+ * t was dropped.  In: ye [R, d], idx, pos, drop, gate [T, k], offsets [N + 1].
+ * Out: out [T, d] (dtype). */
+int32_t moe_combine(const moe_config* cfg, const void* ye, const int32_t* idx,
+                    const int32_t* pos, const uint8_t* drop, const float* gate,
+                    const int32_t* offsets, void* out, void* stream);
+
+/* The whole layer forward in one call (rows A1-A8), fused where it pays:
+ * the top-1 bf16 path scatters gate * E(x) straight from the second GEMM's
+ * epilogue into out.
+ * In:  x, w_r, b_r (nullable), w1, b1 (nullable), w3 (SwiGLU), b3 (nullable),
+ *      w2, b2 (nullable).
+ * Out: out [T, d] (required); idx, gate, pos, drop, counts, kept, offsets, f, P,
+ *      aux: each nullable (when NULL the value stays in the workspace). */
+int32_t moe_forward(const moe_config* cfg, const void* x, const float* w_r, const float* b_r,
+                    const void* w1, const void* b1, const void* w3, const void* b3,
+                    const void* w2, const void* b2, void* out,
+                    int32_t* idx, float* gate, int32_t* pos, uint8_t* drop,
+                    int32_t* counts, int32_t* kept, int32_t* offsets,
+                    double* f, double* P, double* aux,
+                    void* ws, size_t ws_bytes, void* stream);
+
+/* moe_forward, plus stage timing for profiling: `events` points to 6 cudaEvent_t
+ * handles (passed as void*, created by the caller; any entry may be NULL) that
+ * are recorded on `stream` at the stage boundaries: [0] before the router,
+ * [1] after the router and aux loss, [2] after the dispatch and gather, [3]
+ * after the first expert GEMM, [4] after the second expert GEMM, [5] after the
+ * combine (equal to [4] on the fused top-1 path).  events == NULL behaves as
+ * moe_forward.  The kernels launched are identical to moe_forward's. */
+int32_t moe_forward_events(const moe_config* cfg, const void* x, const float* w_r, const float* b_r,
+                           const void* w1, const void* b1, const void* w3, const void* b3,
+                           const void* w2, const void* b2, void* out,
+                           int32_t* idx, float* gate, int32_t* pos, uint8_t* drop,
+                           int32_t* counts, int32_t* kept, int32_t* offsets,
+                           double* f, double* P, double* aux,
+                           void* ws, size_t ws_bytes, void* stream, void* const* events);
+
+/* Synchronise `stream`, then return (and clear) the device status latched in
+ * the workspace: MOE_OK, or MOE_ERR_TIMEOUT if a bounded device-side wait gave
+ * up during an earlier call on this workspace.  The outputs of such a call are
+ * undefined; the CUDA context stays usable. */
+int32_t moe_read_device_status(void* ws, void* stream);
+
+/* Test hook (not part of the layer): launch one block of the dispatch scan's
+ * look-back in isolation, waiting on a predecessor that never publishes, with a
+ * wait limit of `limit_ns` nanoseconds.  The wait gives up, latches
+ * MOE_ERR_TIMEOUT in the workspace and returns; read it back with
+ * moe_read_device_status. */
+int32_t moe_test_lookback_timeout(void* ws, size_t ws_bytes, int64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,414 @@
+// C-ABI front end of libmoe_b200: argument validation, workspace layout and
+// the launch sequence of each entry point (declared and documented in
+// include/moe.h).  No entry point allocates, frees or synchronises, except
+// moe_read_device_status, which synchronises its stream.
+#include <cmath>
+#include <cstring>
+
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+struct Layout {
+    size_t hdr, part_cnt, part_psum, scan_state;
+    size_t idx, gate, pos, drop, counts, kept, offsets, f, P, aux;
+    size_t row_token, row_gate, xe, h, ye;
+    size_t total;
+    int64_t rows;   // min(k T, N C): compact rows the buffers hold
+};
+
+int64_t compact_rows(const moe_config& c) {
+    int64_t a = (int64_t)c.top_k * c.T;
+    int64_t b = (int64_t)c.n_experts * c.capacity;
+    return a < b ? a : b;
+}
+
+Layout layout_of(const moe_config& c) {
+    Layout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off += round_up(bytes > 0 ? bytes : 1, 256);
+        return o;
+    };
+    const size_t T = (size_t)c.T, k = (size_t)c.top_k, N = (size_t)c.n_experts;
+    const size_t esz = c.dtype == MOE_BF16 ? 2 : 4;
+    L.rows = compact_rows(c);
+    const size_t R = (size_t)(L.rows > 0 ? L.rows : 1);
+    L.hdr = take(sizeof(WsHeader));
+    const size_t nbr = (size_t)router_blocks(c.T, c.n_experts);
+    L.part_cnt = take(4 * nbr * N);
+    L.part_psum = take(4 * nbr * N);
+    const size_t nbs = (size_t)scan_blocks(c.T);
+    L.scan_state = take(4 * (nbs * k * N > 8 ? nbs * k * N : 8));
+    L.idx = take(4 * T * k);
+    L.gate = take(4 * T * k);
+    L.pos = take(4 * T * k);
+    L.drop = take(T * k);
+    L.counts = take(4 * k * N);
+    L.kept = take(4 * N);
+    L.offsets = take(4 * (N + 1));
+    L.f = take(8 * N);
+    L.P = take(8 * N);
+    L.aux = take(8);
+    L.row_token = take(4 * R);
+    L.row_gate = take(4 * R);
+    L.xe = take(esz * R * (size_t)c.d_model);
+    L.h = take(esz * R * (size_t)c.d_ff);
+    L.ye = take(esz * R * (size_t)c.d_model);
+    L.total = off;
+    return L;
+}
+
+bool aligned(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int32_t validate(const moe_config* c) {
+    if (!c) return MOE_ERR_INVALID_ARG;
+    if (c->T < 0 || c->d_model < 1 || c->d_ff < 1 || c->n_experts < 1 || c->top_k < 1 || c->capacity < 0)
+        return MOE_ERR_INVALID_ARG;
+    if (c->dtype != MOE_F32 && c->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+    if (c->act != MOE_RELU && c->act != MOE_SWIGLU) return MOE_ERR_INVALID_ARG;
+    if (c->top_k > c->n_experts) return MOE_ERR_INVALID_ARG;
+    if (!std::isfinite(c->alpha)) return MOE_ERR_INVALID_ARG;
+    if (c->T >= (1 << 28) || c->n_experts > 128 || c->top_k > 2) return MOE_ERR_UNSUPPORTED;
+    if (c->dtype == MOE_BF16 && (c->d_model % 16 != 0 || c->d_ff % 16 != 0)) return MOE_ERR_UNSUPPORTED;
+    if ((int64_t)c->d_model * c->d_ff >= ((int64_t)1 << 40)) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+int32_t check_ws(const moe_config* c, void* ws, size_t ws_bytes) {
+    if (!ws || !aligned(ws)) return MOE_ERR_WORKSPACE;
+    if (ws_bytes < layout_of(*c).total) return MOE_ERR_WORKSPACE;
+    return MOE_OK;
+}
+
+// required pointer: non-null and 16-byte aligned; optional: null or aligned
+bool req(const void* p) { return p != nullptr && aligned(p); }
+bool opt(const void* p) { return p == nullptr || aligned(p); }
+
+template <typename T>
+T* at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(reinterpret_cast<char*>(ws) + off);
+}
+
+int32_t cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+int32_t moe_capacity(int64_t T, int32_t n_experts, int32_t top_k, double cf) {
+    if (T < 0 || n_experts < 1 || top_k < 1 || !(cf >= 0.0) || std::isinf(cf)) return -1;
+    if (T == 0 || cf == 0.0) return 0;
+    // cf = m * 2^ex exactly, m an integer below 2^53
+    int ex = 0;
+    double fr = std::frexp(cf, &ex);
+    long long m = (long long)std::ldexp(fr, 53);
+    ex -= 53;
+    while ((m & 1) == 0 && ex < 0) {
+        m >>= 1;
+        ++ex;
+    }
+    unsigned __int128 num = (unsigned __int128)top_k * (unsigned __int128)T * (unsigned __int128)m;
+    unsigned __int128 den = (unsigned __int128)n_experts;
+    if (ex >= 0) {
+        if (ex > 60) return -1;
+        num <<= ex;
+    } else {
+        if (-ex > 100) return 0;
+        den <<= -ex;
+    }
+    unsigned __int128 q = num / den;
+    if (q > (unsigned __int128)2147483647) return -1;
+    return (int32_t)q;
+}
+
+size_t moe_workspace_bytes(const moe_config* cfg) {
+    if (validate(cfg) != MOE_OK) return 0;
+    return layout_of(*cfg).total;
+}
+
+int32_t moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+    if (!ws || !aligned(ws) || ws_bytes < sizeof(WsHeader)) return MOE_ERR_WORKSPACE;
+    return cuda_status(cudaMemsetAsync(ws, 0, sizeof(WsHeader), (cudaStream_t)stream));
+}
+
+const char* moe_status_string(int32_t status) {
+    switch (status) {
+        case MOE_OK: return "ok";
+        case MOE_ERR_INVALID_ARG: return "invalid argument";
+        case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+        case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case MOE_ERR_CUDA: return "CUDA call failed";
+        case MOE_ERR_TIMEOUT: return "device-side wait timed out";
+        default: return "unknown status";
+    }
+}
+
+int32_t moe_route(const moe_config* cfg, const void* x, const float* w_r, const float* b_r, int32_t* idx,
+                  float* gate, float* probs, double* f, double* P, double* aux, void* ws, size_t ws_bytes,
+                  void* stream) {
+    int32_t st = validate(cfg);
+    if (st != MOE_OK) return st;
+    if (!req(w_r) || !opt(b_r) || !opt(probs) || !opt(f) || !opt(P) || !opt(aux)) return MOE_ERR_INVALID_ARG;
+    if (cfg->T > 0 && (!req(x) || !req(idx) || !req(gate))) return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+    const Layout L = layout_of(*cfg);
+    RouterArgs a{};
+    a.x = x;
+    a.dtype = cfg->dtype;
+    a.w_r = w_r;
+    a.b_r = b_r;
+    a.T = cfg->T;
+    a.d = cfg->d_model;
+    a.N = cfg->n_experts;
+    a.k = cfg->top_k;
+    a.idx = idx;
+    a.gate = gate;
+    a.probs = probs;
+    a.part_cnt = at<int32_t>(ws, L.part_cnt);
+    a.part_psum = at<float>(ws, L.part_psum);
+    a.f = f;
+    a.P = P;
+    a.aux = aux;
+    a.alpha = cfg->alpha;
+    return cuda_status(launch_router(a, (cudaStream_t)stream));
+}
+
+static int32_t dispatch_impl(const moe_config* cfg, const void* x, const int32_t* idx, const float* gate,
+                             int32_t* pos, uint8_t* drop, int32_t* counts, int32_t* kept, int32_t* offsets,
+                             int32_t* row_token, float* row_gate, void* xe, void* zero_out, void* ws,
+                             cudaStream_t s) {
+    const Layout L = layout_of(*cfg);
+    if (cfg->T == 0) {
+        cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->top_k * cfg->n_experts, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(kept, 0, sizeof(int32_t) * cfg->n_experts, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (cfg->n_experts + 1), s);
+        return cuda_status(e);
+    }
+    DispatchArgs a{};
+    a.x = x;
+    a.dtype = cfg->dtype;
+    a.idx = idx;
+    a.gate = gate;
+    a.T = cfg->T;
+    a.d = cfg->d_model;
+    a.N = cfg->n_experts;
+    a.k = cfg->top_k;
+    a.C = cfg->capacity;
+    a.pos = pos;
+    a.drop = drop;
+    a.counts = counts;
+    a.kept = kept;
+    a.offsets = offsets;
+    a.row_token = row_token;
+    a.row_gate = row_gate;
+    a.xe = xe;
+    a.zero_out = zero_out;
+    a.scan_state = at<uint32_t>(ws, L.scan_state);
+    a.hdr = at<WsHeader>(ws, L.hdr);
+    return cuda_status(launch_dispatch(a, s));
+}
+
+int32_t moe_dispatch(const moe_config* cfg, const void* x, const int32_t* idx, const float* gate, int32_t* pos,
+                     uint8_t* drop, int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* row_token,
+                     float* row_gate, void* xe, void* ws, size_t ws_bytes, void* stream) {
+    int32_t st = validate(cfg);
+    if (st != MOE_OK) return st;
+    if (!req(counts) || !req(kept) || !req(offsets) || !opt(xe) || !opt(x)) return MOE_ERR_INVALID_ARG;
+    if (cfg->T > 0 && (!req(idx) || !req(gate) || !req(pos) || !req(drop) || !req(row_token) || !req(row_gate)))
+        return MOE_ERR_INVALID_ARG;
+    if (xe && cfg->T > 0 && !req(x)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+    return dispatch_impl(cfg, x, idx, gate, pos, drop, counts, kept, offsets, row_token, row_gate, xe, nullptr, ws,
+                         (cudaStream_t)stream);
+}
+
+static int32_t ffn_impl(const moe_config* cfg, const void* xe, const int32_t* offsets, const void* w1,
+                        const void* b1, const void* w3, const void* b3, const void* w2, const void* b2, void* ye,
+                        void* scatter_out, const int32_t* row_token, const float* row_gate, void* ws,
+                        cudaStream_t s, void* const* mid_event = nullptr) {
+    const Layout L = layout_of(*cfg);
+    if (L.rows <= 0) {   // nothing can be kept
+        if (mid_event && *mid_event) return cuda_status(cudaEventRecord((cudaEvent_t)*mid_event, s));
+        return MOE_OK;
+    }
+    FfnArgs a{};
+    a.dtype = cfg->dtype;
+    a.act = cfg->act;
+    a.N = cfg->n_experts;
+    a.d = cfg->d_model;
+    a.d_ff = cfg->d_ff;
+    a.C = (int)(L.rows < cfg->capacity ? L.rows : cfg->capacity);
+    a.R_cap = L.rows;
+    a.xe = xe;
+    a.offsets = offsets;
+    a.w1 = w1;
+    a.b1 = b1;
+    a.w3 = w3;
+    a.b3 = b3;
+    a.w2 = w2;
+    a.b2 = b2;
+    a.h = at<void>(ws, L.h);
+    a.ye = ye;
+    a.scatter_out = scatter_out;
+    a.row_token = row_token;
+    a.row_gate = row_gate;
+    a.hdr = at<WsHeader>(ws, L.hdr);
+    a.mid_event = mid_event ? *mid_event : nullptr;
+    return cuda_status(launch_expert_ffn(a, s));
+}
+
+int32_t moe_expert_ffn(const moe_config* cfg, const void* xe, const int32_t* offsets, const void* w1, const void* b1,
+                       const void* w3, const void* b3, const void* w2, const void* b2, void* ye, void* ws,
+                       size_t ws_bytes, void* stream) {
+    int32_t st = validate(cfg);
+    if (st != MOE_OK) return st;
+    if (!req(xe) || !req(offsets) || !req(w1) || !req(w2) || !req(ye) || !opt(b1) || !opt(b2) || !opt(b3))
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->act == MOE_SWIGLU ? !req(w3) : !opt(w3)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+    return ffn_impl(cfg, xe, offsets, w1, b1, w3, b3, w2, b2, ye, nullptr, nullptr, nullptr, ws,
+                    (cudaStream_t)stream);
+}
+
+int32_t moe_combine(const moe_config* cfg, const void* ye, const int32_t* idx, const int32_t* pos,
+                    const uint8_t* drop, const float* gate, const int32_t* offsets, void* out, void* stream) {
+    int32_t st = validate(cfg);
+    if (st != MOE_OK) return st;
+    if (cfg->T > 0 && (!req(idx) || !req(pos) || !req(drop) || !req(gate) || !req(offsets) || !req(out)))
+        return MOE_ERR_INVALID_ARG;
+    if (!opt(ye)) return MOE_ERR_INVALID_ARG;
+    if (cfg->T > 0 && compact_rows(*cfg) > 0 && !ye) return MOE_ERR_INVALID_ARG;
+    CombineArgs a{};
+    a.dtype = cfg->dtype;
+    a.T = cfg->T;
+    a.d = cfg->d_model;
+    a.k = cfg->top_k;
+    a.ye = ye;
+    a.idx = idx;
+    a.pos = pos;
+    a.drop = drop;
+    a.gate = gate;
+    a.offsets = offsets;
+    a.out = out;
+    return cuda_status(launch_combine(a, (cudaStream_t)stream));
+}
+
+static int32_t forward_impl(const moe_config* cfg, const void* x, const float* w_r, const float* b_r,
+                            const void* w1, const void* b1, const void* w3, const void* b3, const void* w2,
+                            const void* b2, void* out, int32_t* idx, float* gate, int32_t* pos, uint8_t* drop,
+                            int32_t* counts, int32_t* kept, int32_t* offsets, double* f, double* P, double* aux,
+                            void* ws, size_t ws_bytes, cudaStream_t s, void* const* events) {
+    int32_t st = validate(cfg);
+    if (st != MOE_OK) return st;
+    if (!req(w_r) || !req(w1) || !req(w2) || !opt(b_r) || !opt(b1) || !opt(b2) || !opt(b3)) return MOE_ERR_INVALID_ARG;
+    if (cfg->act == MOE_SWIGLU ? !req(w3) : !opt(w3)) return MOE_ERR_INVALID_ARG;
+    if (cfg->T > 0 && (!req(x) || !req(out))) return MOE_ERR_INVALID_ARG;
+    if (!opt(idx) || !opt(gate) || !opt(pos) || !opt(drop) || !opt(counts) || !opt(kept) || !opt(offsets) || !opt(f) ||
+        !opt(P) || !opt(aux))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+    const Layout L = layout_of(*cfg);
+    auto mark = [&](int i) -> bool {
+        if (!events || !events[i]) return true;
+        return cudaEventRecord((cudaEvent_t)events[i], s) == cudaSuccess;
+    };
+    if (!idx) idx = at<int32_t>(ws, L.idx);
+    if (!gate) gate = at<float>(ws, L.gate);
+    if (!pos) pos = at<int32_t>(ws, L.pos);
+    if (!drop) drop = at<uint8_t>(ws, L.drop);
+    if (!counts) counts = at<int32_t>(ws, L.counts);
+    if (!kept) kept = at<int32_t>(ws, L.kept);
+    if (!offsets) offsets = at<int32_t>(ws, L.offsets);
+    if (!f) f = at<double>(ws, L.f);
+    if (!P) P = at<double>(ws, L.P);
+    if (!aux) aux = at<double>(ws, L.aux);
+    int32_t* row_token = at<int32_t>(ws, L.row_token);
+    float* row_gate = at<float>(ws, L.row_gate);
+    void* xe = at<void>(ws, L.xe);
+    void* ye = at<void>(ws, L.ye);
+
+    if (!mark(0)) return MOE_ERR_CUDA;
+    st = moe_route(cfg, x, w_r, b_r, idx, gate, nullptr, f, P, aux, ws, ws_bytes, s);
+    if (st != MOE_OK) return st;
+    if (!mark(1)) return MOE_ERR_CUDA;
+    // top-1 bf16: the second GEMM scatters gate * E(x) into out; dispatch zeroes
+    // the rows of dropped tokens.  Otherwise expert outputs go through the combine.
+    const bool fused = cfg->dtype == MOE_BF16 && cfg->top_k == 1;
+    st = dispatch_impl(cfg, x, idx, gate, pos, drop, counts, kept, offsets, row_token, row_gate, xe,
+                       fused ? out : nullptr, ws, s);
+    if (st != MOE_OK) return st;
+    if (!mark(2)) return MOE_ERR_CUDA;
+    st = ffn_impl(cfg, xe, offsets, w1, b1, w3, b3, w2, b2, ye, fused ? out : nullptr, row_token, row_gate, ws, s,
+                  events ? events + 3 : nullptr);
+    if (st != MOE_OK) return st;
+    if (!mark(4)) return MOE_ERR_CUDA;
+    if (!fused) {
+        CombineArgs a{};
+        a.dtype = cfg->dtype;
+        a.T = cfg->T;
+        a.d = cfg->d_model;
+        a.k = cfg->top_k;
+        a.ye = ye;
+        a.idx = idx;
+        a.pos = pos;
+        a.drop = drop;
+        a.gate = gate;
+        a.offsets = offsets;
+        a.out = out;
+        st = cuda_status(launch_combine(a, s));
+        if (st != MOE_OK) return st;
+    }
+    if (!mark(5)) return MOE_ERR_CUDA;
+    return MOE_OK;
+}
+
+int32_t moe_forward(const moe_config* cfg, const void* x, const float* w_r, const float* b_r, const void* w1,
+                    const void* b1, const void* w3, const void* b3, const void* w2, const void* b2, void* out,
+                    int32_t* idx, float* gate, int32_t* pos, uint8_t* drop, int32_t* counts, int32_t* kept,
+                    int32_t* offsets, double* f, double* P, double* aux, void* ws, size_t ws_bytes, void* stream) {
+    return forward_impl(cfg, x, w_r, b_r, w1, b1, w3, b3, w2, b2, out, idx, gate, pos, drop, counts, kept, offsets,
+                        f, P, aux, ws, ws_bytes, (cudaStream_t)stream, nullptr);
+}
+
+int32_t moe_forward_events(const moe_config* cfg, const void* x, const float* w_r, const float* b_r,
+                           const void* w1, const void* b1, const void* w3, const void* b3, const void* w2,
+                           const void* b2, void* out, int32_t* idx, float* gate, int32_t* pos, uint8_t* drop,
+                           int32_t* counts, int32_t* kept, int32_t* offsets, double* f, double* P, double* aux,
+                           void* ws, size_t ws_bytes, void* stream, void* const* events) {
+    return forward_impl(cfg, x, w_r, b_r, w1, b1, w3, b3, w2, b2, out, idx, gate, pos, drop, counts, kept, offsets,
+                        f, P, aux, ws, ws_bytes, (cudaStream_t)stream, events);
+}
+
+int32_t moe_read_device_status(void* ws, void* stream) {
+    if (!ws || !aligned(ws)) return MOE_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
+    int32_t host = 0;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (cudaMemcpyAsync(&host, &hdr->status, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return MOE_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (host != MOE_OK) {
+        if (cudaMemsetAsync(&hdr->status, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+        if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
+    }
+    return host;
+}
+
+int32_t moe_test_lookback_timeout(void* ws, size_t ws_bytes, int64_t limit_ns, void* stream) {
+    if (!ws || !aligned(ws) || ws_bytes < sizeof(WsHeader) + 256) return MOE_ERR_WORKSPACE;
+    if (limit_ns <= 0 || limit_ns > 10000000000LL) return MOE_ERR_INVALID_ARG;
+    WsHeader* hdr = reinterpret_cast<WsHeader*>(ws);
+    uint32_t* state = at<uint32_t>(ws, sizeof(WsHeader));
+    return cuda_status(launch_lookback_timeout_probe(state, hdr, (long long)limit_ns, (cudaStream_t)stream));
+}
+
+}  // extern "C"

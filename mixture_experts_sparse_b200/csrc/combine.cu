@@ -1,0 +1,76 @@
+// Gate-scaled combine back to token order:
+//   out_t = sum over kept r of gate[t, r] * ye[offsets[idx[t, r]] + pos[t, r]]
+// accumulated in fp32 in rank order and rounded once; a token whose every
+// assignment was dropped outputs zero (its residual connection, outside the
+// layer, carries it).  "From Switch Transformer to GLaM": y = p_{i*} E_{i*}(x)
+// for top-1 and y = w1 E_{i1}(x) + w2 E_{i2}(x) for top-2, "Expert Capacity and
+// Token Dropping" (an overflowing token skips the expert FFN).
+// One warp per token, 16-byte vector loads/stores: an HBM-bound gather.
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+template <typename XT>
+__global__ void __launch_bounds__(256)
+combine_kernel(const XT* __restrict__ ye, const int32_t* __restrict__ idx, const int32_t* __restrict__ pos,
+               const uint8_t* __restrict__ drop, const float* __restrict__ gate,
+               const int32_t* __restrict__ offsets, int64_t T, int d, int k, XT* __restrict__ out) {
+    constexpr int VEC = 16 / sizeof(XT);
+    const int lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (t >= T) return;
+    int64_t row[2] = {-1, -1};
+    float g[2] = {0.f, 0.f};
+    for (int r = 0; r < k; ++r) {
+        const int64_t a = t * k + r;
+        if (!drop[a]) {
+            row[r] = (int64_t)offsets[idx[a]] + pos[a];
+            g[r] = gate[a];
+        }
+    }
+    XT* dst = out + t * (int64_t)d;
+    if (((size_t)d * sizeof(XT)) % 16 == 0) {
+        for (int c = lane * VEC; c < d; c += 32 * VEC) {
+            float acc[VEC];
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) acc[j] = 0.f;
+            for (int r = 0; r < k; ++r) {
+                if (row[r] < 0) continue;
+                uint4 v = __ldg(reinterpret_cast<const uint4*>(ye + row[r] * d + c));
+                const XT* xv = reinterpret_cast<const XT*>(&v);
+#pragma unroll
+                for (int j = 0; j < VEC; ++j) acc[j] = fmaf(g[r], Elem<XT>::to_f(xv[j]), acc[j]);
+            }
+            XT o[VEC];
+#pragma unroll
+            for (int j = 0; j < VEC; ++j) o[j] = Elem<XT>::from_f(acc[j]);
+            *reinterpret_cast<uint4*>(dst + c) = *reinterpret_cast<uint4*>(o);
+        }
+    } else {
+        for (int c = lane; c < d; c += 32) {
+            float acc = 0.f;
+            for (int r = 0; r < k; ++r)
+                if (row[r] >= 0) acc = fmaf(g[r], Elem<XT>::to_f(ye[row[r] * d + c]), acc);
+            dst[c] = Elem<XT>::from_f(acc);
+        }
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
+    if (a.T <= 0) return cudaSuccess;
+    const unsigned grid = (unsigned)((a.T + 7) / 8);
+    if (a.dtype == MOE_BF16) {
+        combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+            reinterpret_cast<const __nv_bfloat16*>(a.ye), a.idx, a.pos, a.drop, a.gate, a.offsets, a.T, a.d, a.k,
+            reinterpret_cast<__nv_bfloat16*>(a.out));
+    } else {
+        combine_kernel<float><<<grid, 256, 0, s>>>(reinterpret_cast<const float*>(a.ye), a.idx, a.pos, a.drop,
+                                                   a.gate, a.offsets, a.T, a.d, a.k, reinterpret_cast<float*>(a.out));
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace moe

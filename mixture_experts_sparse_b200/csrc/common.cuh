@@ -1,0 +1,102 @@
+// Shared device/host helpers of libmoe_b200 (internal header).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// ---- workspace header (first 256 bytes of every workspace) ----------------
+struct WsHeader {
+    int32_t status;        // latched moe_status of device-side failures
+    int32_t scan_ticket;   // dynamic block index of the dispatch scan
+    int32_t scan_done;     // finished-block counter of the dispatch scan
+    int32_t route_done;    // unused slot kept for alignment
+    int32_t pad[60];
+};
+static_assert(sizeof(WsHeader) == 256, "header size");
+
+// Default limit of every device-side bounded wait: far above any legitimate
+// wait (microseconds), low enough that a wedged wait returns promptly.
+constexpr long long kWaitLimitNs = 2000000000LL;
+
+__device__ __forceinline__ long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return (long long)t;
+}
+
+__device__ __forceinline__ void latch_status(int32_t* status, int32_t code) {
+    atomicCAS(status, 0, code);
+}
+
+// ---- bf16 / f32 element access ------------------------------------------
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+    static __device__ __forceinline__ float load(const float* p) { return *p; }
+    static __device__ __forceinline__ float to_f(float v) { return v; }
+    static __device__ __forceinline__ float from_f(float v) { return v; }
+};
+template <> struct Elem<__nv_bfloat16> {
+    static __device__ __forceinline__ float load(const __nv_bfloat16* p) { return __bfloat162float(*p); }
+    static __device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+    static __device__ __forceinline__ __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
+};
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// ---- launchers implemented in the .cu files ---------------------------------
+struct RouterArgs {
+    const void* x; int dtype; const float* w_r; const float* b_r;
+    int64_t T; int d; int N; int k;
+    int32_t* idx; float* gate; float* probs;
+    int32_t* part_cnt; float* part_psum;   // [nblk, N]
+    double* f; double* P; double* aux; float alpha;
+};
+int router_blocks(int64_t T, int N);
+cudaError_t launch_router(const RouterArgs& a, cudaStream_t s);
+
+struct DispatchArgs {
+    const void* x; int dtype; const int32_t* idx; const float* gate;
+    int64_t T; int d; int N; int k; int C;
+    int32_t* pos; uint8_t* drop; int32_t* counts; int32_t* kept; int32_t* offsets;
+    int32_t* row_token; float* row_gate; void* xe;
+    void* zero_out;              // top-1 fused path: rows of dropped tokens are zeroed
+    uint32_t* scan_state; WsHeader* hdr;
+};
+int scan_blocks(int64_t T);
+cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s);
+cudaError_t launch_lookback_timeout_probe(uint32_t* state, WsHeader* hdr, long long limit_ns,
+                                          cudaStream_t s);
+
+struct FfnArgs {
+    int dtype; int act; int N; int d; int d_ff; int C; int64_t R_cap;
+    const void* xe; const int32_t* offsets;
+    const void* w1; const void* b1; const void* w3; const void* b3;
+    const void* w2; const void* b2;
+    void* h;                      // [R_cap, d_ff] scratch
+    void* ye;                     // [R, d] (used when scatter_out == nullptr)
+    void* scatter_out;            // top-1 fused: out[row_token[r]] = row_gate[r] * E(x)
+    const int32_t* row_token; const float* row_gate;
+    WsHeader* hdr;
+    void* mid_event;              // optional cudaEvent_t recorded between the two stages
+};
+cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t s);
+
+struct CombineArgs {
+    int dtype; int64_t T; int d; int k;
+    const void* ye; const int32_t* idx; const int32_t* pos; const uint8_t* drop;
+    const float* gate; const int32_t* offsets; void* out;
+};
+cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
+
+}  // namespace moe

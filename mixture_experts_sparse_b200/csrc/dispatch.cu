@@ -1,0 +1,265 @@
+// Capacity-limited dispatch of the MoE layer: slot claiming in token order,
+// drop mask, compact expert-major row map and the gather of x into it.
+//
+// Definition: CS25 Lecture 05 notes "Scaling Transformers through Sparsity",
+// section "Static compilation meets dynamic routing" (capacity-aware dispatch:
+// in token order a token joins its expert's slots while fewer than C are taken,
+// otherwise it skips the expert); CMU 10-423 Lecture 16, section 6.1 (GShard
+// rule: every token's first choice is placed before any second choice); "From
+// Switch Transformer to GLaM", "Expert Capacity and Token Dropping".
+//
+// pos[t, r] = number of earlier claims on idx[t, r], where "earlier" is
+// rank-major then token order; an assignment is kept iff pos < C.  This is an
+// exclusive prefix count over (rank, token) per expert, computed as:
+//   1. scan_kernel: a block owns 1024 consecutive tokens.  Warps rank their
+//      32-token groups with __match_any_sync (tokens of a warp that pick the same
+//      expert), giving in-block ranks and a per-(rank, expert) block aggregate;
+//      a decoupled look-back across blocks (dynamic block tickets, bounded
+//      spin) turns the aggregates into exclusive block prefixes.  The last block
+//      to finish derives counts, kept = min(count, C) and the offsets.
+//   2. scatter_kernel: one warp per assignment adds the rank-0 total to rank-1
+//      positions, writes pos/drop and the row map, and copies x[t] into its
+//      compact row with 16-byte vector accesses.
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kScanThreads = 256;
+constexpr int kScanTokens = 1024;          // tokens per scan block (8 warps x 128)
+constexpr int kWarpTokens = kScanTokens / 8;
+constexpr uint32_t kFlagAgg = 1u << 30;    // block aggregate published
+constexpr uint32_t kFlagPre = 2u << 30;    // inclusive prefix published
+constexpr uint32_t kValMask = (1u << 30) - 1u;
+
+__device__ __forceinline__ uint32_t ld_relaxed(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_relaxed(uint32_t* p, uint32_t v) {
+    asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Decoupled look-back for one counter: publish this block's aggregate, then walk
+// back over predecessors until one with an inclusive prefix is found.  Waiting
+// on a predecessor that has not published is bounded by limit_ns; on expiry the
+// wait latches MOE_ERR_TIMEOUT and this block publishes anyway, so successors
+// never wait on it.
+__device__ uint32_t lookback(uint32_t* state, int bid, int c, int kN, uint32_t agg,
+                             long long limit_ns, int32_t* status) {
+    if (bid == 0) {
+        st_relaxed(state + c, kFlagPre | agg);
+        return 0u;
+    }
+    st_relaxed(state + (int64_t)bid * kN + c, kFlagAgg | agg);
+    uint32_t excl = 0;
+    int p = bid - 1;
+    long long t_start = -1;
+    unsigned spins = 0;
+    while (p >= 0) {
+        uint32_t v = ld_relaxed(state + (int64_t)p * kN + c);
+        uint32_t fl = v & ~kValMask;
+        if (fl == 0u) {
+            if (t_start < 0) t_start = global_ns();
+            if ((++spins & 63u) == 0u && global_ns() - t_start > limit_ns) {
+                latch_status(status, MOE_ERR_TIMEOUT);
+                break;
+            }
+            __nanosleep(64);
+            continue;
+        }
+        excl += v & kValMask;
+        if (fl == kFlagPre) break;
+        --p;
+    }
+    st_relaxed(state + (int64_t)bid * kN + c, kFlagPre | ((excl + agg) & kValMask));
+    return excl;
+}
+
+__global__ void __launch_bounds__(kScanThreads)
+scan_kernel(const int32_t* __restrict__ idx, int64_t T, int N, int k, int C, int nblk,
+            int32_t* __restrict__ pos, int32_t* __restrict__ counts, int32_t* __restrict__ kept,
+            int32_t* __restrict__ offsets, uint32_t* __restrict__ state, WsHeader* hdr,
+            long long limit_ns) {
+    __shared__ int s_bid;
+    __shared__ int s_last;
+    __shared__ int s_wcnt[8][256];
+    __shared__ uint32_t s_excl[256];
+    __shared__ int s_tot[256];
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int kN = k * N;
+    if (tid == 0) s_bid = atomicAdd(&hdr->scan_ticket, 1);
+    for (int q = tid; q < 8 * 256; q += kScanThreads) (&s_wcnt[0][0])[q] = 0;
+    __syncthreads();
+    const int bid = s_bid;
+    const int64_t tw0 = (int64_t)bid * kScanTokens + warp * kWarpTokens;
+
+    // 1. in-warp ranks, in token order, per (rank, expert) counter
+    int rank[kWarpTokens / 32][2];
+    const unsigned lt_mask = (1u << lane) - 1u;
+#pragma unroll
+    for (int it = 0; it < kWarpTokens / 32; ++it) {
+        const int64_t t = tw0 + it * 32 + lane;
+        const bool valid = t < T;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            if (r >= k) break;
+            const int key = valid ? r * N + idx[t * k + r] : -1;
+            const unsigned peers = __match_any_sync(0xffffffffu, key);
+            const int before = __popc(peers & lt_mask);
+            if (valid) rank[it][r] = s_wcnt[warp][key] + before;
+            __syncwarp();
+            if (valid && lane == __ffs(peers) - 1) s_wcnt[warp][key] += __popc(peers);
+            __syncwarp();
+        }
+    }
+    __syncthreads();
+
+    // 2. per counter: warp offsets inside the block, block aggregate, look-back
+    for (int c = tid; c < kN; c += kScanThreads) {
+        int run = 0;
+        for (int w = 0; w < 8; ++w) {
+            int v = s_wcnt[w][c];
+            s_wcnt[w][c] = run;
+            run += v;
+        }
+        s_excl[c] = lookback(state, bid, c, kN, (uint32_t)run, limit_ns, &hdr->status);
+    }
+    __syncthreads();
+
+    // 3. local claim numbers (rank 1 still lacks the global rank-0 total)
+#pragma unroll
+    for (int it = 0; it < kWarpTokens / 32; ++it) {
+        const int64_t t = tw0 + it * 32 + lane;
+        if (t >= T) break;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            if (r >= k) break;
+            const int key = r * N + idx[t * k + r];
+            pos[t * k + r] = (int)s_excl[key] + s_wcnt[warp][key] + rank[it][r];
+        }
+    }
+
+    // 4. the last block to finish derives counts, kept and offsets
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = (atomicAdd(&hdr->scan_done, 1) == nblk - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    for (int c = tid; c < kN; c += kScanThreads) {
+        int tot = (int)(ld_relaxed(state + (int64_t)(nblk - 1) * kN + c) & kValMask);
+        s_tot[c] = tot;
+        counts[c] = tot;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int acc = 0;
+        for (int e = 0; e < N; ++e) {
+            int total = s_tot[e] + (k == 2 ? s_tot[N + e] : 0);
+            int ke = total < C ? total : C;
+            kept[e] = ke;
+            offsets[e] = acc;
+            acc += ke;
+        }
+        offsets[N] = acc;
+    }
+}
+
+template <typename XT>
+__global__ void __launch_bounds__(256)
+scatter_kernel(const XT* __restrict__ x, const int32_t* __restrict__ idx, const float* __restrict__ gate,
+               int64_t T, int d, int N, int k, int C,
+               int32_t* __restrict__ pos, uint8_t* __restrict__ drop, const int32_t* __restrict__ counts,
+               const int32_t* __restrict__ offsets, int32_t* __restrict__ row_token,
+               float* __restrict__ row_gate, XT* __restrict__ xe, XT* __restrict__ zero_out) {
+    const int lane = threadIdx.x & 31;
+    const int64_t a = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (a >= T * k) return;
+    const int64_t t = a / k;
+    const int r = (int)(a - t * k);
+    int row = -1;
+    if (lane == 0) {
+        const int e = idx[a];
+        int p = pos[a];
+        if (r == 1) p += counts[e];          // every rank-0 claim precedes rank-1 claims
+        const bool keep = p < C;
+        pos[a] = p;
+        drop[a] = keep ? 0 : 1;
+        if (keep) {
+            row = offsets[e] + p;
+            row_token[row] = (int32_t)t;
+            row_gate[row] = gate[a];
+        }
+    }
+    row = __shfl_sync(0xffffffffu, row, 0);
+    const size_t bytes = (size_t)d * sizeof(XT);
+    if (row >= 0) {
+        if (xe == nullptr) return;
+        const char* src = reinterpret_cast<const char*>(x + t * (int64_t)d);
+        char* dst = reinterpret_cast<char*>(xe + (int64_t)row * d);
+        if (bytes % 16 == 0) {
+            for (size_t o = (size_t)lane * 16; o < bytes; o += 32 * 16)
+                *reinterpret_cast<uint4*>(dst + o) = __ldg(reinterpret_cast<const uint4*>(src + o));
+        } else {
+            for (int j = lane; j < d; j += 32) xe[(int64_t)row * d + j] = x[t * (int64_t)d + j];
+        }
+    } else if (zero_out != nullptr) {
+        char* dst = reinterpret_cast<char*>(zero_out + t * (int64_t)d);
+        if (bytes % 16 == 0) {
+            for (size_t o = (size_t)lane * 16; o < bytes; o += 32 * 16)
+                *reinterpret_cast<uint4*>(dst + o) = make_uint4(0, 0, 0, 0);
+        } else {
+            for (int j = lane; j < d; j += 32) zero_out[t * (int64_t)d + j] = XT(0.f);
+        }
+    }
+}
+
+// Test hook: one block whose predecessor (block 0) never publishes.
+__global__ void lookback_probe_kernel(uint32_t* state, WsHeader* hdr, long long limit_ns) {
+    if (threadIdx.x < 4) lookback(state, 1, threadIdx.x, 4, 1u, limit_ns, &hdr->status);
+}
+
+}  // namespace
+
+int scan_blocks(int64_t T) { return (int)((T + kScanTokens - 1) / kScanTokens); }
+
+cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
+    const int nblk = scan_blocks(a.T);
+    if (nblk == 0) return cudaSuccess;
+    // fresh tickets and look-back flags for this call
+    cudaError_t err = cudaMemsetAsync(&a.hdr->scan_ticket, 0, 2 * sizeof(int32_t), s);
+    if (err != cudaSuccess) return err;
+    err = cudaMemsetAsync(a.scan_state, 0, sizeof(uint32_t) * (size_t)nblk * a.k * a.N, s);
+    if (err != cudaSuccess) return err;
+    scan_kernel<<<nblk, kScanThreads, 0, s>>>(a.idx, a.T, a.N, a.k, a.C, nblk, a.pos, a.counts, a.kept,
+                                             a.offsets, a.scan_state, a.hdr, kWaitLimitNs);
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    const int64_t warps = a.T * a.k;
+    const unsigned grid = (unsigned)((warps + 7) / 8);
+    if (a.dtype == MOE_BF16) {
+        scatter_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
+            reinterpret_cast<const __nv_bfloat16*>(a.x), a.idx, a.gate, a.T, a.d, a.N, a.k, a.C, a.pos,
+            a.drop, a.counts, a.offsets, a.row_token, a.row_gate, reinterpret_cast<__nv_bfloat16*>(a.xe),
+            reinterpret_cast<__nv_bfloat16*>(a.zero_out));
+    } else {
+        scatter_kernel<float><<<grid, 256, 0, s>>>(
+            reinterpret_cast<const float*>(a.x), a.idx, a.gate, a.T, a.d, a.N, a.k, a.C, a.pos, a.drop,
+            a.counts, a.offsets, a.row_token, a.row_gate, reinterpret_cast<float*>(a.xe),
+            reinterpret_cast<float*>(a.zero_out));
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_lookback_timeout_probe(uint32_t* state, WsHeader* hdr, long long limit_ns,
+                                          cudaStream_t s) {
+    cudaError_t err = cudaMemsetAsync(state, 0, 8 * sizeof(uint32_t), s);
+    if (err != cudaSuccess) return err;
+    lookback_probe_kernel<<<1, 32, 0, s>>>(state, hdr, limit_ns);
+    return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,175 @@
+"""ctypes binding of libmoe_b200.so -- argument marshalling only.
+
+Every function has the name and argument order of the C entry point in
+include/moe.h.  Array arguments are torch CUDA tensors (or None for a nullable
+pointer); `stream` defaults to torch's current stream.  Each call returns the
+integer moe_status; ``check`` turns a non-zero status into an exception.
+
+The shared library is loaded on first use.  If it is missing the binding raises
+(there is no fallback implementation); build it with
+``python -m mixture_experts_sparse_b200.build``.
+"""
+import ctypes
+import os
+
+MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_ERR_CUDA, MOE_ERR_TIMEOUT = range(6)
+MOE_F32, MOE_BF16 = 0, 1
+MOE_RELU, MOE_SWIGLU = 0, 1
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200.so")
+
+
+class MoeConfig(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int32), ("d_model", ctypes.c_int32), ("d_ff", ctypes.c_int32),
+                ("n_experts", ctypes.c_int32), ("top_k", ctypes.c_int32), ("capacity", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("act", ctypes.c_int32), ("alpha", ctypes.c_float)]
+
+
+class MoeError(RuntimeError):
+    def __init__(self, status):
+        self.status = status
+        super().__init__(f"moe status {status}: {moe_status_string(status)}")
+
+
+_lib = None
+_P = ctypes.c_void_p
+_SIGS = {
+    "moe_capacity": ([ctypes.c_int64, ctypes.c_int32, ctypes.c_int32, ctypes.c_double], ctypes.c_int32),
+    "moe_workspace_bytes": ([ctypes.POINTER(MoeConfig)], ctypes.c_size_t),
+    "moe_status_string": ([ctypes.c_int32], ctypes.c_char_p),
+    "moe_workspace_init": ([_P, ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_route": ([ctypes.POINTER(MoeConfig)] + [_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_dispatch": ([ctypes.POINTER(MoeConfig)] + [_P] * 12 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_expert_ffn": ([ctypes.POINTER(MoeConfig)] + [_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_combine": ([ctypes.POINTER(MoeConfig)] + [_P] * 8, ctypes.c_int32),
+    "moe_forward": ([ctypes.POINTER(MoeConfig)] + [_P] * 21 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_forward_events": ([ctypes.POINTER(MoeConfig)] + [_P] * 21 + [ctypes.c_size_t, _P, _P], ctypes.c_int32),
+    "moe_read_device_status": ([_P, _P], ctypes.c_int32),
+    "moe_test_lookback_timeout": ([_P, ctypes.c_size_t, ctypes.c_int64, _P], ctypes.c_int32),
+}
+
+
+def lib():
+    """Load the library (raises OSError if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise OSError(f"{LIB_PATH} is missing: build it with python -m mixture_experts_sparse_b200.build")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            fn = getattr(handle, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = handle
+    return _lib
+
+
+def config(T, d_model, d_ff, n_experts, top_k, capacity, dtype="bf16", act="relu", alpha=1e-2):
+    return MoeConfig(int(T), int(d_model), int(d_ff), int(n_experts), int(top_k), int(capacity),
+                     MOE_BF16 if dtype in ("bf16", MOE_BF16) else MOE_F32,
+                     MOE_SWIGLU if act in ("swiglu", MOE_SWIGLU) else MOE_RELU, float(alpha))
+
+
+def _p(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return ctypes.c_void_p(t)
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _s(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _nbytes(ws):
+    return ws.numel() * ws.element_size()
+
+
+def check(status):
+    if status != MOE_OK:
+        raise MoeError(status)
+    return status
+
+
+def moe_capacity(T, n_experts, top_k, capacity_factor):
+    return int(lib().moe_capacity(int(T), int(n_experts), int(top_k), float(capacity_factor)))
+
+
+def moe_workspace_bytes(cfg):
+    return int(lib().moe_workspace_bytes(ctypes.byref(cfg)))
+
+
+def moe_workspace_init(ws, stream=None):
+    return lib().moe_workspace_init(_p(ws), _nbytes(ws), _s(stream))
+
+
+def new_workspace(cfg, device="cuda", stream=None):
+    """Allocate (torch) and initialise a workspace for `cfg`."""
+    import torch
+    nbytes = moe_workspace_bytes(cfg)
+    if nbytes == 0:
+        raise ValueError("invalid layer configuration")
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    check(moe_workspace_init(ws, stream))
+    return ws
+
+
+def moe_status_string(status):
+    return lib().moe_status_string(int(status)).decode()
+
+
+def moe_route(cfg, x, w_r, b_r, idx, gate, probs, f, P, aux, ws, stream=None):
+    return lib().moe_route(ctypes.byref(cfg), _p(x), _p(w_r), _p(b_r), _p(idx), _p(gate), _p(probs),
+                           _p(f), _p(P), _p(aux), _p(ws), _nbytes(ws), _s(stream))
+
+
+def moe_dispatch(cfg, x, idx, gate, pos, drop, counts, kept, offsets, row_token, row_gate, xe, ws,
+                 stream=None):
+    return lib().moe_dispatch(ctypes.byref(cfg), _p(x), _p(idx), _p(gate), _p(pos), _p(drop), _p(counts),
+                              _p(kept), _p(offsets), _p(row_token), _p(row_gate), _p(xe), _p(ws),
+                              _nbytes(ws), _s(stream))
+
+
+def moe_expert_ffn(cfg, xe, offsets, w1, b1, w3, b3, w2, b2, ye, ws, stream=None):
+    return lib().moe_expert_ffn(ctypes.byref(cfg), _p(xe), _p(offsets), _p(w1), _p(b1), _p(w3), _p(b3),
+                                _p(w2), _p(b2), _p(ye), _p(ws), _nbytes(ws), _s(stream))
+
+
+def moe_combine(cfg, ye, idx, pos, drop, gate, offsets, out, stream=None):
+    return lib().moe_combine(ctypes.byref(cfg), _p(ye), _p(idx), _p(pos), _p(drop), _p(gate), _p(offsets),
+                             _p(out), _s(stream))
+
+
+def moe_forward(cfg, x, w_r, b_r, w1, b1, w3, b3, w2, b2, out, idx=None, gate=None, pos=None, drop=None,
+                counts=None, kept=None, offsets=None, f=None, P=None, aux=None, ws=None, stream=None):
+    return lib().moe_forward(ctypes.byref(cfg), _p(x), _p(w_r), _p(b_r), _p(w1), _p(b1), _p(w3), _p(b3),
+                             _p(w2), _p(b2), _p(out), _p(idx), _p(gate), _p(pos), _p(drop), _p(counts),
+                             _p(kept), _p(offsets), _p(f), _p(P), _p(aux), _p(ws), _nbytes(ws), _s(stream))
+
+
+def moe_forward_events(cfg, x, w_r, b_r, w1, b1, w3, b3, w2, b2, out, idx=None, gate=None, pos=None,
+                       drop=None, counts=None, kept=None, offsets=None, f=None, P=None, aux=None, ws=None,
+                       stream=None, events=None):
+    """events: a sequence of 6 raw cudaEvent_t handles (int or ctypes.c_void_p; entries may be None)."""
+    arr = None
+    if events is not None:
+        arr = (ctypes.c_void_p * 6)(*[None if e is None else (e.value if isinstance(e, ctypes.c_void_p) else e)
+                                      for e in events])
+    return lib().moe_forward_events(ctypes.byref(cfg), _p(x), _p(w_r), _p(b_r), _p(w1), _p(b1), _p(w3), _p(b3),
+                                    _p(w2), _p(b2), _p(out), _p(idx), _p(gate), _p(pos), _p(drop), _p(counts),
+                                    _p(kept), _p(offsets), _p(f), _p(P), _p(aux), _p(ws), _nbytes(ws),
+                                    _s(stream), arr)
+
+
+def moe_read_device_status(ws, stream=None):
+    return lib().moe_read_device_status(_p(ws), _s(stream))
+
+
+def moe_test_lookback_timeout(ws, limit_ns, stream=None):
+    return lib().moe_test_lookback_timeout(_p(ws), _nbytes(ws), int(limit_ns), _s(stream))

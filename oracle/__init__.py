@@ -34,6 +34,8 @@ def _load():
         sz = ctypes.c_size_t
         lib.oracle_float_to_bf16_bits.argtypes = [ctypes.c_float]
         lib.oracle_float_to_bf16_bits.restype = ctypes.c_uint16
+        lib.oracle_float_to_bf16_array.argtypes = [P, P, i64]
+        lib.oracle_float_to_bf16_array.restype = None
         lib.oracle_bf16_round.argtypes = [ctypes.c_float]
         lib.oracle_bf16_round.restype = ctypes.c_float
         lib.oracle_router.argtypes = [i64, i32, i32, i32, P, i32, P, P, P, P, P, P]
@@ -76,11 +78,9 @@ def _as_input(a):
 def bf16_bits(v):
     """fp32 -> bf16 bit pattern, round to nearest even (format definition)."""
     lib = _load()
-    v = np.asarray(v, dtype=np.float32)
+    v = np.ascontiguousarray(np.asarray(v, dtype=np.float32))
     out = np.empty(v.shape, dtype=np.uint16)
-    flat_in, flat_out = v.reshape(-1), out.reshape(-1)
-    for i in range(flat_in.size):
-        flat_out[i] = lib.oracle_float_to_bf16_bits(float(flat_in[i]))
+    lib.oracle_float_to_bf16_array(_ptr(v), _ptr(out), v.size)
     return out
 
 

@@ -78,6 +78,10 @@ uint16_t oracle_float_to_bf16_bits(float f) {
     return (uint16_t)upper;
 }
 
+void oracle_float_to_bf16_array(const float* in, uint16_t* out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_float_to_bf16_bits(in[i]);
+}
+
 float oracle_bf16_round(float f) {
     return bf16_bits_to_float(oracle_float_to_bf16_bits(f));
 }
