@@ -104,6 +104,45 @@ class RawEvents:
 
 # ------------------------------------------------------------------ clocks ----
 
+class SmiSampler:
+    """Fallback: nvidia-smi's own sampling loop (the profiling recipe's clocks line)."""
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        import subprocess
+        import tempfile
+        import torch
+        props = torch.cuda.get_device_properties(device_index)
+        self.bus = ("%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)).lower()
+        self.tmp = tempfile.NamedTemporaryFile(mode="w+", suffix=".csv", delete=False)
+        self.proc = subprocess.Popen(["nvidia-smi", "--id=" + self.bus, "--query-gpu=" + self.FIELDS,
+                                      "--format=csv,noheader,nounits", "-lms", "50"],
+                                     stdout=self.tmp, stderr=subprocess.DEVNULL)
+
+    def stop(self):
+        self.proc.terminate()
+        self.proc.wait()
+        self.tmp.seek(0)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.tmp.read().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 6:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[2:]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        os.unlink(self.tmp.name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm), "source": "nvidia-smi -lms 50"}
+
+
 class ClockSampler:
     """Samples SM clock and clock-event reasons through NVML while running."""
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
@@ -126,8 +165,15 @@ class ClockSampler:
             self.nv = pynvml
             self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
             self.ok = True
-        except Exception:
+        except Exception as exc:   # noqa: BLE001
             self.ok = False
+            self.error = repr(exc)
+        self.smi = None
+        if not self.ok:
+            try:
+                self.smi = SmiSampler(device_index)
+            except Exception as exc:   # noqa: BLE001
+                self.error = getattr(self, "error", "") + " / " + repr(exc)
 
     def _run(self):
         nv = self.nv
@@ -149,14 +195,17 @@ class ClockSampler:
             self._thread.start()
 
     def stop(self):
+        if self.smi is not None:
+            return self.smi.stop()
         if self._thread:
             self._stop.set()
             self._thread.join()
         if not self.ok or not self.samples:
-            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0,
+                    "error": getattr(self, "error", None)}
         names = [n for bit, n in self.REASONS.items() if self.reasons & bit]
         return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz, "reasons": names,
-                "samples": len(self.samples)}
+                "samples": len(self.samples), "source": "NVML, every 2 ms"}
 
 
 # ------------------------------------------------------------- cpu oracle ----
@@ -177,10 +226,14 @@ def oracle_tokens_per_s(L, w, target_s, max_tokens=None):
                        out_dtype=out_dtype)
         return time.perf_counter() - t0
 
-    n = 8
+    # start where every expert has a few slots, so the probe does expert work
+    n = int(min(limit, max(64, -(-16 * w.n_experts // max(1, int(w.top_k * w.capacity_factor))))))
     dt = run(n)
-    while dt < target_s and n < limit:
-        n = int(min(limit, max(2 * n, n * 0.9 * target_s / max(dt, 1e-6))))
+    for _ in range(4):   # a few probes, each aiming slightly past the target
+        if dt >= target_s or n >= limit:
+            break
+        n = int(min(limit, 4 * n, max(2 * n if dt < 0.25 * target_s else n + 1,
+                                      n * 1.15 * target_s / max(dt, 1e-6))))
         dt = run(n)
     return n / dt, n, dt
 
@@ -212,6 +265,8 @@ def run_ours(args, rank, world, local):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
                                 device_id=torch.device("cuda", local))
     w = WORKLOADS[args.workload]
+    if args.tokens:
+        w = w.scaled(T=args.tokens)
     C = nat.moe_capacity(w.T, w.n_experts, w.top_k, w.capacity_factor)
     L = inputs.make_workload(w, seed=w.seed + rank)
     layer = MoeLayer(w.T, w.d_model, w.d_ff, w.n_experts, w.top_k, C, w.dtype, w.act, L, alpha=w.alpha)
@@ -355,6 +410,8 @@ def run_reference(args, rank, world):
     from oracle import capacity
 
     w = WORKLOADS[args.workload]
+    if args.tokens:
+        w = w.scaled(T=args.tokens)
     L = inputs.make_workload(w)
     C = capacity(w.T, w.n_experts, w.top_k, w.capacity_factor)
     # size one step so the whole run stays within a few minutes
@@ -398,6 +455,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=sorted(WORKLOADS), default="switch_base")
+    ap.add_argument("--tokens", type=int, default=None, help="override the workload's T (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--reference-budget-s", type=float, default=150.0)

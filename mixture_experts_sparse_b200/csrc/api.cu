@@ -13,7 +13,7 @@ namespace {
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Layout {
-    size_t hdr, part_cnt, part_psum, scan_state;
+    size_t hdr, part_cnt, part_psum, w_split, scan_state;
     size_t idx, gate, pos, drop, counts, kept, offsets, f, P, aux;
     size_t row_token, row_gate, xe, h, ye;
     size_t total;
@@ -39,9 +39,10 @@ Layout layout_of(const moe_config& c) {
     L.rows = compact_rows(c);
     const size_t R = (size_t)(L.rows > 0 ? L.rows : 1);
     L.hdr = take(sizeof(WsHeader));
-    const size_t nbr = (size_t)router_blocks(c.T, c.n_experts);
+    const size_t nbr = (size_t)router_partial_rows(c.T, c.n_experts);
     L.part_cnt = take(4 * nbr * N);
     L.part_psum = take(4 * nbr * N);
+    L.w_split = take(c.dtype == MOE_BF16 ? 2 * 3 * (size_t)router_tc_padded_experts(c.n_experts) * c.d_model : 0);
     const size_t nbs = (size_t)scan_blocks(c.T);
     L.scan_state = take(4 * (nbs * k * N > 8 ? nbs * k * N : 8));
     L.idx = take(4 * T * k);
@@ -178,6 +179,8 @@ int32_t moe_route(const moe_config* cfg, const void* x, const float* w_r, const 
     a.P = P;
     a.aux = aux;
     a.alpha = cfg->alpha;
+    a.w_split = at<void>(ws, L.w_split);
+    a.status = &at<WsHeader>(ws, L.hdr)->status;
     return cuda_status(launch_router(a, (cudaStream_t)stream));
 }
 

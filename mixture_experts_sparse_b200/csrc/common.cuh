@@ -61,9 +61,16 @@ struct RouterArgs {
     int32_t* idx; float* gate; float* probs;
     int32_t* part_cnt; float* part_psum;   // [nblk, N]
     double* f; double* P; double* aux; float alpha;
+    void* w_split;                         // bf16 [3, NP, d] scratch (tensor-core router)
+    int32_t* status;
 };
-int router_blocks(int64_t T, int N);
+int router_blocks(int64_t T, int N);               // partial rows the FP32-pipe router writes
+int router_partial_rows(int64_t T, int N);         // partial rows any router path writes
+int router_tc_padded_experts(int N);
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t s);
+cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t s);
+cudaError_t launch_aux_finalize(const int32_t* part_cnt, const float* part_psum, int nblk, int N, int64_t T,
+                                float alpha, double* f, double* P, double* aux, cudaStream_t s);
 
 struct DispatchArgs {
     const void* x; int dtype; const int32_t* idx; const float* gate;

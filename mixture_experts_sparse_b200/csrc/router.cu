@@ -321,9 +321,7 @@ cudaError_t launch_router_t(const RouterArgs& a, cudaStream_t s) {
         err = cudaGetLastError();
         if (err != cudaSuccess) return err;
     }
-    aux_finalize_kernel<<<1, 1024, 0, s>>>(a.part_cnt, a.part_psum, nblk, a.N, a.T, a.alpha, a.f, a.P,
-                                           a.aux);
-    return cudaGetLastError();
+    return launch_aux_finalize(a.part_cnt, a.part_psum, nblk, a.N, a.T, a.alpha, a.f, a.P, a.aux, s);
 }
 
 template <typename XT>
@@ -346,8 +344,22 @@ int router_blocks(int64_t T, int N) {
     return (int)((T + tb - 1) / tb);
 }
 
+int router_partial_rows(int64_t T, int N) {
+    const int tc_rows = (int)((T + 127) / 128);
+    const int simt_rows = router_blocks(T, N);
+    return tc_rows > simt_rows ? tc_rows : simt_rows;
+}
+
+cudaError_t launch_aux_finalize(const int32_t* part_cnt, const float* part_psum, int nblk, int N, int64_t T,
+                                float alpha, double* f, double* P, double* aux, cudaStream_t s) {
+    aux_finalize_kernel<<<1, 1024, 0, s>>>(part_cnt, part_psum, nblk, N, T, alpha, f, P, aux);
+    return cudaGetLastError();
+}
+
+// bf16 activations: the tensor-core router (exact three-way split of W_r);
+// fp32 activations: the FP32-pipe router.
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t s) {
-    if (a.dtype == MOE_BF16) return launch_router_x<__nv_bfloat16>(a, s);
+    if (a.dtype == MOE_BF16) return launch_router_tc(a, s);
     return launch_router_x<float>(a, s);
 }
 

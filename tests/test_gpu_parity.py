@@ -295,3 +295,21 @@ def test_mixtral_literal_capacity():
     res = oracle_layer(L, w.top_k, C, w.act, w.dtype, w.alpha, tokens=tokens)
     compare_routing(layer, res)
     assert_close_out(widen_out(layer.out)[res["tokens"]], res["out_exact"], w.dtype)
+
+
+def test_single_cta_gemm_variant_in_subprocess():
+    # the one-CTA (M=128) grouped GEMM, selected by MOE_B200_GEMM=single at
+    # library load, must match the oracle as well
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = (
+        "import sys; sys.path.insert(0, %r); sys.path.insert(0, %r)\n"
+        "from test_gpu_parity import SMALL, test_forward_small_full_oracle\n"
+        "for case in (SMALL[0], SMALL[1], SMALL[2], SMALL[4], SMALL[8]):\n"
+        "    test_forward_small_full_oracle(case)\n"
+        "print('single ok')\n" % (root, os.path.join(root, "tests")))
+    env = dict(os.environ, MOE_B200_GEMM="single")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and "single ok" in r.stdout, r.stdout[-2000:] + r.stderr[-4000:]
