@@ -179,10 +179,12 @@ int32_t moe_forward_events(const moe_config* cfg, const void* x, const float* w_
                            double* f, double* P, double* aux,
                            void* ws, size_t ws_bytes, void* stream, void* const* events);
 
-/* Synchronise `stream`, then return (and clear) the device status latched in
- * the workspace: MOE_OK, or MOE_ERR_TIMEOUT if a bounded device-side wait gave
- * up during an earlier call on this workspace.  The outputs of such a call are
- * undefined; the CUDA context stays usable. */
+/* Synchronise `stream`, then return the device status latched in the
+ * workspace: MOE_OK, or MOE_ERR_TIMEOUT if a bounded device-side wait gave up
+ * during an earlier call on this workspace.  The outputs of such a call are
+ * undefined; the CUDA context stays usable.  A non-OK status is cleared by the
+ * read, together with the workspace's per-call counters, so the workspace is
+ * ready for the next call. */
 int32_t moe_read_device_status(void* ws, void* stream);
 
 /* Test hook (not part of the layer): launch one block of the dispatch scan's

@@ -181,6 +181,7 @@ int32_t moe_route(const moe_config* cfg, const void* x, const float* w_r, const 
     a.alpha = cfg->alpha;
     a.w_split = at<void>(ws, L.w_split);
     a.status = &at<WsHeader>(ws, L.hdr)->status;
+    a.ticket = &at<WsHeader>(ws, L.hdr)->route_ticket;
     return cuda_status(launch_router(a, (cudaStream_t)stream));
 }
 
@@ -399,8 +400,8 @@ int32_t moe_read_device_status(void* ws, void* stream) {
     if (cudaMemcpyAsync(&host, &hdr->status, sizeof(int32_t), cudaMemcpyDeviceToHost, s) != cudaSuccess)
         return MOE_ERR_CUDA;
     if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
-    if (host != MOE_OK) {
-        if (cudaMemsetAsync(&hdr->status, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+    if (host != MOE_OK) {   // a call gave up: clear the status and the per-call counters
+        if (cudaMemsetAsync(hdr, 0, sizeof(WsHeader), s) != cudaSuccess) return MOE_ERR_CUDA;
         if (cudaStreamSynchronize(s) != cudaSuccess) return MOE_ERR_CUDA;
     }
     return host;

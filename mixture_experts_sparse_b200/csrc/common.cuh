@@ -14,7 +14,7 @@ struct WsHeader {
     int32_t status;        // latched moe_status of device-side failures
     int32_t scan_ticket;   // dynamic block index of the dispatch scan
     int32_t scan_done;     // finished-block counter of the dispatch scan
-    int32_t route_done;    // unused slot kept for alignment
+    int32_t route_ticket;  // finished-CTA counter of the tensor-core router
     int32_t pad[60];
 };
 static_assert(sizeof(WsHeader) == 256, "header size");
@@ -62,6 +62,7 @@ struct RouterArgs {
     int32_t* part_cnt; float* part_psum;   // [nblk, N]
     double* f; double* P; double* aux; float alpha;
     void* w_split;                         // bf16 [3, NP, d] scratch (tensor-core router)
+    int32_t* ticket;                       // finished-CTA counter of the tensor-core router
     int32_t* status;
 };
 int router_blocks(int64_t T, int N);               // partial rows the FP32-pipe router writes

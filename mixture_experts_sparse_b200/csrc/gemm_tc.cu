@@ -327,6 +327,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
             const __nv_bfloat16* bias_e = p.bias ? p.bias + (int64_t)ti.e * p.n_dim : nullptr;
             const __nv_bfloat16* bias3_e = p.bias3 ? p.bias3 + (int64_t)ti.e * p.n_dim : nullptr;
+            // destination row pointer of the row this lane stores in step k4 (rows
+            // 4*k4 + lane/8 of the warp), or null when that row is not valid
+            __nv_bfloat16* dst_row[8];
+#pragma unroll
+            for (int k4 = 0; k4 < 8; ++k4) {
+                const int r = 4 * k4 + (lane >> 3);
+                const bool rv = __shfl_sync(0xffffffffu, valid, r);
+                const long long ro = __shfl_sync(0xffffffffu, (long long)orow, r);
+                dst_row[k4] = rv ? p.out + ro * (int64_t)p.out_ld : nullptr;
+            }
 #pragma unroll 1
             for (int c = 0; c < BN_OUT / CW; ++c) {
                 const int col0 = ti.n0 + c * CW;
@@ -395,22 +405,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 #pragma unroll
                 for (int k4 = 0; k4 < 8; ++k4) {   // rows 4*k4 .. 4*k4+3 of the warp
                     const int r = 4 * k4 + (lane >> 3);
-                    const bool rv = __shfl_sync(0xffffffffu, valid, r);
-                    const long long ro = __shfl_sync(0xffffffffu, (long long)orow, r);
                     uint4 val;
                     const uint32_t srcp = ebuf + r * 128 + ((gi ^ (r & 7)) << 4);
                     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
                                  : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
                                  : "r"(srcp)
                                  : "memory");
-                    if (rv && col_ok)
-                        *reinterpret_cast<uint4*>(p.out + ro * (int64_t)p.out_ld + col0 + 8 * gi) = val;
+                    if (dst_row[k4] != nullptr && col_ok)
+                        *reinterpret_cast<uint4*>(dst_row[k4] + col0 + 8 * gi) = val;
                 }
                 __syncwarp();
             }
             tc_fence_before();
-            if (PAIR) mbar_arrive_cluster(acc ? tempty_leader1 : tempty_leader0);
-            else mbar_arrive(smem_u32(&tempty_bar[acc]));
+            if (PAIR) mbar_arrive_cluster_relaxed(acc ? tempty_leader1 : tempty_leader0);
+            else mbar_arrive_relaxed(smem_u32(&tempty_bar[acc]));
         }
     }
 
@@ -428,7 +436,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
 struct DeviceInfo {
     int sms = 0;
-    bool attr_set[2][4] = {{false, false, false, false}, {false, false, false, false}};
+    bool attr_set[2][4] = {};
 };
 std::mutex g_mu;
 DeviceInfo g_dev[64];
@@ -456,10 +464,10 @@ cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorM
         }
         sms = di.sms;
     }
-    if (!PAIR) {
+    if constexpr (!PAIR) {
         grouped_gemm_kernel<EPI, false><<<sms, GEMM_THREADS, S::SMEM_BYTES, s>>>(a, b, b3, p);
         return cudaGetLastError();
-    }
+    } else {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(sms / 2) * 2, 1, 1);
     cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
@@ -472,7 +480,8 @@ cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorM
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<EPI, PAIR>, a, b, b3, p);
+    return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<EPI, true>, a, b, b3, p);
+    }
 }
 
 // Variant choice: the CTA-pair kernel unless MOE_B200_GEMM=single (kept for
@@ -526,13 +535,15 @@ bool tc::make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t
     return r == CUDA_SUCCESS;
 }
 
-// Stage 1 + stage 2 of the bf16 expert FFN on the tensor cores.
+// Stage 1 + stage 2 of the bf16 expert FFN on the tensor cores: stage 1 on
+// one-CTA tiles (its short K makes the pair's larger tiles no faster), stage 2
+// on CTA pairs unless MOE_B200_GEMM=single.
 cudaError_t launch_expert_ffn_tc(const FfnArgs& a, cudaStream_t s) {
     const int64_t R = a.R_cap > 0 ? a.R_cap : 1;
     const bool pair = use_pair();
     const bool swiglu = a.act == MOE_SWIGLU;
     // B rows per CTA and load: pair -> 128; single -> 256 (ReLU) or 128 + 128 (SwiGLU)
-    const int b1_box = (pair || swiglu) ? BN / 2 : BN;
+    const int b1_box = swiglu ? BN / 2 : BN;
     const int b2_box = pair ? BN / 2 : BN;
     CUtensorMap mA1, mB1, mB3, mA2, mB2;
     if (!make_map_bf16(&mA1, a.xe, R, a.d, BM) || !make_map_bf16(&mB1, a.w1, (int64_t)a.N * a.d_ff, a.d, b1_box) ||
@@ -554,7 +565,8 @@ cudaError_t launch_expert_ffn_tc(const FfnArgs& a, cudaStream_t s) {
     p1.out = reinterpret_cast<__nv_bfloat16*>(a.h);
     p1.status = &a.hdr->status;
     p1.limit_ns = kWaitLimitNs;
-    cudaError_t err = swiglu ? run_gemm_any<EPI_SWIGLU>(mA1, mB1, mB3, p1, s) : run_gemm_any<EPI_RELU>(mA1, mB1, mB3, p1, s);
+    cudaError_t err = swiglu ? run_gemm<EPI_SWIGLU, false>(mA1, mB1, mB3, p1, s)
+                             : run_gemm<EPI_RELU, false>(mA1, mB1, mB3, p1, s);
     if (err != cudaSuccess) return err;
     if (a.mid_event && (err = cudaEventRecord((cudaEvent_t)a.mid_event, s)) != cudaSuccess) return err;
 

@@ -278,10 +278,23 @@ aux_finalize_kernel(const int32_t* __restrict__ part_cnt, const float* __restric
     const int tpe = 1024 / npow;
     const int tid = threadIdx.x, e = tid % npow, j = tid / npow;
     double a = 0.0, c = 0.0;
-    if (e < N) {
-        for (int b = j; b < nblk; b += tpe) {
-            a += (double)part_psum[(int64_t)b * N + e];
-            c += (double)part_cnt[(int64_t)b * N + e];
+    if (e < N) {   // blocks j, j + tpe, ... in order, 8 independent loads in flight
+        for (int b0 = j; b0 < nblk; b0 += 8 * tpe) {
+            float pv[8];
+            int cv[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int b = b0 + u * tpe;
+                pv[u] = b < nblk ? part_psum[(int64_t)b * N + e] : 0.f;
+                cv[u] = b < nblk ? part_cnt[(int64_t)b * N + e] : 0;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (b0 + u * tpe < nblk) {
+                    a += (double)pv[u];
+                    c += (double)cv[u];
+                }
+            }
         }
     }
     sp[tid] = a;
@@ -345,7 +358,7 @@ int router_blocks(int64_t T, int N) {
 }
 
 int router_partial_rows(int64_t T, int N) {
-    const int tc_rows = (int)((T + 127) / 128);
+    const int tc_rows = (int)((T + 127) / 128);   // >= the tensor-core router's grid
     const int simt_rows = router_blocks(T, N);
     return tc_rows > simt_rows ? tc_rows : simt_rows;
 }

@@ -14,11 +14,13 @@
 // and the tensor core accumulates them in fp32, so
 //   h = sum_j x_j w0_j + sum_j x_j w1_j + sum_j x_j w2_j
 // is the fp32 dot product up to accumulation rounding -- three bf16 MMAs per
-// K step.  The tensor core's fp32 accumulation truncates, so its error grows
-// with the number of MMAs summed into one accumulator; the K loop is therefore
-// cut into G groups of at most 8 k-blocks (<= 96 MMAs), each accumulating into
-// its own TMEM column block, and the epilogue adds the G partial logits in fp32
-// with round-to-nearest in a fixed order.  The router then costs about one read
+// K step.  With 3 NP <= 256 the three parts are adjacent rows of one B tile, so
+// a single MMA of N = 3 NP produces the three partial logits side by side in
+// TMEM (the epilogue adds them in fp32).  The tensor core's fp32 accumulation
+// truncates, so its error grows with the number of MMAs summed into one
+// accumulator; the K loop is therefore cut into G groups of at most 64 MMAs per
+// accumulator, each group in its own TMEM column block, and the epilogue adds
+// the partial logits in fp32 with round-to-nearest in a fixed order.  The router then costs about one read
 // of x from HBM instead of 2 d N FP32-pipe FLOPs per token.
 //
 // Kernel: persistent, 192 threads: warp 0 TMA producer (x tile 128 x 64 and
@@ -44,13 +46,21 @@ struct RtShape {
     static constexpr int A_BYTES = RT_BM * RT_BK * 2;
     static constexpr int P_BYTES = NP * RT_BK * 2;             // one W part
     static constexpr int STAGE_BYTES = A_BYTES + 3 * P_BYTES;
-    static constexpr int STAGES = NP <= 64 ? 4 : 3;
-    static constexpr int RED_FLOATS = 4 * 32 * 33;              // per-warp transpose buffers
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + RED_FLOATS * 4;
-    static constexpr int TMEM_COLS = 512;                      // 2 buffers x G groups x NP columns
-    static constexpr int MAX_GROUPS = TMEM_COLS / (2 * NP);
+    static constexpr int STAGES = NP <= 64 ? 4 : 2;
+    // per epilogue thread, a row of running sums of p over its tokens (padded
+    // by one float so the rows of a warp fall in different banks)
+    static constexpr int ACC_STRIDE = NP + 1;
+    static constexpr int ACC_BYTES = 4 * 32 * ACC_STRIDE * 4;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + ACC_BYTES;
+    // merged: one MMA of N = 3 NP covers the three W parts (adjacent in shared
+    // memory) and leaves three partial-logit blocks side by side in TMEM
+    static constexpr bool MERGED = 3 * NP <= 256;
+    static constexpr int ACC_COLS = MERGED ? 3 * NP : NP;      // TMEM columns per K-group accumulator
+    static constexpr int TMEM_COLS = 512;                      // 2 buffers x G groups x ACC_COLS
+    static constexpr int MAX_GROUPS = TMEM_COLS / (2 * ACC_COLS);
+    static constexpr int MMA_PER_KB = MERGED ? RT_BK / 16 : 3 * (RT_BK / 16);
+    static constexpr int KB_PER_GROUP = 64 / MMA_PER_KB;       // <= 64 MMAs per accumulator
 };
-constexpr int RT_KB_PER_GROUP = 8;
 
 struct RtParams {
     int64_t T;
@@ -61,8 +71,13 @@ struct RtParams {
     int32_t* idx;
     float* gate;
     float* probs;
-    int32_t* part_cnt;
-    float* part_psum;
+    int32_t* part_cnt;    // [gridDim.x, N] per-CTA top-1 counts
+    float* part_psum;     // [gridDim.x, N] per-CTA sums of p
+    double* f;            // outputs of the aux loss (nullable)
+    double* P;
+    double* aux;
+    float alpha;
+    int32_t* ticket;      // finished-CTA counter, 0 between calls
     int32_t* status;
     long long limit_ns;
 };
@@ -78,10 +93,10 @@ template <int NP>
 __global__ void __launch_bounds__(RT_THREADS, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, const RtParams p) {
     using S = RtShape<NP>;
-    constexpr uint32_t IDESC = idesc_bf16_f32(RT_BM, NP);
+    constexpr uint32_t IDESC = idesc_bf16_f32(RT_BM, S::ACC_COLS);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    float* red = reinterpret_cast<float*>(smem + S::STAGES * S::STAGE_BYTES);
+    float* pacc = reinterpret_cast<float*>(smem + S::STAGES * S::STAGE_BYTES);   // [4][32][NP + 1]
     __shared__ __align__(8) uint64_t full_bar[S::STAGES];
     __shared__ __align__(8) uint64_t empty_bar[S::STAGES];
     __shared__ __align__(8) uint64_t tfull_bar[2];
@@ -89,9 +104,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     __shared__ __align__(8) uint64_t done_bar;
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
-    __shared__ float s_wpart[4][NP];
     __shared__ int s_hist[NP];
-    __shared__ int s_ok[2][4];
+    __shared__ int s_last;
+    __shared__ double s_fp[NP];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
@@ -108,6 +123,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         mbar_fence_init();
     }
     for (int e = tid; e < NP; e += RT_THREADS) s_hist[e] = 0;
+    for (int i = tid; i < 4 * 32 * S::ACC_STRIDE; i += RT_THREADS) pacc[i] = 0.f;
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmX);
         prefetch_tmap(&tmW);
@@ -159,6 +175,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             uint32_t phase = 0;
             int it = 0;
             bool ok = true, issued = false;
+            const uint64_t desc0 = umma_desc(smem_u32(smem));
             for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
                 const int acc = it & 1;
                 const uint32_t acc_par = (uint32_t)((it >> 1) & 1);
@@ -167,21 +184,25 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 for (int kb = 0; kb < nkb; ++kb) {
                     const int g = kb / p.kb_per_group;
                     const bool first = kb == g * p.kb_per_group;
-                    const uint32_t d_tmem = tmem_base + (uint32_t)((acc * p.groups + g) * NP);
+                    const uint32_t d_tmem = tmem_base + (uint32_t)((acc * p.groups + g) * S::ACC_COLS);
                     if (!wait_bar(smem_u32(&full_bar[stage]), phase, w)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
                     issued = true;
-                    const uint32_t a_addr = smem_u32(smem + stage * S::STAGE_BYTES);
+                    // descriptors advance by (byte offset >> 4) in their address field
+                    const uint64_t a_desc = desc0 + (uint64_t)((stage * S::STAGE_BYTES) >> 4);
+                    const uint64_t b_desc = a_desc + (uint64_t)(S::A_BYTES >> 4);
 #pragma unroll
                     for (int kk = 0; kk < RT_BK / 16; ++kk) {
+                        if constexpr (S::MERGED) {
+                            umma_f16(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, IDESC, (!first || kk != 0) ? 1u : 0u);
+                        } else {
 #pragma unroll
-                        for (int part = 0; part < 3; ++part) {
-                            const uint32_t b_addr = a_addr + S::A_BYTES + part * S::P_BYTES;
-                            umma_f16(d_tmem, umma_desc(a_addr + kk * 32), umma_desc(b_addr + kk * 32), IDESC,
-                                     (!first || (kk | part) != 0) ? 1u : 0u);
+                            for (int part = 0; part < 3; ++part)
+                                umma_f16(d_tmem, a_desc + 2 * kk, b_desc + (uint64_t)((part * S::P_BYTES) >> 4) + 2 * kk,
+                                         IDESC, (!first || (kk | part) != 0) ? 1u : 0u);
                         }
                     }
                     umma_commit(smem_u32(&empty_bar[stage]));
@@ -201,37 +222,41 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     } else {
         // ---------------- epilogue: one thread per token ----------------
         const int q = warp & 3;
-        float* tr = red + q * 32 * 33;   // this warp's 32 x 33 transpose buffer
+        float* prow = pacc + (q * 32 + lane) * S::ACC_STRIDE;   // this thread's running sums
         const int N = p.N, k = p.k;
         int it = 0;
         for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
             const int acc = it & 1;
             const uint32_t acc_par = (uint32_t)((it >> 1) & 1);
-            // all four epilogue warps agree before going on, so that none is left
-            // waiting at the named barriers below if another gave up
-            const bool got = __all_sync(0xffffffffu, wait_bar(smem_u32(&tfull_bar[acc]), acc_par, w));
-            if (lane == 0) s_ok[it & 1][q] = got ? 1 : 0;
-            named_bar(1, 128);
-            if (!(s_ok[it & 1][0] & s_ok[it & 1][1] & s_ok[it & 1][2] & s_ok[it & 1][3])) break;
+            const bool got = wait_bar(smem_u32(&tfull_bar[acc]), acc_par, w);
+            if (!__all_sync(0xffffffffu, got)) break;   // warp-uniform exit on abort
             tc_fence_after();
             const int64_t t = (int64_t)tile * RT_BM + q * 32 + lane;
             const bool valid = t < p.T;
             float v[NP];
 #pragma unroll
             for (int e = 0; e < NP; ++e) v[e] = 0.f;
-            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * p.groups * NP);
-            for (int g = 0; g < p.groups; ++g) {   // partial logits of the K groups, in order
+            const uint32_t tbase =
+                tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * p.groups * S::ACC_COLS);
+            for (int g = 0; g < p.groups; ++g) {   // partial logits of the K groups (and W parts), in order
+                constexpr int CH = NP < 64 ? NP : 64;   // columns per TMEM load
 #pragma unroll
-                for (int c = 0; c < NP / 16; ++c) {
-                    uint32_t r[16];
-                    tmem_ld16(tbase + g * NP + c * 16, r);
-                    tmem_wait_ld();
+                for (int part = 0; part < (S::MERGED ? 3 : 1); ++part) {
 #pragma unroll
-                    for (int j = 0; j < 16; ++j) v[c * 16 + j] += __uint_as_float(r[j]);
+                    for (int c = 0; c < NP / CH; ++c) {
+                        const uint32_t col = tbase + g * S::ACC_COLS + part * NP + c * CH;
+                        uint32_t r[CH];
+                        if (CH == 64) tmem_ld64(col, r);
+                        else if (CH == 32) tmem_ld32(col, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+                        else tmem_ld16(col, *reinterpret_cast<uint32_t(*)[16]>(&r[0]));
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < CH; ++e) v[c * CH + e] += __uint_as_float(r[e]);
+                    }
                 }
             }
             tc_fence_before();
-            mbar_arrive(smem_u32(&tempty_bar[acc]));   // the accumulator is free again
+            mbar_arrive_relaxed(smem_u32(&tempty_bar[acc]));   // the accumulator is free again
 
             float m = -INFINITY;
             int i1 = 0x7fffffff;
@@ -257,7 +282,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 s += ex;
                 v[e] = ex;   // v now holds exp(h - max)
             }
-            const float inv = 1.f / s;
+            const float inv = valid ? 1.f / s : 0.f;
             if (valid) {
                 if (k == 1) {
                     p.idx[t] = i1;
@@ -276,30 +301,63 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 }
                 atomicAdd(&s_hist[i1], 1);
             }
-            // per-tile sums of p over the tile's tokens: lanes (tokens) in order
-            // inside a warp through a 32 x 33 transpose, then warps 0..3
 #pragma unroll
-            for (int c = 0; c < NP / 32 + (NP % 32 ? 1 : 0); ++c) {
+            for (int e = 0; e < NP; ++e) prow[e] += v[e] * inv;   // this thread's tokens, in tile order
+        }
+        // ---- per-CTA partials, then the aux loss by the last CTA to finish ----
+        named_bar(1, 128);
+        const int et = tid - 64;   // 0..127 across the four epilogue warps
+        if (et < N) {
+            float ps = 0.f;   // fixed order: warp quadrant, then lane
+            for (int r = 0; r < 128; r += 8) {
+                float pv[8];
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int e = c * 32 + j;
-                    if (e < NP) tr[lane * 33 + j] = (valid && e < N) ? v[e] * inv : 0.f;
-                }
-                __syncwarp();
-                float a = 0.f;
-                for (int l = 0; l < 32; ++l) a += tr[l * 33 + lane];
-                if (c * 32 + lane < NP) s_wpart[q][c * 32 + lane] = a;
-                __syncwarp();
+                for (int j = 0; j < 8; ++j) pv[j] = pacc[(r + j) * S::ACC_STRIDE + et];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) ps += pv[j];
             }
-            named_bar(1, 128);
-            const int et = tid - 64;   // 0..127 across the four epilogue warps
+            p.part_psum[(int64_t)blockIdx.x * N + et] = ps;
+            p.part_cnt[(int64_t)blockIdx.x * N + et] = s_hist[et];
+            __threadfence();
+        }
+        named_bar(1, 128);
+        if (et == 0) s_last = (atomicAdd(p.ticket, 1) == (int)gridDim.x - 1);
+        named_bar(1, 128);
+        if (s_last) {
+            __threadfence();
             if (et < N) {
-                const float ps = ((s_wpart[0][et] + s_wpart[1][et]) + s_wpart[2][et]) + s_wpart[3][et];
-                p.part_psum[(int64_t)tile * N + et] = ps;
-                p.part_cnt[(int64_t)tile * N + et] = s_hist[et];
-                s_hist[et] = 0;
+                // CTAs in order; 16 independent loads in flight per step
+                double pa = 0.0, ca = 0.0;
+                const int G = (int)gridDim.x;
+                for (int b0 = 0; b0 < G; b0 += 16) {
+                    float pv[16];
+                    int cv[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int b = b0 + j < G ? b0 + j : G - 1;
+                        pv[j] = __ldcg(p.part_psum + (int64_t)b * N + et);
+                        cv[j] = __ldcg(p.part_cnt + (int64_t)b * N + et);
+                    }
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        if (b0 + j < G) {
+                            pa += (double)pv[j];
+                            ca += (double)cv[j];
+                        }
+                    }
+                }
+                const double Pe = pa / (double)p.T, fe = ca / (double)p.T;
+                if (p.P) p.P[et] = Pe;
+                if (p.f) p.f[et] = fe;
+                s_fp[et] = fe * Pe;
             }
             named_bar(1, 128);
+            if (et == 0) {
+                double sfp = 0.0;
+                for (int e = 0; e < N; ++e) sfp += s_fp[e];
+                if (p.aux) *p.aux = (double)p.alpha * (double)N * sfp;
+                *p.ticket = 0;   // ready for the next call
+            }
         }
     }
 
@@ -342,7 +400,7 @@ cudaError_t run_router_tc(const RouterArgs& a, cudaStream_t s, int sms) {
         return cudaErrorInvalidValue;
     RtParams p{};
     const int nkb = (a.d + RT_BK - 1) / RT_BK;
-    int groups = (nkb + RT_KB_PER_GROUP - 1) / RT_KB_PER_GROUP;
+    int groups = (nkb + S::KB_PER_GROUP - 1) / S::KB_PER_GROUP;
     if (groups > S::MAX_GROUPS) groups = S::MAX_GROUPS;
     p.T = a.T;
     p.N = a.N;
@@ -359,6 +417,11 @@ cudaError_t run_router_tc(const RouterArgs& a, cudaStream_t s, int sms) {
     p.probs = a.probs;
     p.part_cnt = a.part_cnt;
     p.part_psum = a.part_psum;
+    p.f = a.f;
+    p.P = a.P;
+    p.aux = a.aux;
+    p.alpha = a.alpha;
+    p.ticket = a.ticket;
     p.status = a.status;
     p.limit_ns = kWaitLimitNs;
     auto kern = router_tc_kernel<NP>;
@@ -379,16 +442,13 @@ cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t s) {
     cudaError_t err = cudaGetDevice(&dev);
     if (err == cudaSuccess) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (err != cudaSuccess) return err;
-    if (a.T > 0) {
-        const int np = router_tc_padded_experts(a.N);
-        if (np == 16) err = run_router_tc<16>(a, s, sms);
-        else if (np == 32) err = run_router_tc<32>(a, s, sms);
-        else if (np == 64) err = run_router_tc<64>(a, s, sms);
-        else err = run_router_tc<128>(a, s, sms);
-        if (err != cudaSuccess) return err;
-    }
-    return launch_aux_finalize(a.part_cnt, a.part_psum, (int)((a.T + RT_BM - 1) / RT_BM), a.N, a.T, a.alpha, a.f,
-                               a.P, a.aux, s);
+    if (a.T == 0)   // no tokens: f, P and the aux loss are zero
+        return launch_aux_finalize(a.part_cnt, a.part_psum, 0, a.N, a.T, a.alpha, a.f, a.P, a.aux, s);
+    const int np = router_tc_padded_experts(a.N);
+    if (np == 16) return run_router_tc<16>(a, s, sms);
+    if (np == 32) return run_router_tc<32>(a, s, sms);
+    if (np == 64) return run_router_tc<64>(a, s, sms);
+    return run_router_tc<128>(a, s, sms);
 }
 
 }  // namespace moe
