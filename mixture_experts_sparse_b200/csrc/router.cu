@@ -358,7 +358,7 @@ int router_blocks(int64_t T, int N) {
 }
 
 int router_partial_rows(int64_t T, int N) {
-    const int tc_rows = (int)((T + 127) / 128);   // >= the tensor-core router's grid
+    const int tc_rows = (int)(((T + 127) / 128 + 3) / 4 * 4);   // >= the tensor-core router's grid, rounded to 4
     const int simt_rows = router_blocks(T, N);
     return tc_rows > simt_rows ? tc_rows : simt_rows;
 }

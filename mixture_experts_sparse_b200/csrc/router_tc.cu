@@ -71,8 +71,8 @@ struct RtParams {
     int32_t* idx;
     float* gate;
     float* probs;
-    int32_t* part_cnt;    // [gridDim.x, N] per-CTA top-1 counts
-    float* part_psum;     // [gridDim.x, N] per-CTA sums of p
+    int32_t* part_cnt;    // [N, Gp] per-CTA top-1 counts (Gp = gridDim.x rounded up to 4)
+    float* part_psum;     // [N, Gp] per-CTA sums of p
     double* f;            // outputs of the aux loss (nullable)
     double* P;
     double* aux;
@@ -82,11 +82,45 @@ struct RtParams {
     long long limit_ns;
 };
 
-__device__ __forceinline__ void take_max(float& v, int& i, float ov, int oi) {
-    if (ov > v || (ov == v && oi < i)) {
-        v = ov;
-        i = oi;
-    }
+// Fixed-order tree reductions over a thread's NP values (short dependency
+// chains; a serial chain over NP values is latency-bound with one warp per SM
+// sub-partition).
+// (excl: an index whose value is treated as -inf; -1 for none)
+template <int NP>
+__device__ __forceinline__ float tree_max(const float (&v)[NP], int excl = -1) {
+    float t[NP / 2];
+#pragma unroll
+    for (int j = 0; j < NP / 2; ++j)
+        t[j] = fmaxf(2 * j == excl ? -INFINITY : v[2 * j], 2 * j + 1 == excl ? -INFINITY : v[2 * j + 1]);
+#pragma unroll
+    for (int w = NP / 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int j = 0; j < w; ++j) t[j] = fmaxf(t[j], t[j + w]);
+    return t[0];
+}
+template <int NP>
+__device__ __forceinline__ float tree_sum(const float (&v)[NP]) {
+    float t[NP / 2];
+#pragma unroll
+    for (int j = 0; j < NP / 2; ++j) t[j] = v[2 * j] + v[2 * j + 1];
+#pragma unroll
+    for (int w = NP / 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int j = 0; j < w; ++j) t[j] = t[j] + t[j + w];
+    return t[0];
+}
+// lowest index e with v[e] == m (NP if none)
+template <int NP>
+__device__ __forceinline__ int tree_first(const float (&v)[NP], float m, int excl = -1) {
+    int t[NP / 2];
+#pragma unroll
+    for (int j = 0; j < NP / 2; ++j)
+        t[j] = (v[2 * j] == m && 2 * j != excl) ? 2 * j : ((v[2 * j + 1] == m && 2 * j + 1 != excl) ? 2 * j + 1 : NP);
+#pragma unroll
+    for (int w = NP / 4; w >= 1; w >>= 1)
+#pragma unroll
+        for (int j = 0; j < w; ++j) t[j] = min(t[j], t[j + w]);
+    return t[0];
 }
 
 template <int NP>
@@ -258,30 +292,27 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             tc_fence_before();
             mbar_arrive_relaxed(smem_u32(&tempty_bar[acc]));   // the accumulator is free again
 
-            float m = -INFINITY;
-            int i1 = 0x7fffffff;
-#pragma unroll
-            for (int e = 0; e < NP; ++e) {
-                if (e < N) {
-                    if (p.b_r) v[e] += __ldg(p.b_r + e);
-                    take_max(m, i1, v[e], e);
-                }
-            }
-            // second choice: largest logit among the others (lower index on ties)
-            float m2 = -INFINITY;
-            int i2 = 0x7fffffff;
-            if (k == 2) {
+            if (p.b_r) {
 #pragma unroll
                 for (int e = 0; e < NP; ++e)
-                    if (e < N && e != i1) take_max(m2, i2, v[e], e);
+                    if (e < N) v[e] += __ldg(p.b_r + e);
             }
-            float s = 0.f;
 #pragma unroll
-            for (int e = 0; e < NP; ++e) {
-                float ex = (e < N) ? expf(v[e] - m) : 0.f;
-                s += ex;
-                v[e] = ex;   // v now holds exp(h - max)
+            for (int e = 0; e < NP; ++e)
+                if (e >= N) v[e] = -INFINITY;   // padding experts never win
+            // first choice: the largest logit, lowest index among equals
+            const float m = tree_max(v);
+            const int i1 = tree_first(v, m);
+            // second choice: the largest of the others, lowest index among equals
+            float m2 = -INFINITY;
+            int i2 = 0;
+            if (k == 2) {
+                m2 = tree_max(v, i1);
+                i2 = tree_first(v, m2, i1);
             }
+#pragma unroll
+            for (int e = 0; e < NP; ++e) v[e] = (e < N) ? expf(v[e] - m) : 0.f;   // v now holds exp(h - max)
+            const float s = tree_sum(v);
             const float inv = valid ? 1.f / s : 0.f;
             if (valid) {
                 if (k == 1) {
@@ -304,9 +335,10 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 #pragma unroll
             for (int e = 0; e < NP; ++e) prow[e] += v[e] * inv;   // this thread's tokens, in tile order
         }
-        // ---- per-CTA partials, then the aux loss by the last CTA to finish ----
+        // ---- this CTA's partials, expert-major: part[e][blockIdx.x] ----
         named_bar(1, 128);
         const int et = tid - 64;   // 0..127 across the four epilogue warps
+        const int Gp = ((int)gridDim.x + 3) & ~3;
         if (et < N) {
             float ps = 0.f;   // fixed order: warp quadrant, then lane
             for (int r = 0; r < 128; r += 8) {
@@ -316,48 +348,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 #pragma unroll
                 for (int j = 0; j < 8; ++j) ps += pv[j];
             }
-            p.part_psum[(int64_t)blockIdx.x * N + et] = ps;
-            p.part_cnt[(int64_t)blockIdx.x * N + et] = s_hist[et];
+            p.part_psum[(int64_t)et * Gp + blockIdx.x] = ps;
+            p.part_cnt[(int64_t)et * Gp + blockIdx.x] = s_hist[et];
             __threadfence();
-        }
-        named_bar(1, 128);
-        if (et == 0) s_last = (atomicAdd(p.ticket, 1) == (int)gridDim.x - 1);
-        named_bar(1, 128);
-        if (s_last) {
-            __threadfence();
-            if (et < N) {
-                // CTAs in order; 16 independent loads in flight per step
-                double pa = 0.0, ca = 0.0;
-                const int G = (int)gridDim.x;
-                for (int b0 = 0; b0 < G; b0 += 16) {
-                    float pv[16];
-                    int cv[16];
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const int b = b0 + j < G ? b0 + j : G - 1;
-                        pv[j] = __ldcg(p.part_psum + (int64_t)b * N + et);
-                        cv[j] = __ldcg(p.part_cnt + (int64_t)b * N + et);
-                    }
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        if (b0 + j < G) {
-                            pa += (double)pv[j];
-                            ca += (double)cv[j];
-                        }
-                    }
-                }
-                const double Pe = pa / (double)p.T, fe = ca / (double)p.T;
-                if (p.P) p.P[et] = Pe;
-                if (p.f) p.f[et] = fe;
-                s_fp[et] = fe * Pe;
-            }
-            named_bar(1, 128);
-            if (et == 0) {
-                double sfp = 0.0;
-                for (int e = 0; e < N; ++e) sfp += s_fp[e];
-                if (p.aux) *p.aux = (double)p.alpha * (double)N * sfp;
-                *p.ticket = 0;   // ready for the next call
-            }
         }
     }
 
@@ -365,6 +358,63 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     __syncthreads();
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem_base, S::TMEM_COLS);
+
+    // ---- the last CTA to finish reduces every CTA's partials: f, P, aux ----
+    if (tid == 0) s_last = (atomicAdd(p.ticket, 1) == (int)gridDim.x - 1);
+    __syncthreads();
+    if (!s_last) return;
+    __threadfence();
+    {
+        const int N = p.N, G = (int)gridDim.x, Gp = (G + 3) & ~3, nch = Gp / 4;
+        const int tpe = RT_THREADS / N;   // threads per expert
+        const int e = tid / tpe, j = tid % tpe;
+        double* sp = reinterpret_cast<double*>(smem);   // pipeline buffers are free now
+        double* sc = sp + RT_THREADS;
+        double pa = 0.0, ca = 0.0;
+        if (e < N) {   // this thread: chunks j, j + tpe, ... of 4 CTAs each, in order
+            const float4* ps4 = reinterpret_cast<const float4*>(p.part_psum + (int64_t)e * Gp);
+            const int4* cs4 = reinterpret_cast<const int4*>(p.part_cnt + (int64_t)e * Gp);
+            for (int c0 = j; c0 < nch; c0 += 4 * tpe) {
+                float4 pv[4];
+                int4 cv[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int c = c0 + u * tpe;
+                    pv[u] = c < nch ? __ldcg(ps4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+                    cv[u] = c < nch ? __ldcg(cs4 + c) : make_int4(0, 0, 0, 0);
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int b = 4 * (c0 + u * tpe);   // first CTA of the chunk
+                    if (b + 0 < G) { pa += (double)pv[u].x; ca += (double)cv[u].x; }
+                    if (b + 1 < G) { pa += (double)pv[u].y; ca += (double)cv[u].y; }
+                    if (b + 2 < G) { pa += (double)pv[u].z; ca += (double)cv[u].z; }
+                    if (b + 3 < G) { pa += (double)pv[u].w; ca += (double)cv[u].w; }
+                }
+            }
+        }
+        sp[tid] = pa;
+        sc[tid] = ca;
+        __syncthreads();
+        if (tid < N) {
+            double pt = 0.0, ct = 0.0;
+            for (int q2 = 0; q2 < tpe; ++q2) {
+                pt += sp[tid * tpe + q2];
+                ct += sc[tid * tpe + q2];
+            }
+            const double Pe = pt / (double)p.T, fe = ct / (double)p.T;
+            if (p.P) p.P[tid] = Pe;
+            if (p.f) p.f[tid] = fe;
+            s_fp[tid] = fe * Pe;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            double sfp = 0.0;
+            for (int q2 = 0; q2 < N; ++q2) sfp += s_fp[q2];
+            if (p.aux) *p.aux = (double)p.alpha * (double)N * sfp;
+            *p.ticket = 0;   // ready for the next call
+        }
+    }
 }
 
 // fp32 [N, d] -> bf16 [3, NP, d]: w = w0 + w1 + w2 exactly; rows >= N are zero.
