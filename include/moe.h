@@ -187,6 +187,32 @@ int32_t moe_forward_events(const moe_config* cfg, const void* x, const float* w_
  * ready for the next call. */
 int32_t moe_read_device_status(void* ws, void* stream);
 
+/* moe_dispatch without a workspace, for callers that cannot allocate device
+ * memory when they call the layer: plugin interfaces that give a kernel only
+ * its input and output tensors, and serving runtimes that reserve all device
+ * memory at start-up and allow no cudaMalloc later (it synchronises the device
+ * and can fail once memory is fragmented).  The pages have no counterpart to
+ * this entry point; it computes exactly what moe_dispatch computes, with the
+ * same launches.
+ * Scratch: the dispatch scan's flags and counters live in a fixed-size
+ * __device__ array inside the library (about 256 KB, held on every GPU that
+ * loads the library until the process exits).  Limit: T <= 262144 tokens;
+ * larger T returns MOE_ERR_UNSUPPORTED before anything is launched.  The call
+ * allocates nothing and frees nothing.
+ * The array is shared by every call and keeps the last call's contents (each
+ * call clears what it uses first), so calls whose work can overlap on one GPU
+ * -- different streams, or different host threads on the same device -- race
+ * and must be serialised by the caller.  The first call on each device looks up
+ * the array's device address (cudaGetSymbolAddress) with that device current;
+ * make that first call before any stream capture starts.
+ * Arguments are those of moe_dispatch, without ws/ws_bytes, plus
+ * status: device int32 (nullable) that receives this call's device-side status
+ * (MOE_OK, or MOE_ERR_TIMEOUT if the scan's bounded wait gave up). */
+int32_t moe_dispatch_noalloc(const moe_config* cfg, const void* x, const int32_t* idx, const float* gate,
+                             int32_t* pos, uint8_t* drop, int32_t* counts, int32_t* kept,
+                             int32_t* offsets, int32_t* row_token, float* row_gate, void* xe,
+                             int32_t* status, void* stream);
+
 /* Test hook (not part of the layer): launch one block of the dispatch scan's
  * look-back in isolation, waiting on a predecessor that never publishes, with a
  * wait limit of `limit_ns` nanoseconds.  The wait gives up, latches

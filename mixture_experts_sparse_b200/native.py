@@ -44,6 +44,7 @@ _SIGS = {
     "moe_combine": ([ctypes.POINTER(MoeConfig)] + [_P] * 8, ctypes.c_int32),
     "moe_forward": ([ctypes.POINTER(MoeConfig)] + [_P] * 21 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_forward_events": ([ctypes.POINTER(MoeConfig)] + [_P] * 21 + [ctypes.c_size_t, _P, _P], ctypes.c_int32),
+    "moe_dispatch_noalloc": ([ctypes.POINTER(MoeConfig)] + [_P] * 13, ctypes.c_int32),
     "moe_read_device_status": ([_P, _P], ctypes.c_int32),
     "moe_test_lookback_timeout": ([_P, ctypes.c_size_t, ctypes.c_int64, _P], ctypes.c_int32),
 }
@@ -134,6 +135,13 @@ def moe_dispatch(cfg, x, idx, gate, pos, drop, counts, kept, offsets, row_token,
     return lib().moe_dispatch(ctypes.byref(cfg), _p(x), _p(idx), _p(gate), _p(pos), _p(drop), _p(counts),
                               _p(kept), _p(offsets), _p(row_token), _p(row_gate), _p(xe), _p(ws),
                               _nbytes(ws), _s(stream))
+
+
+def moe_dispatch_noalloc(cfg, x, idx, gate, pos, drop, counts, kept, offsets, row_token, row_gate, xe, status,
+                         stream=None):
+    return lib().moe_dispatch_noalloc(ctypes.byref(cfg), _p(x), _p(idx), _p(gate), _p(pos), _p(drop), _p(counts),
+                                      _p(kept), _p(offsets), _p(row_token), _p(row_gate), _p(xe), _p(status),
+                                      _s(stream))
 
 
 def moe_expert_ffn(cfg, xe, offsets, w1, b1, w3, b3, w2, b2, ye, ws, stream=None):
