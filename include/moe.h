@@ -131,6 +131,51 @@ int32_t moe_dispatch(const moe_config* cfg, const void* x, const int32_t* idx, c
                      int32_t* offsets, int32_t* row_token, float* row_gate, void* xe,
                      void* ws, size_t ws_bytes, void* stream);
 
+/* ---- One routing group split over several shards (one per GPU) ------------
+ * Capacity is defined per routing group, and claims follow token order over the
+ * whole group (CS25 Lecture 05 notes, capacity-aware dispatch).  When a group's
+ * tokens are split into contiguous shards, shard s computes exactly what a
+ * single call over the whole group computes for its tokens if it knows, per
+ * (rank, expert), how many claims come before its own:
+ *   1. moe_route on the shard;  2. moe_expert_counts -> this shard's claims
+ *   counts_s[k][N];  3. every shard gathers all shards' counts into
+ *   [S][k][N] (one small all-gather, the only exchange);  4. moe_claim_base;
+ *   5. moe_dispatch_shard;  then moe_expert_ffn on the shard's own compact
+ *   rows and moe_combine_shard;  6. the aux loss over the group with moe_aux_shards from
+ *   every shard's f, P and token count (one more small all-gather).
+ * Routing integers and outputs are then identical to the single call. */
+
+/* Claims of this shard: counts[r][e] = number of tokens whose rank-r choice is
+ * e (before capacity).  In: idx [T, k].  Out: counts [k, N] int32. */
+int32_t moe_expert_counts(const moe_config* cfg, const int32_t* idx, int32_t* counts, void* stream);
+
+/* Claim base of shard `shard` among n_shards contiguous shards (shard order =
+ * token order).  In: shard_counts [n_shards][top_k][n_experts] int32 (device).
+ * Out: claim_base [top_k][n_experts] int32 (device):
+ *   claim_base[0][e] = rank-0 claims on e by earlier shards,
+ *   claim_base[1][e] = every shard's rank-0 claims on e + rank-1 claims on e
+ *                      by earlier shards. */
+int32_t moe_claim_base(const int32_t* shard_counts, int32_t n_shards, int32_t shard, int32_t top_k,
+                       int32_t n_experts, int32_t* claim_base, void* stream);
+
+/* moe_dispatch for one shard of a routing group: cfg->T is the shard's token
+ * count, cfg->capacity the group's C.  pos are the group-wide claim numbers
+ * (claim_base + the shard's own claim order), drop = pos >= C; counts are the
+ * shard's own claims; kept/offsets/row_token/row_gate/xe describe the shard's
+ * kept assignments, in the order moe_dispatch would give them. */
+int32_t moe_dispatch_shard(const moe_config* cfg, const void* x, const int32_t* idx, const float* gate,
+                           const int32_t* claim_base, int32_t* pos, uint8_t* drop, int32_t* counts,
+                           int32_t* kept, int32_t* offsets, int32_t* row_token, float* row_gate, void* xe,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* Load-balancing loss of a routing group from its shards (GLaM page, Load
+ * balancing): f = sum_s T_s f_s / sum_s T_s, likewise P, aux = alpha N sum f P,
+ * in fp64 in shard order.  In: shard_tokens [S] int64, f_all, P_all [S][N]
+ * fp64 (each shard's moe_route outputs), all device.  Out: f, P [N], aux [1]
+ * fp64 (each nullable). */
+int32_t moe_aux_shards(int32_t n_shards, int32_t n_experts, const int64_t* shard_tokens, const double* f_all,
+                       const double* P_all, float alpha, double* f, double* P, double* aux, void* stream);
+
 /* Grouped expert FFN over the compact rows (rows A5, A6).
  * In:  xe [R, d] (dtype) with R = offsets[N]; offsets [N + 1]; w1, w2 and
  *      (SwiGLU) w3; b1, b3, b2 nullable.
@@ -148,6 +193,18 @@ int32_t moe_expert_ffn(const moe_config* cfg, const void* xe, const int32_t* off
 int32_t moe_combine(const moe_config* cfg, const void* ye, const int32_t* idx,
                     const int32_t* pos, const uint8_t* drop, const float* gate,
                     const int32_t* offsets, void* out, void* stream);
+
+/* moe_combine for one shard of a routing group, after moe_dispatch_shard:
+ * pos are group-wide claim numbers, and the row of a kept claim p on expert e
+ * is offsets[e] + p - claim_base[0][e] for rank 0 and offsets[e] +
+ * kept0[e] + p - claim_base[1][e] for rank 1, kept0[e] = how many of the
+ * shard's rank-0 claims on e fall below C.  In: claim_base [k, N] (from
+ * moe_claim_base) and counts [k, N] (the shard's own, from
+ * moe_dispatch_shard), both required; the rest as moe_combine. */
+int32_t moe_combine_shard(const moe_config* cfg, const void* ye, const int32_t* idx,
+                          const int32_t* pos, const uint8_t* drop, const float* gate,
+                          const int32_t* offsets, const int32_t* claim_base,
+                          const int32_t* counts, void* out, void* stream);
 
 /* The whole layer forward in one call (rows A1-A8), fused where it pays:
  * the top-1 bf16 path scatters gate * E(x) straight from the second GEMM's

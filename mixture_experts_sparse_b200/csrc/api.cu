@@ -4,10 +4,44 @@
 // moe_read_device_status, which synchronises its stream.
 #include <cmath>
 #include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
 
 #include "common.cuh"
 
 namespace moe {
+
+cudaError_t once_per_device(const void* key, cudaError_t (*set)(const void*)) {
+    static std::mutex mu;
+    static std::map<std::pair<int, const void*>, cudaError_t> done;
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = done.find({dev, key});
+    if (it != done.end()) return it->second;
+    err = set(key);
+    done[{dev, key}] = err;
+    return err;
+}
+
+cudaError_t device_sm_count(int* sms) {
+    static std::mutex mu;
+    static int cache[64] = {};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cache[dev] == 0) {
+        err = cudaDeviceGetAttribute(&cache[dev], cudaDevAttrMultiProcessorCount, dev);
+        if (err != cudaSuccess) return err;
+    }
+    *sms = cache[dev];
+    return cudaSuccess;
+}
+
 namespace {
 
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
@@ -188,7 +222,7 @@ int32_t moe_route(const moe_config* cfg, const void* x, const float* w_r, const 
 static int32_t dispatch_impl(const moe_config* cfg, const void* x, const int32_t* idx, const float* gate,
                              int32_t* pos, uint8_t* drop, int32_t* counts, int32_t* kept, int32_t* offsets,
                              int32_t* row_token, float* row_gate, void* xe, void* zero_out, void* ws,
-                             cudaStream_t s) {
+                             cudaStream_t s, const int32_t* claim_base = nullptr) {
     const Layout L = layout_of(*cfg);
     if (cfg->T == 0) {
         cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->top_k * cfg->n_experts, s);
@@ -217,6 +251,7 @@ static int32_t dispatch_impl(const moe_config* cfg, const void* x, const int32_t
     a.zero_out = zero_out;
     a.scan_state = at<uint32_t>(ws, L.scan_state);
     a.hdr = at<WsHeader>(ws, L.hdr);
+    a.claim_base = claim_base;
     return cuda_status(launch_dispatch(a, s));
 }
 
@@ -232,6 +267,48 @@ int32_t moe_dispatch(const moe_config* cfg, const void* x, const int32_t* idx, c
     if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
     return dispatch_impl(cfg, x, idx, gate, pos, drop, counts, kept, offsets, row_token, row_gate, xe, nullptr, ws,
                          (cudaStream_t)stream);
+}
+
+int32_t moe_dispatch_shard(const moe_config* cfg, const void* x, const int32_t* idx, const float* gate,
+                           const int32_t* claim_base, int32_t* pos, uint8_t* drop, int32_t* counts, int32_t* kept,
+                           int32_t* offsets, int32_t* row_token, float* row_gate, void* xe, void* ws,
+                           size_t ws_bytes, void* stream) {
+    int32_t st = validate(cfg);
+    if (st != MOE_OK) return st;
+    if (!req(claim_base) || !req(counts) || !req(kept) || !req(offsets) || !opt(xe) || !opt(x))
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->T > 0 && (!req(idx) || !req(gate) || !req(pos) || !req(drop) || !req(row_token) || !req(row_gate)))
+        return MOE_ERR_INVALID_ARG;
+    if (xe && cfg->T > 0 && !req(x)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+    return dispatch_impl(cfg, x, idx, gate, pos, drop, counts, kept, offsets, row_token, row_gate, xe, nullptr, ws,
+                         (cudaStream_t)stream, claim_base);
+}
+
+int32_t moe_expert_counts(const moe_config* cfg, const int32_t* idx, int32_t* counts, void* stream) {
+    int32_t st = validate(cfg);
+    if (st != MOE_OK) return st;
+    if (!req(counts) || (cfg->T > 0 && !req(idx))) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_counts(idx, cfg->T, cfg->n_experts, cfg->top_k, counts, (cudaStream_t)stream));
+}
+
+int32_t moe_claim_base(const int32_t* shard_counts, int32_t n_shards, int32_t shard, int32_t top_k,
+                       int32_t n_experts, int32_t* claim_base, void* stream) {
+    if (n_shards < 1 || shard < 0 || shard >= n_shards || top_k < 1 || n_experts < 1) return MOE_ERR_INVALID_ARG;
+    if (top_k > 2 || n_experts > 128) return MOE_ERR_UNSUPPORTED;
+    if (!req(shard_counts) || !req(claim_base)) return MOE_ERR_INVALID_ARG;
+    return cuda_status(
+        launch_claim_base(shard_counts, n_shards, shard, top_k, n_experts, claim_base, (cudaStream_t)stream));
+}
+
+int32_t moe_aux_shards(int32_t n_shards, int32_t n_experts, const int64_t* shard_tokens, const double* f_all,
+                       const double* P_all, float alpha, double* f, double* P, double* aux, void* stream) {
+    if (n_shards < 1 || n_experts < 1 || !std::isfinite(alpha)) return MOE_ERR_INVALID_ARG;
+    if (n_experts > 128) return MOE_ERR_UNSUPPORTED;
+    if (!req(shard_tokens) || !req(f_all) || !req(P_all) || !opt(f) || !opt(P) || !opt(aux))
+        return MOE_ERR_INVALID_ARG;
+    return cuda_status(
+        launch_aux_shards(n_shards, n_experts, shard_tokens, f_all, P_all, alpha, f, P, aux, (cudaStream_t)stream));
 }
 
 static int32_t ffn_impl(const moe_config* cfg, const void* xe, const int32_t* offsets, const void* w1,
@@ -282,13 +359,14 @@ int32_t moe_expert_ffn(const moe_config* cfg, const void* xe, const int32_t* off
                     (cudaStream_t)stream);
 }
 
-int32_t moe_combine(const moe_config* cfg, const void* ye, const int32_t* idx, const int32_t* pos,
-                    const uint8_t* drop, const float* gate, const int32_t* offsets, void* out, void* stream) {
+static int32_t combine_impl(const moe_config* cfg, const void* ye, const int32_t* idx, const int32_t* pos,
+                            const uint8_t* drop, const float* gate, const int32_t* offsets,
+                            const int32_t* claim_base, const int32_t* counts, void* out, void* stream) {
     int32_t st = validate(cfg);
     if (st != MOE_OK) return st;
     if (cfg->T > 0 && (!req(idx) || !req(pos) || !req(drop) || !req(gate) || !req(offsets) || !req(out)))
         return MOE_ERR_INVALID_ARG;
-    if (!opt(ye)) return MOE_ERR_INVALID_ARG;
+    if (!opt(ye) || !opt(claim_base) || !opt(counts)) return MOE_ERR_INVALID_ARG;
     if (cfg->T > 0 && compact_rows(*cfg) > 0 && !ye) return MOE_ERR_INVALID_ARG;
     CombineArgs a{};
     a.dtype = cfg->dtype;
@@ -302,7 +380,23 @@ int32_t moe_combine(const moe_config* cfg, const void* ye, const int32_t* idx, c
     a.gate = gate;
     a.offsets = offsets;
     a.out = out;
+    a.claim_base = claim_base;
+    a.counts = counts;
+    a.C = (int)cfg->capacity;
+    a.N = (int)cfg->n_experts;
     return cuda_status(launch_combine(a, (cudaStream_t)stream));
+}
+
+int32_t moe_combine(const moe_config* cfg, const void* ye, const int32_t* idx, const int32_t* pos,
+                    const uint8_t* drop, const float* gate, const int32_t* offsets, void* out, void* stream) {
+    return combine_impl(cfg, ye, idx, pos, drop, gate, offsets, nullptr, nullptr, out, stream);
+}
+
+int32_t moe_combine_shard(const moe_config* cfg, const void* ye, const int32_t* idx, const int32_t* pos,
+                          const uint8_t* drop, const float* gate, const int32_t* offsets,
+                          const int32_t* claim_base, const int32_t* counts, void* out, void* stream) {
+    if (!claim_base || !counts) return MOE_ERR_INVALID_ARG;
+    return combine_impl(cfg, ye, idx, pos, drop, gate, offsets, claim_base, counts, out, stream);
 }
 
 static int32_t forward_impl(const moe_config* cfg, const void* x, const float* w_r, const float* b_r,

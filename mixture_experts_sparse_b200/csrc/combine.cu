@@ -6,6 +6,12 @@
 // for top-1 and y = w1 E_{i1}(x) + w2 E_{i2}(x) for top-2, "Expert Capacity and
 // Token Dropping" (an overflowing token skips the expert FFN).
 // One warp per token, 16-byte vector loads/stores: an HBM-bound gather.
+//
+// For one shard of a routing group pos holds group-wide claim numbers; the
+// shard's rows of expert e hold its kept rank-0 claims (numbers base0[e] ...)
+// and then its kept rank-1 claims (numbers base1[e] ...), so the row of a kept
+// claim p is p - base0[e] (rank 0) or kept0[e] + p - base1[e] (rank 1), kept0
+// being how many of the shard's rank-0 claims on e fall below C.
 #include "common.cuh"
 
 namespace moe {
@@ -15,7 +21,8 @@ template <typename XT>
 __global__ void __launch_bounds__(256)
 combine_kernel(const XT* __restrict__ ye, const int32_t* __restrict__ idx, const int32_t* __restrict__ pos,
                const uint8_t* __restrict__ drop, const float* __restrict__ gate,
-               const int32_t* __restrict__ offsets, int64_t T, int d, int k, XT* __restrict__ out) {
+               const int32_t* __restrict__ offsets, const int32_t* __restrict__ claim_base,
+               const int32_t* __restrict__ counts, int C, int N, int64_t T, int d, int k, XT* __restrict__ out) {
     constexpr int VEC = 16 / sizeof(XT);
     const int lane = threadIdx.x & 31;
     const int64_t t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -25,7 +32,12 @@ combine_kernel(const XT* __restrict__ ye, const int32_t* __restrict__ idx, const
     for (int r = 0; r < k; ++r) {
         const int64_t a = t * k + r;
         if (!drop[a]) {
-            row[r] = (int64_t)offsets[idx[a]] + pos[a];
+            const int e = idx[a];
+            int local = pos[a];
+            if (claim_base)
+                local = r == 0 ? local - claim_base[e]
+                               : kept_after(claim_base[e], counts[e], C) + local - claim_base[N + e];
+            row[r] = (int64_t)offsets[e] + local;
             g[r] = gate[a];
         }
     }
@@ -64,11 +76,12 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
     const unsigned grid = (unsigned)((a.T + 7) / 8);
     if (a.dtype == MOE_BF16) {
         combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-            reinterpret_cast<const __nv_bfloat16*>(a.ye), a.idx, a.pos, a.drop, a.gate, a.offsets, a.T, a.d, a.k,
-            reinterpret_cast<__nv_bfloat16*>(a.out));
+            reinterpret_cast<const __nv_bfloat16*>(a.ye), a.idx, a.pos, a.drop, a.gate, a.offsets, a.claim_base,
+            a.counts, a.C, a.N, a.T, a.d, a.k, reinterpret_cast<__nv_bfloat16*>(a.out));
     } else {
         combine_kernel<float><<<grid, 256, 0, s>>>(reinterpret_cast<const float*>(a.ye), a.idx, a.pos, a.drop,
-                                                   a.gate, a.offsets, a.T, a.d, a.k, reinterpret_cast<float*>(a.out));
+                                                   a.gate, a.offsets, a.claim_base, a.counts, a.C, a.N, a.T, a.d,
+                                                   a.k, reinterpret_cast<float*>(a.out));
     }
     return cudaGetLastError();
 }

@@ -54,6 +54,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// ---- per-device one-time settings ------------------------------------------
+// Runs `set` once per (device, key); later calls return its first result.  key
+// identifies the kernel instance (e.g. its address).  Thread-safe.
+cudaError_t once_per_device(const void* key, cudaError_t (*set)(const void*));
+// Number of SMs of the current device (cached).
+cudaError_t device_sm_count(int* sms);
+
 // ---- launchers implemented in the .cu files ---------------------------------
 struct RouterArgs {
     const void* x; int dtype; const float* w_r; const float* b_r;
@@ -73,6 +80,12 @@ cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t s);
 cudaError_t launch_aux_finalize(const int32_t* part_cnt, const float* part_psum, int nblk, int N, int64_t T,
                                 float alpha, double* f, double* P, double* aux, cudaStream_t s);
 
+// Number of claims numbered base, base+1, ..., base+count-1 that fall below C.
+__host__ __device__ __forceinline__ int kept_after(int base, int count, int C) {
+    const int room = C - base;
+    return room <= 0 ? 0 : (room < count ? room : count);
+}
+
 struct DispatchArgs {
     const void* x; int dtype; const int32_t* idx; const float* gate;
     int64_t T; int d; int N; int k; int C;
@@ -80,9 +93,14 @@ struct DispatchArgs {
     int32_t* row_token; float* row_gate; void* xe;
     void* zero_out;              // top-1 fused path: rows of dropped tokens are zeroed
     uint32_t* scan_state; WsHeader* hdr;
+    const int32_t* claim_base;   // [k, N] claims made before this shard (sharded batch), or null
 };
 int scan_blocks(int64_t T);
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s);
+cudaError_t launch_counts(const int32_t* idx, int64_t T, int N, int k, int32_t* counts, cudaStream_t s);
+cudaError_t launch_claim_base(const int32_t* all, int S, int shard, int k, int N, int32_t* base, cudaStream_t s);
+cudaError_t launch_aux_shards(int S, int N, const int64_t* tokens, const double* f_all, const double* P_all,
+                              float alpha, double* f, double* P, double* aux, cudaStream_t s);
 cudaError_t launch_lookback_timeout_probe(uint32_t* state, WsHeader* hdr, long long limit_ns,
                                           cudaStream_t s);
 
@@ -104,6 +122,10 @@ struct CombineArgs {
     int dtype; int64_t T; int d; int k;
     const void* ye; const int32_t* idx; const int32_t* pos; const uint8_t* drop;
     const float* gate; const int32_t* offsets; void* out;
+    // one shard of a routing group (both null otherwise): pos are group-wide
+    // claim numbers; claim_base [k, N] and the shard's own counts [k, N] map
+    // them to the shard's rows.  C is the group capacity.
+    const int32_t* claim_base; const int32_t* counts; int C; int N;
 };
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 

@@ -79,8 +79,8 @@ __device__ uint32_t lookback(uint32_t* state, int bid, int c, int kN, uint32_t a
 
 __global__ void __launch_bounds__(kScanThreads)
 scan_kernel(const int32_t* __restrict__ idx, int64_t T, int N, int k, int C, int nblk,
-            int32_t* __restrict__ pos, int32_t* __restrict__ counts, int32_t* __restrict__ kept,
-            int32_t* __restrict__ offsets, uint32_t* __restrict__ state, WsHeader* hdr,
+            const int32_t* __restrict__ claim_base, int32_t* __restrict__ pos, int32_t* __restrict__ counts,
+            int32_t* __restrict__ kept, int32_t* __restrict__ offsets, uint32_t* __restrict__ state, WsHeader* hdr,
             long long limit_ns) {
     __shared__ int s_bid;
     __shared__ int s_last;
@@ -158,8 +158,13 @@ scan_kernel(const int32_t* __restrict__ idx, int64_t T, int N, int k, int C, int
     if (tid == 0) {
         int acc = 0;
         for (int e = 0; e < N; ++e) {
-            int total = s_tot[e] + (k == 2 ? s_tot[N + e] : 0);
-            int ke = total < C ? total : C;
+            // this shard's kept claims: rank-0 claims numbered from base0, rank-1
+            // claims from base1 (after every rank-0 claim); a whole batch is one
+            // shard with base0 = 0 and base1 = its own rank-0 total
+            const int c0 = s_tot[e], c1 = k == 2 ? s_tot[N + e] : 0;
+            const int base0 = claim_base ? claim_base[e] : 0;
+            const int base1 = claim_base ? claim_base[N + e] : c0;
+            const int ke = kept_after(base0, c0, C) + (k == 2 ? kept_after(base1, c1, C) : 0);
             kept[e] = ke;
             offsets[e] = acc;
             acc += ke;
@@ -172,8 +177,8 @@ template <typename XT>
 __global__ void __launch_bounds__(256)
 scatter_kernel(const XT* __restrict__ x, const int32_t* __restrict__ idx, const float* __restrict__ gate,
                int64_t T, int d, int N, int k, int C,
-               int32_t* __restrict__ pos, uint8_t* __restrict__ drop, const int32_t* __restrict__ counts,
-               const int32_t* __restrict__ offsets, int32_t* __restrict__ row_token,
+               const int32_t* __restrict__ claim_base, int32_t* __restrict__ pos, uint8_t* __restrict__ drop,
+               const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets, int32_t* __restrict__ row_token,
                float* __restrict__ row_gate, XT* __restrict__ xe, XT* __restrict__ zero_out) {
     const int lane = threadIdx.x & 31;
     const int64_t a = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -183,13 +188,21 @@ scatter_kernel(const XT* __restrict__ x, const int32_t* __restrict__ idx, const 
     int row = -1;
     if (lane == 0) {
         const int e = idx[a];
-        int p = pos[a];
-        if (r == 1) p += counts[e];          // every rank-0 claim precedes rank-1 claims
+        const int lp = pos[a];                  // claim number among this shard's rank-r claims on e
+        int p, row_off;
+        if (r == 0) {
+            p = (claim_base ? claim_base[e] : 0) + lp;
+            row_off = lp;
+        } else {                                // every rank-0 claim precedes the rank-1 claims
+            const int base0 = claim_base ? claim_base[e] : 0;
+            p = (claim_base ? claim_base[N + e] : counts[e]) + lp;
+            row_off = kept_after(base0, counts[e], C) + lp;
+        }
         const bool keep = p < C;
         pos[a] = p;
         drop[a] = keep ? 0 : 1;
         if (keep) {
-            row = offsets[e] + p;
+            row = offsets[e] + row_off;
             row_token[row] = (int32_t)t;
             row_gate[row] = gate[a];
         }
@@ -217,6 +230,69 @@ scatter_kernel(const XT* __restrict__ x, const int32_t* __restrict__ idx, const 
     }
 }
 
+// Claims per (rank, expert) of this shard: counts[r][e] (int atomics, so the
+// result is exact and order-independent).
+__global__ void __launch_bounds__(256)
+count_kernel(const int32_t* __restrict__ idx, int64_t T, int N, int k, int32_t* __restrict__ counts) {
+    __shared__ int h[256];
+    for (int c = threadIdx.x; c < k * N; c += blockDim.x) h[c] = 0;
+    __syncthreads();
+    const int64_t n = T * k;
+    for (int64_t a = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; a < n; a += (int64_t)gridDim.x * blockDim.x)
+        atomicAdd(&h[(int)(a % k) * N + idx[a]], 1);
+    __syncthreads();
+    for (int c = threadIdx.x; c < k * N; c += blockDim.x)
+        if (h[c]) atomicAdd(&counts[c], h[c]);
+}
+
+// Claim base of shard `shard` from every shard's counts [S][k][N]:
+//   base[0][e] = rank-0 claims on e by shards before this one;
+//   base[1][e] = all shards' rank-0 claims on e + rank-1 claims by earlier shards.
+__global__ void claim_base_kernel(const int32_t* __restrict__ all, int S, int shard, int k, int N,
+                                  int32_t* __restrict__ base) {
+    const int e = blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= N) return;
+    int b0 = 0, tot0 = 0, b1 = 0;
+    for (int s = 0; s < S; ++s) {
+        const int c0 = all[(int64_t)s * k * N + e];
+        tot0 += c0;
+        if (s < shard) {
+            b0 += c0;
+            if (k == 2) b1 += all[(int64_t)s * k * N + N + e];
+        }
+    }
+    base[e] = b0;
+    if (k == 2) base[N + e] = tot0 + b1;
+}
+
+// Load-balancing loss over shards: f and P are token-weighted means of the
+// shards' f_s and P_s (fp64, shard order), aux = alpha N sum_i f_i P_i.
+__global__ void aux_shards_kernel(int S, int N, const int64_t* __restrict__ tokens, const double* __restrict__ f_all,
+                                  const double* __restrict__ P_all, float alpha, double* __restrict__ f,
+                                  double* __restrict__ P, double* __restrict__ aux) {
+    __shared__ double fp[128];
+    const int e = threadIdx.x;
+    double T = 0.0;
+    for (int s = 0; s < S; ++s) T += (double)tokens[s];
+    if (e < N) {
+        double fs = 0.0, ps = 0.0;
+        for (int s = 0; s < S; ++s) {
+            fs += (double)tokens[s] * f_all[(int64_t)s * N + e];
+            ps += (double)tokens[s] * P_all[(int64_t)s * N + e];
+        }
+        const double fe = T > 0 ? fs / T : 0.0, pe = T > 0 ? ps / T : 0.0;
+        if (f) f[e] = fe;
+        if (P) P[e] = pe;
+        fp[e] = fe * pe;
+    }
+    __syncthreads();
+    if (e == 0 && aux) {
+        double acc = 0.0;
+        for (int q = 0; q < N; ++q) acc += fp[q];
+        *aux = (double)alpha * (double)N * acc;
+    }
+}
+
 // Test hook: one block whose predecessor (block 0) never publishes.
 __global__ void lookback_probe_kernel(uint32_t* state, WsHeader* hdr, long long limit_ns) {
     if (threadIdx.x < 4) lookback(state, 1, threadIdx.x, 4, 1u, limit_ns, &hdr->status);
@@ -234,23 +310,44 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
     if (err != cudaSuccess) return err;
     err = cudaMemsetAsync(a.scan_state, 0, sizeof(uint32_t) * (size_t)nblk * a.k * a.N, s);
     if (err != cudaSuccess) return err;
-    scan_kernel<<<nblk, kScanThreads, 0, s>>>(a.idx, a.T, a.N, a.k, a.C, nblk, a.pos, a.counts, a.kept,
-                                             a.offsets, a.scan_state, a.hdr, kWaitLimitNs);
+    scan_kernel<<<nblk, kScanThreads, 0, s>>>(a.idx, a.T, a.N, a.k, a.C, nblk, a.claim_base, a.pos, a.counts,
+                                             a.kept, a.offsets, a.scan_state, a.hdr, kWaitLimitNs);
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     const int64_t warps = a.T * a.k;
     const unsigned grid = (unsigned)((warps + 7) / 8);
     if (a.dtype == MOE_BF16) {
         scatter_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-            reinterpret_cast<const __nv_bfloat16*>(a.x), a.idx, a.gate, a.T, a.d, a.N, a.k, a.C, a.pos,
-            a.drop, a.counts, a.offsets, a.row_token, a.row_gate, reinterpret_cast<__nv_bfloat16*>(a.xe),
+            reinterpret_cast<const __nv_bfloat16*>(a.x), a.idx, a.gate, a.T, a.d, a.N, a.k, a.C, a.claim_base,
+            a.pos, a.drop, a.counts, a.offsets, a.row_token, a.row_gate, reinterpret_cast<__nv_bfloat16*>(a.xe),
             reinterpret_cast<__nv_bfloat16*>(a.zero_out));
     } else {
         scatter_kernel<float><<<grid, 256, 0, s>>>(
-            reinterpret_cast<const float*>(a.x), a.idx, a.gate, a.T, a.d, a.N, a.k, a.C, a.pos, a.drop,
-            a.counts, a.offsets, a.row_token, a.row_gate, reinterpret_cast<float*>(a.xe),
+            reinterpret_cast<const float*>(a.x), a.idx, a.gate, a.T, a.d, a.N, a.k, a.C, a.claim_base, a.pos,
+            a.drop, a.counts, a.offsets, a.row_token, a.row_gate, reinterpret_cast<float*>(a.xe),
             reinterpret_cast<float*>(a.zero_out));
     }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_counts(const int32_t* idx, int64_t T, int N, int k, int32_t* counts, cudaStream_t s) {
+    cudaError_t err = cudaMemsetAsync(counts, 0, sizeof(int32_t) * (size_t)k * N, s);
+    if (err != cudaSuccess || T == 0) return err;
+    const int64_t n = T * k;
+    int blocks = (int)((n + 255) / 256);
+    if (blocks > 1024) blocks = 1024;
+    count_kernel<<<blocks, 256, 0, s>>>(idx, T, N, k, counts);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_claim_base(const int32_t* all, int S, int shard, int k, int N, int32_t* base, cudaStream_t s) {
+    claim_base_kernel<<<1, 128, 0, s>>>(all, S, shard, k, N, base);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_aux_shards(int S, int N, const int64_t* tokens, const double* f_all, const double* P_all,
+                              float alpha, double* f, double* P, double* aux, cudaStream_t s) {
+    aux_shards_kernel<<<1, 128, 0, s>>>(S, N, tokens, f_all, P_all, alpha, f, P, aux);
     return cudaGetLastError();
 }
 

@@ -326,7 +326,10 @@ cudaError_t launch_router_t(const RouterArgs& a, cudaStream_t s) {
     const int nblk = (int)((a.T + S::TB - 1) / S::TB);
     const size_t smem = sizeof(float) * S::SMEM_FLOATS;
     auto kern = router_kernel<XT, TE, EG>;
-    cudaError_t err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t err = once_per_device(reinterpret_cast<const void*>(kern), [](const void* k) {
+        return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)(sizeof(float) * RouterShape<TE, EG>::SMEM_FLOATS));
+    });
     if (err != cudaSuccess) return err;
     if (nblk > 0) {
         kern<<<nblk, kThreads, smem, s>>>(reinterpret_cast<const XT*>(a.x), a.w_r, a.b_r, a.T, a.d, a.N,

@@ -475,8 +475,10 @@ cudaError_t run_router_tc(const RouterArgs& a, cudaStream_t s, int sms) {
     p.status = a.status;
     p.limit_ns = kWaitLimitNs;
     auto kern = router_tc_kernel<NP>;
-    if ((err = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_BYTES)) != cudaSuccess)
-        return err;
+    err = once_per_device(reinterpret_cast<const void*>(kern), [](const void* k) {
+        return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, RtShape<NP>::SMEM_BYTES);
+    });
+    if (err != cudaSuccess) return err;
     const int ntiles = (int)((a.T + RT_BM - 1) / RT_BM);
     const int grid = ntiles < sms ? ntiles : sms;
     kern<<<grid, RT_THREADS, S::SMEM_BYTES, s>>>(mx, mw, p);
@@ -488,9 +490,8 @@ cudaError_t run_router_tc(const RouterArgs& a, cudaStream_t s, int sms) {
 int router_tc_padded_experts(int N) { return N <= 16 ? 16 : (N <= 32 ? 32 : (N <= 64 ? 64 : 128)); }
 
 cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t s) {
-    int dev = 0, sms = 0;
-    cudaError_t err = cudaGetDevice(&dev);
-    if (err == cudaSuccess) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    int sms = 0;
+    cudaError_t err = device_sm_count(&sms);
     if (err != cudaSuccess) return err;
     if (a.T == 0)   // no tokens: f, P and the aux loss are zero
         return launch_aux_finalize(a.part_cnt, a.part_psum, 0, a.N, a.T, a.alpha, a.f, a.P, a.aux, s);

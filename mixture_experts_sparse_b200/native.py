@@ -42,9 +42,15 @@ _SIGS = {
     "moe_dispatch": ([ctypes.POINTER(MoeConfig)] + [_P] * 12 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_expert_ffn": ([ctypes.POINTER(MoeConfig)] + [_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_combine": ([ctypes.POINTER(MoeConfig)] + [_P] * 8, ctypes.c_int32),
+    "moe_combine_shard": ([ctypes.POINTER(MoeConfig)] + [_P] * 10, ctypes.c_int32),
     "moe_forward": ([ctypes.POINTER(MoeConfig)] + [_P] * 21 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_forward_events": ([ctypes.POINTER(MoeConfig)] + [_P] * 21 + [ctypes.c_size_t, _P, _P], ctypes.c_int32),
     "moe_dispatch_noalloc": ([ctypes.POINTER(MoeConfig)] + [_P] * 13, ctypes.c_int32),
+    "moe_dispatch_shard": ([ctypes.POINTER(MoeConfig)] + [_P] * 13 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_expert_counts": ([ctypes.POINTER(MoeConfig), _P, _P, _P], ctypes.c_int32),
+    "moe_claim_base": ([_P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _P, _P], ctypes.c_int32),
+    "moe_aux_shards": ([ctypes.c_int32, ctypes.c_int32, _P, _P, _P, ctypes.c_float, _P, _P, _P, _P],
+                       ctypes.c_int32),
     "moe_read_device_status": ([_P, _P], ctypes.c_int32),
     "moe_test_lookback_timeout": ([_P, ctypes.c_size_t, ctypes.c_int64, _P], ctypes.c_int32),
 }
@@ -144,6 +150,27 @@ def moe_dispatch_noalloc(cfg, x, idx, gate, pos, drop, counts, kept, offsets, ro
                                       _s(stream))
 
 
+def moe_expert_counts(cfg, idx, counts, stream=None):
+    return lib().moe_expert_counts(ctypes.byref(cfg), _p(idx), _p(counts), _s(stream))
+
+
+def moe_claim_base(shard_counts, n_shards, shard, top_k, n_experts, claim_base, stream=None):
+    return lib().moe_claim_base(_p(shard_counts), int(n_shards), int(shard), int(top_k), int(n_experts),
+                                _p(claim_base), _s(stream))
+
+
+def moe_dispatch_shard(cfg, x, idx, gate, claim_base, pos, drop, counts, kept, offsets, row_token, row_gate, xe,
+                       ws, stream=None):
+    return lib().moe_dispatch_shard(ctypes.byref(cfg), _p(x), _p(idx), _p(gate), _p(claim_base), _p(pos), _p(drop),
+                                    _p(counts), _p(kept), _p(offsets), _p(row_token), _p(row_gate), _p(xe), _p(ws),
+                                    _nbytes(ws), _s(stream))
+
+
+def moe_aux_shards(n_shards, n_experts, shard_tokens, f_all, P_all, alpha, f, P, aux, stream=None):
+    return lib().moe_aux_shards(int(n_shards), int(n_experts), _p(shard_tokens), _p(f_all), _p(P_all),
+                                float(alpha), _p(f), _p(P), _p(aux), _s(stream))
+
+
 def moe_expert_ffn(cfg, xe, offsets, w1, b1, w3, b3, w2, b2, ye, ws, stream=None):
     return lib().moe_expert_ffn(ctypes.byref(cfg), _p(xe), _p(offsets), _p(w1), _p(b1), _p(w3), _p(b3),
                                 _p(w2), _p(b2), _p(ye), _p(ws), _nbytes(ws), _s(stream))
@@ -152,6 +179,11 @@ def moe_expert_ffn(cfg, xe, offsets, w1, b1, w3, b3, w2, b2, ye, ws, stream=None
 def moe_combine(cfg, ye, idx, pos, drop, gate, offsets, out, stream=None):
     return lib().moe_combine(ctypes.byref(cfg), _p(ye), _p(idx), _p(pos), _p(drop), _p(gate), _p(offsets),
                              _p(out), _s(stream))
+
+
+def moe_combine_shard(cfg, ye, idx, pos, drop, gate, offsets, claim_base, counts, out, stream=None):
+    return lib().moe_combine_shard(ctypes.byref(cfg), _p(ye), _p(idx), _p(pos), _p(drop), _p(gate),
+                                   _p(offsets), _p(claim_base), _p(counts), _p(out), _s(stream))
 
 
 def moe_forward(cfg, x, w_r, b_r, w1, b1, w3, b3, w2, b2, out, idx=None, gate=None, pos=None, drop=None,
