@@ -170,13 +170,30 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
     __syncthreads();
     const int ntn = (p.n_dim + BN_OUT - 1) / BN_OUT;
-    if (tid == 0) {
-        int acc = 0;
-        for (int e = 0; e < N; ++e) {
-            s_prefix[e] = acc;
-            acc += ((s_off[e + 1] - s_off[e] + S::TILE_M - 1) / S::TILE_M) * ntn;
+    if (warp == 2) {
+        // tiles per expert and their exclusive prefix (one warp, N <= 128: four
+        // experts per lane, then a shuffle scan over the lanes)
+        int cnt[4], sum = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int e = lane * 4 + j;
+            cnt[j] = e < N ? ((s_off[e + 1] - s_off[e] + S::TILE_M - 1) / S::TILE_M) * ntn : 0;
+            sum += cnt[j];
         }
-        s_prefix[N] = acc;
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        int run = incl - sum;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int e = lane * 4 + j;
+            if (e < N) s_prefix[e] = run;
+            run += cnt[j];
+        }
+        if (lane == 31) s_prefix[N] = incl;   // all tiles
     }
     tc_fence_before();
     __syncthreads();
@@ -535,15 +552,14 @@ bool tc::make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t
     return r == CUDA_SUCCESS;
 }
 
-// Stage 1 + stage 2 of the bf16 expert FFN on the tensor cores: stage 1 on
-// one-CTA tiles (its short K makes the pair's larger tiles no faster), stage 2
+// Stage 1 + stage 2 of the bf16 expert FFN on the tensor cores, both
 // on CTA pairs unless MOE_B200_GEMM=single.
 cudaError_t launch_expert_ffn_tc(const FfnArgs& a, cudaStream_t s) {
     const int64_t R = a.R_cap > 0 ? a.R_cap : 1;
     const bool pair = use_pair();
     const bool swiglu = a.act == MOE_SWIGLU;
     // B rows per CTA and load: pair -> 128; single -> 256 (ReLU) or 128 + 128 (SwiGLU)
-    const int b1_box = swiglu ? BN / 2 : BN;
+    const int b1_box = (swiglu || pair) ? BN / 2 : BN;
     const int b2_box = pair ? BN / 2 : BN;
     CUtensorMap mA1, mB1, mB3, mA2, mB2;
     if (!make_map_bf16(&mA1, a.xe, R, a.d, BM) || !make_map_bf16(&mB1, a.w1, (int64_t)a.N * a.d_ff, a.d, b1_box) ||
@@ -565,8 +581,8 @@ cudaError_t launch_expert_ffn_tc(const FfnArgs& a, cudaStream_t s) {
     p1.out = reinterpret_cast<__nv_bfloat16*>(a.h);
     p1.status = &a.hdr->status;
     p1.limit_ns = kWaitLimitNs;
-    cudaError_t err = swiglu ? run_gemm<EPI_SWIGLU, false>(mA1, mB1, mB3, p1, s)
-                             : run_gemm<EPI_RELU, false>(mA1, mB1, mB3, p1, s);
+    cudaError_t err = swiglu ? run_gemm_any<EPI_SWIGLU>(mA1, mB1, mB3, p1, s)
+                             : run_gemm_any<EPI_RELU>(mA1, mB1, mB3, p1, s);
     if (err != cudaSuccess) return err;
     if (a.mid_event && (err = cudaEventRecord((cudaEvent_t)a.mid_event, s)) != cudaSuccess) return err;
 
