@@ -3,6 +3,7 @@
 // include/moe.h).  No entry point allocates, frees or synchronises, except
 // moe_read_device_status, which synchronises its stream.
 #include <cmath>
+#include <cstdlib>
 #include <cstring>
 #include <map>
 #include <mutex>
@@ -24,6 +25,14 @@ cudaError_t once_per_device(const void* key, cudaError_t (*set)(const void*)) {
     err = set(key);
     done[{dev, key}] = err;
     return err;
+}
+
+bool pdl_enabled() {
+    static const bool on = [] {
+        const char* v = getenv("MOE_B200_PDL");
+        return !(v && strcmp(v, "0") == 0);
+    }();
+    return on;
 }
 
 cudaError_t device_sm_count(int* sms) {

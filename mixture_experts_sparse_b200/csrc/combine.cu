@@ -24,6 +24,8 @@ combine_kernel(const XT* __restrict__ ye, const int32_t* __restrict__ idx, const
                const int32_t* __restrict__ offsets, const int32_t* __restrict__ claim_base,
                const int32_t* __restrict__ counts, int C, int N, int64_t T, int d, int k, XT* __restrict__ out) {
     constexpr int VEC = 16 / sizeof(XT);
+    pdl_wait();
+    pdl_launch();
     const int lane = threadIdx.x & 31;
     const int64_t t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (t >= T) return;
@@ -74,16 +76,13 @@ combine_kernel(const XT* __restrict__ ye, const int32_t* __restrict__ idx, const
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
     if (a.T <= 0) return cudaSuccess;
     const unsigned grid = (unsigned)((a.T + 7) / 8);
-    if (a.dtype == MOE_BF16) {
-        combine_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-            reinterpret_cast<const __nv_bfloat16*>(a.ye), a.idx, a.pos, a.drop, a.gate, a.offsets, a.claim_base,
-            a.counts, a.C, a.N, a.T, a.d, a.k, reinterpret_cast<__nv_bfloat16*>(a.out));
-    } else {
-        combine_kernel<float><<<grid, 256, 0, s>>>(reinterpret_cast<const float*>(a.ye), a.idx, a.pos, a.drop,
-                                                   a.gate, a.offsets, a.claim_base, a.counts, a.C, a.N, a.T, a.d,
-                                                   a.k, reinterpret_cast<float*>(a.out));
-    }
-    return cudaGetLastError();
+    if (a.dtype == MOE_BF16)
+        return launch_k(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, 1,
+                        reinterpret_cast<const __nv_bfloat16*>(a.ye), a.idx, a.pos, a.drop, a.gate, a.offsets,
+                        a.claim_base, a.counts, a.C, a.N, a.T, a.d, a.k, reinterpret_cast<__nv_bfloat16*>(a.out));
+    return launch_k(combine_kernel<float>, dim3(grid), dim3(256), 0, s, 1, reinterpret_cast<const float*>(a.ye), a.idx,
+                    a.pos, a.drop, a.gate, a.offsets, a.claim_base, a.counts, a.C, a.N, a.T, a.d, a.k,
+                    reinterpret_cast<float*>(a.out));
 }
 
 }  // namespace moe

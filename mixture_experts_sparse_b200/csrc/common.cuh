@@ -54,6 +54,51 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// ---- programmatic dependent launch ------------------------------------------
+// The layer's kernels are launched with programmatic stream serialization: a
+// kernel may be scheduled while its predecessor in the stream is finishing, so
+// its prologue (barrier init, TMEM allocation, tensor-map prefetch) overlaps
+// the predecessor's tail.  Every such kernel calls pdl_wait() before its first
+// global-memory access (the predecessor has then completed: its writes are
+// visible and its reads are done) and pdl_launch() right after, so a kernel's
+// successor starts only once the kernel itself is past its own wait, and at
+// most two kernels of the stream overlap.  Without the launch attribute both
+// are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// false when MOE_B200_PDL=0 (plain stream order, kept for measurement)
+bool pdl_enabled();
+
+// Launch `kern` on stream s with programmatic stream serialization (unless
+// disabled) and, for cluster_x > 1, clusters of cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, int cluster_x,
+                     Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    unsigned n = 0;
+    if (pdl_enabled()) {
+        attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[n].val.programmaticStreamSerializationAllowed = 1;
+        ++n;
+    }
+    if (cluster_x > 1) {
+        attr[n].id = cudaLaunchAttributeClusterDimension;
+        attr[n].val.clusterDim.x = (unsigned)cluster_x;
+        attr[n].val.clusterDim.y = 1;
+        attr[n].val.clusterDim.z = 1;
+        ++n;
+    }
+    cfg.attrs = attr;
+    cfg.numAttrs = n;
+    return cudaLaunchKernelEx(&cfg, kern, static_cast<Args&&>(args)...);
+}
+
 // ---- per-device one-time settings ------------------------------------------
 // Runs `set` once per (device, key); later calls return its first result.  key
 // identifies the kernel instance (e.g. its address).  Thread-safe.

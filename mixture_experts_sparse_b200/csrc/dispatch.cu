@@ -82,6 +82,8 @@ scan_kernel(const int32_t* __restrict__ idx, int64_t T, int N, int k, int C, int
             const int32_t* __restrict__ claim_base, int32_t* __restrict__ pos, int32_t* __restrict__ counts,
             int32_t* __restrict__ kept, int32_t* __restrict__ offsets, uint32_t* __restrict__ state, WsHeader* hdr,
             long long limit_ns) {
+    pdl_wait();
+    pdl_launch();
     __shared__ int s_bid;
     __shared__ int s_last;
     __shared__ int s_wcnt[8][256];
@@ -180,6 +182,8 @@ scatter_kernel(const XT* __restrict__ x, const int32_t* __restrict__ idx, const 
                const int32_t* __restrict__ claim_base, int32_t* __restrict__ pos, uint8_t* __restrict__ drop,
                const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets, int32_t* __restrict__ row_token,
                float* __restrict__ row_gate, XT* __restrict__ xe, XT* __restrict__ zero_out) {
+    pdl_wait();
+    pdl_launch();
     const int lane = threadIdx.x & 31;
     const int64_t a = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
     if (a >= T * k) return;
@@ -310,24 +314,19 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
     if (err != cudaSuccess) return err;
     err = cudaMemsetAsync(a.scan_state, 0, sizeof(uint32_t) * (size_t)nblk * a.k * a.N, s);
     if (err != cudaSuccess) return err;
-    scan_kernel<<<nblk, kScanThreads, 0, s>>>(a.idx, a.T, a.N, a.k, a.C, nblk, a.claim_base, a.pos, a.counts,
-                                             a.kept, a.offsets, a.scan_state, a.hdr, kWaitLimitNs);
-    err = cudaGetLastError();
+    err = launch_k(scan_kernel, dim3((unsigned)nblk), dim3(kScanThreads), 0, s, 1, a.idx, a.T, a.N, a.k, a.C, nblk,
+                   a.claim_base, a.pos, a.counts, a.kept, a.offsets, a.scan_state, a.hdr, kWaitLimitNs);
     if (err != cudaSuccess) return err;
     const int64_t warps = a.T * a.k;
     const unsigned grid = (unsigned)((warps + 7) / 8);
-    if (a.dtype == MOE_BF16) {
-        scatter_kernel<__nv_bfloat16><<<grid, 256, 0, s>>>(
-            reinterpret_cast<const __nv_bfloat16*>(a.x), a.idx, a.gate, a.T, a.d, a.N, a.k, a.C, a.claim_base,
-            a.pos, a.drop, a.counts, a.offsets, a.row_token, a.row_gate, reinterpret_cast<__nv_bfloat16*>(a.xe),
-            reinterpret_cast<__nv_bfloat16*>(a.zero_out));
-    } else {
-        scatter_kernel<float><<<grid, 256, 0, s>>>(
-            reinterpret_cast<const float*>(a.x), a.idx, a.gate, a.T, a.d, a.N, a.k, a.C, a.claim_base, a.pos,
-            a.drop, a.counts, a.offsets, a.row_token, a.row_gate, reinterpret_cast<float*>(a.xe),
-            reinterpret_cast<float*>(a.zero_out));
-    }
-    return cudaGetLastError();
+    if (a.dtype == MOE_BF16)
+        return launch_k(scatter_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, 1,
+                        reinterpret_cast<const __nv_bfloat16*>(a.x), a.idx, a.gate, a.T, a.d, a.N, a.k, a.C,
+                        a.claim_base, a.pos, a.drop, a.counts, a.offsets, a.row_token, a.row_gate,
+                        reinterpret_cast<__nv_bfloat16*>(a.xe), reinterpret_cast<__nv_bfloat16*>(a.zero_out));
+    return launch_k(scatter_kernel<float>, dim3(grid), dim3(256), 0, s, 1, reinterpret_cast<const float*>(a.x), a.idx,
+                    a.gate, a.T, a.d, a.N, a.k, a.C, a.claim_base, a.pos, a.drop, a.counts, a.offsets, a.row_token,
+                    a.row_gate, reinterpret_cast<float*>(a.xe), reinterpret_cast<float*>(a.zero_out));
 }
 
 cudaError_t launch_counts(const int32_t* idx, int64_t T, int N, int k, int32_t* counts, cudaStream_t s) {

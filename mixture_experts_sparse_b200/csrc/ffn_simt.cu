@@ -26,6 +26,8 @@ __global__ void __launch_bounds__(256)
 simt_gemm_kernel(const float* __restrict__ A, const int32_t* __restrict__ offsets, int K, int n_dim,
                  const float* __restrict__ B, const float* __restrict__ B3, const float* __restrict__ bias,
                  const float* __restrict__ bias3, float* __restrict__ out) {
+    pdl_wait();
+    pdl_launch();
     const int e = blockIdx.z;
     const int row0 = offsets[e];
     const int rows = offsets[e + 1] - row0;
@@ -98,23 +100,20 @@ cudaError_t launch_expert_ffn_simt(const FfnArgs& a, cudaStream_t s) {
     const float* xe = reinterpret_cast<const float*>(a.xe);
     float* h = reinterpret_cast<float*>(a.h);
     dim3 g1(mt, (unsigned)((a.d_ff + TS - 1) / TS), (unsigned)a.N);
-    if (a.act == MOE_SWIGLU) {
-        simt_gemm_kernel<SIMT_SWIGLU><<<g1, 256, 0, s>>>(
-            xe, a.offsets, a.d, a.d_ff, reinterpret_cast<const float*>(a.w1), reinterpret_cast<const float*>(a.w3),
-            reinterpret_cast<const float*>(a.b1), reinterpret_cast<const float*>(a.b3), h);
-    } else {
-        simt_gemm_kernel<SIMT_RELU><<<g1, 256, 0, s>>>(xe, a.offsets, a.d, a.d_ff,
-                                                       reinterpret_cast<const float*>(a.w1), nullptr,
-                                                       reinterpret_cast<const float*>(a.b1), nullptr, h);
-    }
-    cudaError_t err = cudaGetLastError();
+    const float* none = nullptr;
+    cudaError_t err =
+        a.act == MOE_SWIGLU
+            ? launch_k(simt_gemm_kernel<SIMT_SWIGLU>, g1, dim3(256), 0, s, 1, xe, a.offsets, a.d, a.d_ff,
+                       reinterpret_cast<const float*>(a.w1), reinterpret_cast<const float*>(a.w3),
+                       reinterpret_cast<const float*>(a.b1), reinterpret_cast<const float*>(a.b3), h)
+            : launch_k(simt_gemm_kernel<SIMT_RELU>, g1, dim3(256), 0, s, 1, xe, a.offsets, a.d, a.d_ff,
+                       reinterpret_cast<const float*>(a.w1), none, reinterpret_cast<const float*>(a.b1), none, h);
     if (err != cudaSuccess) return err;
     if (a.mid_event && (err = cudaEventRecord((cudaEvent_t)a.mid_event, s)) != cudaSuccess) return err;
     dim3 g2(mt, (unsigned)((a.d + TS - 1) / TS), (unsigned)a.N);
-    simt_gemm_kernel<SIMT_BIAS><<<g2, 256, 0, s>>>(h, a.offsets, a.d_ff, a.d, reinterpret_cast<const float*>(a.w2),
-                                                   nullptr, reinterpret_cast<const float*>(a.b2), nullptr,
-                                                   reinterpret_cast<float*>(a.ye));
-    return cudaGetLastError();
+    return launch_k(simt_gemm_kernel<SIMT_BIAS>, g2, dim3(256), 0, s, 1, static_cast<const float*>(h), a.offsets,
+                    a.d_ff, a.d, reinterpret_cast<const float*>(a.w2), none, reinterpret_cast<const float*>(a.b2), none,
+                    reinterpret_cast<float*>(a.ye));
 }
 
 }  // namespace

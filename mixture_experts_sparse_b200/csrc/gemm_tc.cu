@@ -146,7 +146,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const int first_tile = PAIR ? (int)cluster_id_x() : (int)blockIdx.x;
     const int tile_step = PAIR ? (int)ncluster_x() : (int)gridDim.x;
     const int N = p.N;
-    for (int i = tid; i <= N; i += GEMM_THREADS) s_off[i] = p.offsets[i];
     if (tid == 0) {
         for (int s = 0; s < S::STAGES; ++s) {
             mbar_init(smem_u32(&full_bar[s]), 1);
@@ -168,6 +167,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         if (PAIR) tmem_alloc_pair(&s_tmem, TMEM_COLS);
         else tmem_alloc(&s_tmem, TMEM_COLS);
     }
+    pdl_wait();   // the compact rows and offsets are ready from here on
+    pdl_launch();
+    for (int i = tid; i <= N; i += GEMM_THREADS) s_off[i] = p.offsets[i];
     __syncthreads();
     const int ntn = (p.n_dim + BN_OUT - 1) / BN_OUT;
     if (warp == 2) {
@@ -481,24 +483,12 @@ cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorM
         }
         sms = di.sms;
     }
-    if constexpr (!PAIR) {
-        grouped_gemm_kernel<EPI, false><<<sms, GEMM_THREADS, S::SMEM_BYTES, s>>>(a, b, b3, p);
-        return cudaGetLastError();
-    } else {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(sms / 2) * 2, 1, 1);
-    cfg.blockDim = dim3(GEMM_THREADS, 1, 1);
-    cfg.dynamicSmemBytes = S::SMEM_BYTES;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, grouped_gemm_kernel<EPI, true>, a, b, b3, p);
-    }
+    if constexpr (!PAIR)
+        return launch_k(grouped_gemm_kernel<EPI, false>, dim3((unsigned)sms), dim3(GEMM_THREADS), S::SMEM_BYTES, s,
+                        1, a, b, b3, p);
+    else
+        return launch_k(grouped_gemm_kernel<EPI, true>, dim3((unsigned)(sms / 2) * 2), dim3(GEMM_THREADS),
+                        S::SMEM_BYTES, s, 2, a, b, b3, p);
 }
 
 // Variant choice: the CTA-pair kernel unless MOE_B200_GEMM=single (kept for

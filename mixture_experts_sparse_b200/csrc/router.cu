@@ -54,6 +54,8 @@ router_kernel(const XT* __restrict__ x, const float* __restrict__ w_r, const flo
     constexpr int PARTS = kDK / VEC;              // 16-byte loads per row chunk
     constexpr int NL = S::TB * PARTS / kThreads;  // 16-byte loads per thread per chunk
     static_assert(NL >= 1 && (S::TB * PARTS) % kThreads == 0, "loader shape");
+    pdl_wait();
+    pdl_launch();
 
     extern __shared__ float smem[];
     float* xs = smem;               // [kDK][TB]
@@ -273,6 +275,8 @@ aux_finalize_kernel(const int32_t* __restrict__ part_cnt, const float* __restric
     __shared__ double sp[1024];
     __shared__ double sc[1024];
     __shared__ double sfp[128];
+    pdl_wait();
+    pdl_launch();
     int npow = 1;
     while (npow < N) npow <<= 1;
     const int tpe = 1024 / npow;
@@ -332,9 +336,8 @@ cudaError_t launch_router_t(const RouterArgs& a, cudaStream_t s) {
     });
     if (err != cudaSuccess) return err;
     if (nblk > 0) {
-        kern<<<nblk, kThreads, smem, s>>>(reinterpret_cast<const XT*>(a.x), a.w_r, a.b_r, a.T, a.d, a.N,
-                                          a.k, a.idx, a.gate, a.probs, a.part_cnt, a.part_psum);
-        err = cudaGetLastError();
+        err = launch_k(kern, dim3((unsigned)nblk), dim3(kThreads), smem, s, 1, reinterpret_cast<const XT*>(a.x), a.w_r,
+                       a.b_r, a.T, a.d, a.N, a.k, a.idx, a.gate, a.probs, a.part_cnt, a.part_psum);
         if (err != cudaSuccess) return err;
     }
     return launch_aux_finalize(a.part_cnt, a.part_psum, nblk, a.N, a.T, a.alpha, a.f, a.P, a.aux, s);
@@ -361,15 +364,15 @@ int router_blocks(int64_t T, int N) {
 }
 
 int router_partial_rows(int64_t T, int N) {
-    const int tc_rows = (int)(((T + 127) / 128 + 3) / 4 * 4);   // >= the tensor-core router's grid, rounded to 4
+    const int tc_rows = (int)((2 * ((T + 255) / 256) + 3) / 4 * 4);   // >= the tensor-core router's grid, rounded to 4
     const int simt_rows = router_blocks(T, N);
     return tc_rows > simt_rows ? tc_rows : simt_rows;
 }
 
 cudaError_t launch_aux_finalize(const int32_t* part_cnt, const float* part_psum, int nblk, int N, int64_t T,
                                 float alpha, double* f, double* P, double* aux, cudaStream_t s) {
-    aux_finalize_kernel<<<1, 1024, 0, s>>>(part_cnt, part_psum, nblk, N, T, alpha, f, P, aux);
-    return cudaGetLastError();
+    return launch_k(aux_finalize_kernel, dim3(1), dim3(1024), 0, s, 1, part_cnt, part_psum, nblk, N, T, alpha, f, P,
+                    aux);
 }
 
 // bf16 activations: the tensor-core router (exact three-way split of W_r);

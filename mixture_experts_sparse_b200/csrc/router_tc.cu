@@ -23,12 +23,16 @@
 // the partial logits in fp32 with round-to-nearest in a fixed order.  The router then costs about one read
 // of x from HBM instead of 2 d N FP32-pipe FLOPs per token.
 //
-// Kernel: persistent, 192 threads: warp 0 TMA producer (x tile 128 x 64 and
-// the three W parts, NP x 64 each, 128-byte swizzle), warp 1 TMEM allocator +
-// MMA issuer (M = 128 tokens, N = NP padded experts, K = 16), warps 2-5
-// epilogue with one thread per token: the thread holds its token's NP logits
-// (tcgen05.ld), computes max, softmax, top-1/top-2 and the gate in registers,
-// and writes idx/gate (and probs).  Per-tile partial sums of p and top-1
+// Kernel: persistent CTA pairs (clusters of two), 192 threads per CTA.  A
+// pair owns a 256-token tile and issues cta_group::2 MMAs (M = 256 tokens, 128
+// per CTA): each CTA loads its own 128 x 64 x tile and half of the three W
+// parts' rows, so the W bytes streamed per token are half those of a one-CTA
+// tile and more stages fit.  Warp 0 TMA producer (128-byte swizzle; both
+// CTAs' loads complete on the leader's barrier), warp 1 TMEM allocator + MMA
+// issuer (the leader's), warps 2-5 epilogue with one thread per token of its
+// own CTA: the thread holds its token's NP logits (tcgen05.ld), computes max,
+// softmax, top-1/top-2 and the gate in registers, and writes idx/gate (and
+// probs).  Per-tile partial sums of p and top-1
 // counts are reduced in a fixed order (lanes in a warp through shared memory,
 // then the four warps in quadrant order), so the aux loss is deterministic.
 #include "tc_common.cuh"
@@ -38,34 +42,38 @@ using namespace tc;
 namespace {
 
 constexpr int RT_THREADS = 192;
-constexpr int RT_BM = 128;
+constexpr int RT_BM = 128;       // tokens per CTA (256 per pair)
 constexpr int RT_BK = 64;
 
 template <int NP>
 struct RtShape {
     static constexpr int A_BYTES = RT_BM * RT_BK * 2;
-    static constexpr int P_BYTES = NP * RT_BK * 2;             // one W part
+    static constexpr int P_BYTES = (NP / 2) * RT_BK * 2;       // this CTA's half of one W part
     static constexpr int STAGE_BYTES = A_BYTES + 3 * P_BYTES;
-    static constexpr int STAGES = NP <= 64 ? 4 : 2;
+    static constexpr int STAGES = NP <= 64 ? 6 : 3;
     // per epilogue thread, a row of running sums of p over its tokens (padded
     // by one float so the rows of a warp fall in different banks)
     static constexpr int ACC_STRIDE = NP + 1;
     static constexpr int ACC_BYTES = 4 * 32 * ACC_STRIDE * 4;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + ACC_BYTES;
-    // merged: one MMA of N = 3 NP covers the three W parts (adjacent in shared
-    // memory) and leaves three partial-logit blocks side by side in TMEM
+    // merged: one MMA of N = 3 NP covers the three W parts and leaves three
+    // partial-logit blocks side by side in TMEM; the pair's leader holds W rows
+    // [0, 3 NP / 2) of the stacked parts, the peer rows [3 NP / 2, 3 NP).
+    // Otherwise each part is its own MMA of N = NP, NP / 2 rows per CTA.
     static constexpr bool MERGED = 3 * NP <= 256;
+    static constexpr int W_BOX = MERGED ? 3 * NP / 2 : NP / 2;   // rows per W load
     static constexpr int ACC_COLS = MERGED ? 3 * NP : NP;      // TMEM columns per K-group accumulator
-    static constexpr int TMEM_COLS = 512;                      // 2 buffers x G groups x ACC_COLS
-    static constexpr int MAX_GROUPS = TMEM_COLS / (2 * ACC_COLS);
+    static constexpr int TMEM_COLS = 512;                      // buffers x G groups x ACC_COLS
     static constexpr int MMA_PER_KB = MERGED ? RT_BK / 16 : 3 * (RT_BK / 16);
     static constexpr int KB_PER_GROUP = 64 / MMA_PER_KB;       // <= 64 MMAs per accumulator
+    static_assert(STAGE_BYTES % 1024 == 0, "1024-byte aligned stages");
 };
 
 struct RtParams {
     int64_t T;
     int N, k, d;
     int groups;   // K groups with separate accumulators
+    int nbuf;     // accumulator buffers (2: the epilogue overlaps the next tile's MMAs)
     int kb_per_group;
     const float* b_r;
     int32_t* idx;
@@ -127,7 +135,7 @@ template <int NP>
 __global__ void __launch_bounds__(RT_THREADS, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, const RtParams p) {
     using S = RtShape<NP>;
-    constexpr uint32_t IDESC = idesc_bf16_f32(RT_BM, S::ACC_COLS);
+    constexpr uint32_t IDESC = idesc_bf16_f32(2 * RT_BM, S::ACC_COLS);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     float* pacc = reinterpret_cast<float*>(smem + S::STAGES * S::STAGE_BYTES);   // [4][32][NP + 1]
@@ -143,6 +151,10 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     __shared__ double s_fp[NP];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t rank = cluster_ctarank();   // 0 = the pair's leader
+    const bool leader = rank == 0;
+    const int first_tile = (int)cluster_id_x();
+    const int tile_step = (int)ncluster_x();
     if (tid == 0) {
         for (int s = 0; s < S::STAGES; ++s) {
             mbar_init(smem_u32(&full_bar[s]), 1);
@@ -150,7 +162,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         }
         for (int a = 0; a < 2; ++a) {
             mbar_init(smem_u32(&tfull_bar[a]), 1);
-            mbar_init(smem_u32(&tempty_bar[a]), 128);
+            mbar_init(smem_u32(&tempty_bar[a]), 256);   // both CTAs' epilogue threads
         }
         mbar_init(smem_u32(&done_bar), 1);
         s_abort = 0;
@@ -162,13 +174,16 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         prefetch_tmap(&tmX);
         prefetch_tmap(&tmW);
     }
-    if (warp == 1) tmem_alloc(&s_tmem, S::TMEM_COLS);
+    if (warp == 1) tmem_alloc_pair(&s_tmem, S::TMEM_COLS);
     tc_fence_before();
     __syncthreads();
+    cluster_sync();   // the peer's barriers exist before any cross-CTA signal
     tc_fence_after();
+    pdl_wait();       // x, the W split and the workspace are ready from here on
+    pdl_launch();
 
     const uint32_t tmem_base = s_tmem;
-    const int ntiles = (int)((p.T + RT_BM - 1) / RT_BM);
+    const int ntiles = (int)((p.T + 2 * RT_BM - 1) / (2 * RT_BM));
     const int nkb = (p.d + RT_BK - 1) / RT_BK;
     const Waiter w{&s_abort, p.status, p.limit_ns};
 
@@ -180,19 +195,26 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 #pragma unroll
             for (int s = 0; s < S::STAGES; ++s) last_par[s] = -1;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
+            for (int tile = first_tile; tile < ntiles && ok; tile += tile_step) {
+                const int xrow = tile * 2 * RT_BM + (int)rank * RT_BM;
                 for (int kb = 0; kb < nkb; ++kb) {
                     if (!wait_bar(smem_u32(&empty_bar[stage]), phase ^ 1u, w)) {
                         ok = false;
                         break;
                     }
                     const uint32_t fb = smem_u32(&full_bar[stage]);
+                    const uint32_t fb_leader = map_to_rank(fb, 0);
                     const uint32_t a_dst = smem_u32(smem + stage * S::STAGE_BYTES);
-                    mbar_expect_tx(fb, S::STAGE_BYTES);
-                    tma_load_2d(a_dst, &tmX, fb, kb * RT_BK, tile * RT_BM);
+                    if (leader) mbar_expect_tx(fb, 2 * S::STAGE_BYTES);   // both CTAs' bytes
+                    tma_load_2d_pair(a_dst, &tmX, fb_leader, kb * RT_BK, xrow);
+                    if constexpr (S::MERGED) {
+                        tma_load_2d_pair(a_dst + S::A_BYTES, &tmW, fb_leader, kb * RT_BK, (int)rank * S::W_BOX);
+                    } else {
 #pragma unroll
-                    for (int part = 0; part < 3; ++part)
-                        tma_load_2d(a_dst + S::A_BYTES + part * S::P_BYTES, &tmW, fb, kb * RT_BK, part * NP);
+                        for (int part = 0; part < 3; ++part)
+                            tma_load_2d_pair(a_dst + S::A_BYTES + part * S::P_BYTES, &tmW, fb_leader, kb * RT_BK,
+                                             part * NP + (int)rank * S::W_BOX);
+                    }
                     last_par[stage] = (int)phase;
                     if (++stage == S::STAGES) {
                         stage = 0;
@@ -200,19 +222,21 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     }
                 }
             }
+            // the leader's MMA released every stage this thread filled, which it
+            // does only after the stage's bytes (both CTAs') arrived
             for (int s = 0; s < S::STAGES; ++s)
-                if (last_par[s] >= 0) drain_bar(smem_u32(&full_bar[s]), (uint32_t)last_par[s], p.limit_ns, p.status);
+                if (last_par[s] >= 0) drain_bar(smem_u32(&empty_bar[s]), (uint32_t)last_par[s], p.limit_ns, p.status);
         }
     } else if (warp == 1) {
-        if (lane == 0) {
+        if (lane == 0 && leader) {
             int stage = 0;
             uint32_t phase = 0;
             int it = 0;
             bool ok = true, issued = false;
             const uint64_t desc0 = umma_desc(smem_u32(smem));
-            for (int tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x, ++it) {
-                const int acc = it & 1;
-                const uint32_t acc_par = (uint32_t)((it >> 1) & 1);
+            for (int tile = first_tile; tile < ntiles && ok; tile += tile_step, ++it) {
+                const int acc = p.nbuf == 2 ? (it & 1) : 0;
+                const uint32_t acc_par = (uint32_t)(p.nbuf == 2 ? ((it >> 1) & 1) : (it & 1));
                 if (!wait_bar(smem_u32(&tempty_bar[acc]), acc_par ^ 1u, w)) break;
                 tc_fence_after();
                 for (int kb = 0; kb < nkb; ++kb) {
@@ -231,26 +255,31 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 #pragma unroll
                     for (int kk = 0; kk < RT_BK / 16; ++kk) {
                         if constexpr (S::MERGED) {
-                            umma_f16(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, IDESC, (!first || kk != 0) ? 1u : 0u);
+                            umma_f16_pair(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, IDESC,
+                                          (!first || kk != 0) ? 1u : 0u);
                         } else {
 #pragma unroll
                             for (int part = 0; part < 3; ++part)
-                                umma_f16(d_tmem, a_desc + 2 * kk, b_desc + (uint64_t)((part * S::P_BYTES) >> 4) + 2 * kk,
-                                         IDESC, (!first || (kk | part) != 0) ? 1u : 0u);
+                                umma_f16_pair(d_tmem, a_desc + 2 * kk,
+                                              b_desc + (uint64_t)((part * S::P_BYTES) >> 4) + 2 * kk, IDESC,
+                                              (!first || (kk | part) != 0) ? 1u : 0u);
                         }
                     }
-                    umma_commit(smem_u32(&empty_bar[stage]));
+                    umma_commit_pair(smem_u32(&empty_bar[stage]), 0x3);   // frees the stage in both CTAs
                     if (++stage == S::STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
-                if (ok) umma_commit(smem_u32(&tfull_bar[acc]));
+                if (ok) umma_commit_pair(smem_u32(&tfull_bar[acc]), 0x3);
             }
             if (issued) {
-                umma_commit(smem_u32(&done_bar));
+                umma_commit_pair(smem_u32(&done_bar), 0x3);
                 drain_bar(smem_u32(&done_bar), 0u, p.limit_ns, p.status);
             }
+        } else if (lane == 0 && !leader && first_tile < ntiles) {
+            // the peer's TMEM and shared memory are in use until the leader's MMAs end
+            drain_bar(smem_u32(&done_bar), 0u, p.limit_ns, p.status);
         }
         __syncwarp();
     } else {
@@ -258,14 +287,16 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         const int q = warp & 3;
         float* prow = pacc + (q * 32 + lane) * S::ACC_STRIDE;   // this thread's running sums
         const int N = p.N, k = p.k;
+        const uint32_t tempty_leader0 = map_to_rank(smem_u32(&tempty_bar[0]), 0);
+        const uint32_t tempty_leader1 = map_to_rank(smem_u32(&tempty_bar[1]), 0);
         int it = 0;
-        for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
-            const int acc = it & 1;
-            const uint32_t acc_par = (uint32_t)((it >> 1) & 1);
+        for (int tile = first_tile; tile < ntiles; tile += tile_step, ++it) {
+            const int acc = p.nbuf == 2 ? (it & 1) : 0;
+            const uint32_t acc_par = (uint32_t)(p.nbuf == 2 ? ((it >> 1) & 1) : (it & 1));
             const bool got = wait_bar(smem_u32(&tfull_bar[acc]), acc_par, w);
             if (!__all_sync(0xffffffffu, got)) break;   // warp-uniform exit on abort
             tc_fence_after();
-            const int64_t t = (int64_t)tile * RT_BM + q * 32 + lane;
+            const int64_t t = (int64_t)tile * 2 * RT_BM + (int)rank * RT_BM + q * 32 + lane;
             const bool valid = t < p.T;
             float v[NP];
 #pragma unroll
@@ -290,7 +321,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 }
             }
             tc_fence_before();
-            mbar_arrive_relaxed(smem_u32(&tempty_bar[acc]));   // the accumulator is free again
+            mbar_arrive_cluster_relaxed(acc ? tempty_leader1 : tempty_leader0);   // the accumulator is free again
 
             if (p.b_r) {
 #pragma unroll
@@ -356,8 +387,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 
     tc_fence_before();
     __syncthreads();
+    cluster_sync();   // no CTA leaves while its peer may still signal it
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem_base, S::TMEM_COLS);
+    if (warp == 1) tmem_dealloc_pair(tmem_base, S::TMEM_COLS);
 
     // ---- the last CTA to finish reduces every CTA's partials: f, P, aux ----
     if (tid == 0) s_last = (atomicAdd(p.ticket, 1) == (int)gridDim.x - 1);
@@ -420,6 +452,8 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 // fp32 [N, d] -> bf16 [3, NP, d]: w = w0 + w1 + w2 exactly; rows >= N are zero.
 __global__ void split_router_weights_kernel(const float* __restrict__ w_r, int N, int NP, int d,
                                             __nv_bfloat16* __restrict__ out) {
+    pdl_wait();
+    pdl_launch();
     const int64_t n = (int64_t)NP * d;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
         const int e = (int)(i / d);
@@ -442,23 +476,37 @@ cudaError_t run_router_tc(const RouterArgs& a, cudaStream_t s, int sms) {
     const int threads = 256;
     const int64_t n = (int64_t)NP * a.d;
     const int blocks = (int)((n + threads - 1) / threads < 1024 ? (n + threads - 1) / threads : 1024);
-    split_router_weights_kernel<<<blocks, threads, 0, s>>>(a.w_r, a.N, NP, a.d,
-                                                           reinterpret_cast<__nv_bfloat16*>(a.w_split));
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    err = launch_k(split_router_weights_kernel, dim3((unsigned)blocks), dim3(threads), 0, s, 1, a.w_r, a.N, NP, a.d,
+                   reinterpret_cast<__nv_bfloat16*>(a.w_split));
+    if (err != cudaSuccess) return err;
     CUtensorMap mx, mw;
-    if (!make_map_bf16(&mx, a.x, a.T, a.d, RT_BM) || !make_map_bf16(&mw, a.w_split, 3 * NP, a.d, NP))
+    if (!make_map_bf16(&mx, a.x, a.T, a.d, RT_BM) || !make_map_bf16(&mw, a.w_split, 3 * NP, a.d, S::W_BOX))
         return cudaErrorInvalidValue;
     RtParams p{};
     const int nkb = (a.d + RT_BK - 1) / RT_BK;
+    // K groups of at most KB_PER_GROUP k-blocks (<= 64 MMAs per accumulator).
+    // Two accumulator buffers (the epilogue overlaps the next tile) when the
+    // groups fit in TMEM twice, or when fewer, larger groups of at most 72 MMAs
+    // do; otherwise one buffer with groups of <= 64 MMAs.
     int groups = (nkb + S::KB_PER_GROUP - 1) / S::KB_PER_GROUP;
-    if (groups > S::MAX_GROUPS) groups = S::MAX_GROUPS;
+    if (groups < 1) groups = 1;
+    const int max2 = S::TMEM_COLS / (2 * S::ACC_COLS);
+    int nbuf = 1;
+    if (groups <= max2) {
+        nbuf = 2;
+    } else if (max2 >= 1 && ((nkb + max2 - 1) / max2) * S::MMA_PER_KB <= 72) {
+        nbuf = 2;
+        groups = max2;
+    }
+    const int max_groups = S::TMEM_COLS / (nbuf * S::ACC_COLS);
+    if (groups > max_groups) groups = max_groups;   // d beyond this bound: more MMAs per accumulator
     p.T = a.T;
     p.N = a.N;
     p.k = a.k;
     p.d = a.d;
-    if (groups < 1) groups = 1;
     const int kbpg = (nkb + groups - 1) / groups;
     groups = (nkb + kbpg - 1) / kbpg;   // no empty group
+    p.nbuf = nbuf;
     p.groups = groups;
     p.kb_per_group = kbpg;
     p.b_r = a.b_r;
@@ -479,15 +527,16 @@ cudaError_t run_router_tc(const RouterArgs& a, cudaStream_t s, int sms) {
         return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, RtShape<NP>::SMEM_BYTES);
     });
     if (err != cudaSuccess) return err;
-    const int ntiles = (int)((a.T + RT_BM - 1) / RT_BM);
-    const int grid = ntiles < sms ? ntiles : sms;
-    kern<<<grid, RT_THREADS, S::SMEM_BYTES, s>>>(mx, mw, p);
-    return cudaGetLastError();
+    const int npairs = (int)((a.T + 2 * RT_BM - 1) / (2 * RT_BM));
+    const int grid = 2 * (npairs < sms / 2 ? npairs : sms / 2);
+    return launch_k(kern, dim3((unsigned)grid), dim3(RT_THREADS), S::SMEM_BYTES, s, 2, mx, mw, p);
 }
 
 }  // namespace
 
-int router_tc_padded_experts(int N) { return N <= 16 ? 16 : (N <= 32 ? 32 : (N <= 64 ? 64 : 128)); }
+// At least 32 padded experts: the pair MMA's N (3 NP merged, NP per part) is
+// then a multiple of 32.
+int router_tc_padded_experts(int N) { return N <= 32 ? 32 : (N <= 64 ? 64 : 128); }
 
 cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t s) {
     int sms = 0;
@@ -496,7 +545,6 @@ cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t s) {
     if (a.T == 0)   // no tokens: f, P and the aux loss are zero
         return launch_aux_finalize(a.part_cnt, a.part_psum, 0, a.N, a.T, a.alpha, a.f, a.P, a.aux, s);
     const int np = router_tc_padded_experts(a.N);
-    if (np == 16) return run_router_tc<16>(a, s, sms);
     if (np == 32) return run_router_tc<32>(a, s, sms);
     if (np == 64) return run_router_tc<64>(a, s, sms);
     return run_router_tc<128>(a, s, sms);
