@@ -147,6 +147,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     __shared__ int s_hist[NP];
+    __shared__ float s_bias[NP];   // b_r, 0 without a bias, -inf for padding experts
     __shared__ int s_last;
     __shared__ double s_fp[NP];
 
@@ -181,6 +182,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     tc_fence_after();
     pdl_wait();       // x, the W split and the workspace are ready from here on
     pdl_launch();
+    for (int e = tid; e < NP; e += RT_THREADS)
+        s_bias[e] = e < p.N ? (p.b_r ? p.b_r[e] : 0.f) : -INFINITY;   // padding experts never win
+    __syncthreads();
 
     const uint32_t tmem_base = s_tmem;
     const int ntiles = (int)((p.T + 2 * RT_BM - 1) / (2 * RT_BM));
@@ -298,9 +302,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             tc_fence_after();
             const int64_t t = (int64_t)tile * 2 * RT_BM + (int)rank * RT_BM + q * 32 + lane;
             const bool valid = t < p.T;
-            float v[NP];
+            float v[NP];   // logits: the bias, then the partial products in a fixed order
 #pragma unroll
-            for (int e = 0; e < NP; ++e) v[e] = 0.f;
+            for (int e = 0; e < NP; ++e) v[e] = s_bias[e];
             const uint32_t tbase =
                 tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * p.groups * S::ACC_COLS);
             for (int g = 0; g < p.groups; ++g) {   // partial logits of the K groups (and W parts), in order
@@ -323,14 +327,6 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             tc_fence_before();
             mbar_arrive_cluster_relaxed(acc ? tempty_leader1 : tempty_leader0);   // the accumulator is free again
 
-            if (p.b_r) {
-#pragma unroll
-                for (int e = 0; e < NP; ++e)
-                    if (e < N) v[e] += __ldg(p.b_r + e);
-            }
-#pragma unroll
-            for (int e = 0; e < NP; ++e)
-                if (e >= N) v[e] = -INFINITY;   // padding experts never win
             // first choice: the largest logit, lowest index among equals
             const float m = tree_max(v);
             const int i1 = tree_first(v, m);
@@ -341,8 +337,10 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 m2 = tree_max(v, i1);
                 i2 = tree_first(v, m2, i1);
             }
+            // v now holds exp(h - max) = 2^((h - max) log2 e)
+            constexpr float kLog2e = 1.4426950408889634f;
 #pragma unroll
-            for (int e = 0; e < NP; ++e) v[e] = (e < N) ? expf(v[e] - m) : 0.f;   // v now holds exp(h - max)
+            for (int e = 0; e < NP; ++e) v[e] = (e < N) ? exp2f((v[e] - m) * kLog2e) : 0.f;
             const float s = tree_sum(v);
             const float inv = valid ? 1.f / s : 0.f;
             if (valid) {
@@ -350,7 +348,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     p.idx[t] = i1;
                     p.gate[t] = inv;   // p_{i*} = exp(0) / s
                 } else {
-                    const float r = expf(m2 - m);
+                    const float r = exp2f((m2 - m) * kLog2e);
                     p.idx[2 * t] = i1;
                     p.idx[2 * t + 1] = i2;
                     p.gate[2 * t] = 1.f / (1.f + r);
