@@ -195,9 +195,11 @@ const char* moe_status_string(int32_t status) {
     }
 }
 
-int32_t moe_route(const moe_config* cfg, const void* x, const float* w_r, const float* b_r, int32_t* idx,
-                  float* gate, float* probs, double* f, double* P, double* aux, void* ws, size_t ws_bytes,
-                  void* stream) {
+// The router; with defer (tensor-core router only) its CTAs leave f, P and aux
+// to a later aux_reduce_block over their partials.
+static int32_t route_impl(const moe_config* cfg, const void* x, const float* w_r, const float* b_r, int32_t* idx,
+                          float* gate, float* probs, double* f, double* P, double* aux, void* ws, size_t ws_bytes,
+                          void* stream, bool defer) {
     int32_t st = validate(cfg);
     if (st != MOE_OK) return st;
     if (!req(w_r) || !opt(b_r) || !opt(probs) || !opt(f) || !opt(P) || !opt(aux)) return MOE_ERR_INVALID_ARG;
@@ -225,13 +227,20 @@ int32_t moe_route(const moe_config* cfg, const void* x, const float* w_r, const 
     a.w_split = at<void>(ws, L.w_split);
     a.status = &at<WsHeader>(ws, L.hdr)->status;
     a.ticket = &at<WsHeader>(ws, L.hdr)->route_ticket;
+    a.defer_aux = defer;
     return cuda_status(launch_router(a, (cudaStream_t)stream));
+}
+
+int32_t moe_route(const moe_config* cfg, const void* x, const float* w_r, const float* b_r, int32_t* idx,
+                  float* gate, float* probs, double* f, double* P, double* aux, void* ws, size_t ws_bytes,
+                  void* stream) {
+    return route_impl(cfg, x, w_r, b_r, idx, gate, probs, f, P, aux, ws, ws_bytes, stream, false);
 }
 
 static int32_t dispatch_impl(const moe_config* cfg, const void* x, const int32_t* idx, const float* gate,
                              int32_t* pos, uint8_t* drop, int32_t* counts, int32_t* kept, int32_t* offsets,
                              int32_t* row_token, float* row_gate, void* xe, void* zero_out, void* ws,
-                             cudaStream_t s, const int32_t* claim_base = nullptr) {
+                             cudaStream_t s, const int32_t* claim_base = nullptr, const AuxArgs* aux = nullptr) {
     const Layout L = layout_of(*cfg);
     if (cfg->T == 0) {
         cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->top_k * cfg->n_experts, s);
@@ -261,6 +270,7 @@ static int32_t dispatch_impl(const moe_config* cfg, const void* x, const int32_t
     a.scan_state = at<uint32_t>(ws, L.scan_state);
     a.hdr = at<WsHeader>(ws, L.hdr);
     a.claim_base = claim_base;
+    if (aux) a.aux = *aux;
     return cuda_status(launch_dispatch(a, s));
 }
 
@@ -443,14 +453,24 @@ static int32_t forward_impl(const moe_config* cfg, const void* x, const float* w
     void* ye = at<void>(ws, L.ye);
 
     if (!mark(0)) return MOE_ERR_CUDA;
-    st = moe_route(cfg, x, w_r, b_r, idx, gate, nullptr, f, P, aux, ws, ws_bytes, s);
+    // bf16: the router's CTAs leave the load-balancing loss to one extra block
+    // of the gather, which runs beside the HBM-bound row copies
+    const bool defer = cfg->dtype == MOE_BF16 && cfg->T > 0;
+    AuxArgs aa{};
+    if (defer && (f || P || aux)) {
+        int sms = 0;
+        if (device_sm_count(&sms) != cudaSuccess) return MOE_ERR_CUDA;
+        aa = AuxArgs{at<int32_t>(ws, L.part_cnt), at<float>(ws, L.part_psum), router_tc_grid(cfg->T, sms),
+                     (int)cfg->n_experts, cfg->T, cfg->alpha, f, P, aux};
+    }
+    st = route_impl(cfg, x, w_r, b_r, idx, gate, nullptr, f, P, aux, ws, ws_bytes, s, defer);
     if (st != MOE_OK) return st;
     if (!mark(1)) return MOE_ERR_CUDA;
     // top-1 bf16: the second GEMM scatters gate * E(x) into out; dispatch zeroes
     // the rows of dropped tokens.  Otherwise expert outputs go through the combine.
     const bool fused = cfg->dtype == MOE_BF16 && cfg->top_k == 1;
     st = dispatch_impl(cfg, x, idx, gate, pos, drop, counts, kept, offsets, row_token, row_gate, xe,
-                       fused ? out : nullptr, ws, s);
+                       fused ? out : nullptr, ws, s, nullptr, aa.G > 0 ? &aa : nullptr);
     if (st != MOE_OK) return st;
     if (!mark(2)) return MOE_ERR_CUDA;
     st = ffn_impl(cfg, xe, offsets, w1, b1, w3, b3, w2, b2, ye, fused ? out : nullptr, row_token, row_gate, ws, s,

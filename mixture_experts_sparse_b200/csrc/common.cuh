@@ -106,6 +106,77 @@ cudaError_t once_per_device(const void* key, cudaError_t (*set)(const void*));
 // Number of SMs of the current device (cached).
 cudaError_t device_sm_count(int* sms);
 
+// ---- load-balancing loss from per-CTA router partials -------------------------
+// "From Switch Transformer to GLaM", Load balancing: f_i = fraction of tokens
+// whose top-1 choice is i, P_i = mean router probability of i, aux = alpha N
+// sum_i f_i P_i.  part_cnt / part_psum hold, expert-major ([N][Gp], Gp = G
+// rounded up to 4), each router CTA's top-1 counts and sums of p.  The sums run
+// in fp64 in CTA order with a fixed partition over kAuxThreads threads, so every
+// caller obtains the same bits.
+struct AuxArgs {
+    const int32_t* part_cnt; const float* part_psum;
+    int G; int N; int64_t T; float alpha;   // G = 0: nothing to reduce
+    double* f; double* P; double* aux;      // each nullable
+};
+constexpr int kAuxThreads = 192;
+constexpr int kAuxScratch = 2 * kAuxThreads + 128;   // doubles of shared memory
+
+// Called by every thread of one block of at least kAuxThreads threads.
+__device__ inline void aux_reduce_block(const AuxArgs& a, double* scratch) {
+    const int tid = threadIdx.x;
+    const int N = a.N, G = a.G, Gp = (G + 3) & ~3, nch = Gp / 4;
+    const int tpe = kAuxThreads / N;   // threads per expert
+    const int e = tid / tpe, j = tid % tpe;
+    double* sp = scratch;
+    double* sc = sp + kAuxThreads;
+    double* sfp = sc + kAuxThreads;
+    double pa = 0.0, ca = 0.0;
+    if (tid < kAuxThreads && e < N) {   // this thread: chunks j, j + tpe, ... of 4 CTAs each, in order
+        const float4* ps4 = reinterpret_cast<const float4*>(a.part_psum + (int64_t)e * Gp);
+        const int4* cs4 = reinterpret_cast<const int4*>(a.part_cnt + (int64_t)e * Gp);
+        for (int c0 = j; c0 < nch; c0 += 4 * tpe) {
+            float4 pv[4];
+            int4 cv[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int c = c0 + u * tpe;
+                pv[u] = c < nch ? __ldcg(ps4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
+                cv[u] = c < nch ? __ldcg(cs4 + c) : make_int4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int b = 4 * (c0 + u * tpe);   // first CTA of the chunk
+                if (b + 0 < G) { pa += (double)pv[u].x; ca += (double)cv[u].x; }
+                if (b + 1 < G) { pa += (double)pv[u].y; ca += (double)cv[u].y; }
+                if (b + 2 < G) { pa += (double)pv[u].z; ca += (double)cv[u].z; }
+                if (b + 3 < G) { pa += (double)pv[u].w; ca += (double)cv[u].w; }
+            }
+        }
+    }
+    if (tid < kAuxThreads) {
+        sp[tid] = pa;
+        sc[tid] = ca;
+    }
+    __syncthreads();
+    if (tid < N) {
+        double pt = 0.0, ct = 0.0;
+        for (int q = 0; q < tpe; ++q) {
+            pt += sp[tid * tpe + q];
+            ct += sc[tid * tpe + q];
+        }
+        const double Pe = pt / (double)a.T, fe = ct / (double)a.T;
+        if (a.P) a.P[tid] = Pe;
+        if (a.f) a.f[tid] = fe;
+        sfp[tid] = fe * Pe;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        double s = 0.0;
+        for (int q = 0; q < N; ++q) s += sfp[q];
+        if (a.aux) *a.aux = (double)a.alpha * (double)N * s;
+    }
+}
+
 // ---- launchers implemented in the .cu files ---------------------------------
 struct RouterArgs {
     const void* x; int dtype; const float* w_r; const float* b_r;
@@ -116,7 +187,9 @@ struct RouterArgs {
     void* w_split;                         // bf16 [3, NP, d] scratch (tensor-core router)
     int32_t* ticket;                       // finished-CTA counter of the tensor-core router
     int32_t* status;
+    bool defer_aux;                        // tensor-core router: leave f, P, aux to aux_reduce_block
 };
+int router_tc_grid(int64_t T, int sms);            // CTAs of the tensor-core router (= partial rows used)
 int router_blocks(int64_t T, int N);               // partial rows the FP32-pipe router writes
 int router_partial_rows(int64_t T, int N);         // partial rows any router path writes
 int router_tc_padded_experts(int N);
@@ -139,6 +212,7 @@ struct DispatchArgs {
     void* zero_out;              // top-1 fused path: rows of dropped tokens are zeroed
     uint32_t* scan_state; WsHeader* hdr;
     const int32_t* claim_base;   // [k, N] claims made before this shard (sharded batch), or null
+    AuxArgs aux;                 // G > 0: one extra block of the gather reduces the router partials
 };
 int scan_blocks(int64_t T);
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s);

@@ -181,11 +181,18 @@ scatter_kernel(const XT* __restrict__ x, const int32_t* __restrict__ idx, const 
                int64_t T, int d, int N, int k, int C,
                const int32_t* __restrict__ claim_base, int32_t* __restrict__ pos, uint8_t* __restrict__ drop,
                const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets, int32_t* __restrict__ row_token,
-               float* __restrict__ row_gate, XT* __restrict__ xe, XT* __restrict__ zero_out) {
+               float* __restrict__ row_gate, XT* __restrict__ xe, XT* __restrict__ zero_out, const AuxArgs aux) {
     pdl_wait();
     pdl_launch();
+    // the extra block (the first, so it is scheduled at once and runs beside
+    // the row copies): load-balancing loss from the router's partials
+    if (aux.G > 0 && blockIdx.x == 0) {
+        __shared__ double s_aux[kAuxScratch];
+        aux_reduce_block(aux, s_aux);
+        return;
+    }
     const int lane = threadIdx.x & 31;
-    const int64_t a = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int64_t a = (int64_t)(blockIdx.x - (aux.G > 0 ? 1 : 0)) * 8 + (threadIdx.x >> 5);
     if (a >= T * k) return;
     const int64_t t = a / k;
     const int r = (int)(a - t * k);
@@ -318,15 +325,15 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
                    a.claim_base, a.pos, a.counts, a.kept, a.offsets, a.scan_state, a.hdr, kWaitLimitNs);
     if (err != cudaSuccess) return err;
     const int64_t warps = a.T * a.k;
-    const unsigned grid = (unsigned)((warps + 7) / 8);
+    const unsigned grid = (unsigned)((warps + 7) / 8) + (a.aux.G > 0 ? 1u : 0u);
     if (a.dtype == MOE_BF16)
         return launch_k(scatter_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, 1,
                         reinterpret_cast<const __nv_bfloat16*>(a.x), a.idx, a.gate, a.T, a.d, a.N, a.k, a.C,
                         a.claim_base, a.pos, a.drop, a.counts, a.offsets, a.row_token, a.row_gate,
-                        reinterpret_cast<__nv_bfloat16*>(a.xe), reinterpret_cast<__nv_bfloat16*>(a.zero_out));
+                        reinterpret_cast<__nv_bfloat16*>(a.xe), reinterpret_cast<__nv_bfloat16*>(a.zero_out), a.aux);
     return launch_k(scatter_kernel<float>, dim3(grid), dim3(256), 0, s, 1, reinterpret_cast<const float*>(a.x), a.idx,
                     a.gate, a.T, a.d, a.N, a.k, a.C, a.claim_base, a.pos, a.drop, a.counts, a.offsets, a.row_token,
-                    a.row_gate, reinterpret_cast<float*>(a.xe), reinterpret_cast<float*>(a.zero_out));
+                    a.row_gate, reinterpret_cast<float*>(a.xe), reinterpret_cast<float*>(a.zero_out), a.aux);
 }
 
 cudaError_t launch_counts(const int32_t* idx, int64_t T, int N, int k, int32_t* counts, cudaStream_t s) {

@@ -87,6 +87,7 @@ struct RtParams {
     float alpha;
     int32_t* ticket;      // finished-CTA counter, 0 between calls
     int32_t* status;
+    int defer_aux;        // 1: the partials are reduced later (aux_reduce_block elsewhere)
     long long limit_ns;
 };
 
@@ -149,7 +150,6 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     __shared__ int s_hist[NP];
     __shared__ float s_bias[NP];   // b_r, 0 without a bias, -inf for padding experts
     __shared__ int s_last;
-    __shared__ double s_fp[NP];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t rank = cluster_ctarank();   // 0 = the pair's leader
@@ -389,62 +389,15 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     tc_fence_after();
     if (warp == 1) tmem_dealloc_pair(tmem_base, S::TMEM_COLS);
 
+    if (p.defer_aux) return;
     // ---- the last CTA to finish reduces every CTA's partials: f, P, aux ----
     if (tid == 0) s_last = (atomicAdd(p.ticket, 1) == (int)gridDim.x - 1);
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    {
-        const int N = p.N, G = (int)gridDim.x, Gp = (G + 3) & ~3, nch = Gp / 4;
-        const int tpe = RT_THREADS / N;   // threads per expert
-        const int e = tid / tpe, j = tid % tpe;
-        double* sp = reinterpret_cast<double*>(smem);   // pipeline buffers are free now
-        double* sc = sp + RT_THREADS;
-        double pa = 0.0, ca = 0.0;
-        if (e < N) {   // this thread: chunks j, j + tpe, ... of 4 CTAs each, in order
-            const float4* ps4 = reinterpret_cast<const float4*>(p.part_psum + (int64_t)e * Gp);
-            const int4* cs4 = reinterpret_cast<const int4*>(p.part_cnt + (int64_t)e * Gp);
-            for (int c0 = j; c0 < nch; c0 += 4 * tpe) {
-                float4 pv[4];
-                int4 cv[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int c = c0 + u * tpe;
-                    pv[u] = c < nch ? __ldcg(ps4 + c) : make_float4(0.f, 0.f, 0.f, 0.f);
-                    cv[u] = c < nch ? __ldcg(cs4 + c) : make_int4(0, 0, 0, 0);
-                }
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const int b = 4 * (c0 + u * tpe);   // first CTA of the chunk
-                    if (b + 0 < G) { pa += (double)pv[u].x; ca += (double)cv[u].x; }
-                    if (b + 1 < G) { pa += (double)pv[u].y; ca += (double)cv[u].y; }
-                    if (b + 2 < G) { pa += (double)pv[u].z; ca += (double)cv[u].z; }
-                    if (b + 3 < G) { pa += (double)pv[u].w; ca += (double)cv[u].w; }
-                }
-            }
-        }
-        sp[tid] = pa;
-        sc[tid] = ca;
-        __syncthreads();
-        if (tid < N) {
-            double pt = 0.0, ct = 0.0;
-            for (int q2 = 0; q2 < tpe; ++q2) {
-                pt += sp[tid * tpe + q2];
-                ct += sc[tid * tpe + q2];
-            }
-            const double Pe = pt / (double)p.T, fe = ct / (double)p.T;
-            if (p.P) p.P[tid] = Pe;
-            if (p.f) p.f[tid] = fe;
-            s_fp[tid] = fe * Pe;
-        }
-        __syncthreads();
-        if (tid == 0) {
-            double sfp = 0.0;
-            for (int q2 = 0; q2 < N; ++q2) sfp += s_fp[q2];
-            if (p.aux) *p.aux = (double)p.alpha * (double)N * sfp;
-            *p.ticket = 0;   // ready for the next call
-        }
-    }
+    const AuxArgs aa{p.part_cnt, p.part_psum, (int)gridDim.x, p.N, p.T, p.alpha, p.f, p.P, p.aux};
+    aux_reduce_block(aa, reinterpret_cast<double*>(smem));   // pipeline buffers are free now
+    if (tid == 0) *p.ticket = 0;                             // ready for the next call
 }
 
 // fp32 [N, d] -> bf16 [3, NP, d]: w = w0 + w1 + w2 exactly; rows >= N are zero.
@@ -519,18 +472,23 @@ cudaError_t run_router_tc(const RouterArgs& a, cudaStream_t s, int sms) {
     p.alpha = a.alpha;
     p.ticket = a.ticket;
     p.status = a.status;
+    p.defer_aux = a.defer_aux ? 1 : 0;
     p.limit_ns = kWaitLimitNs;
     auto kern = router_tc_kernel<NP>;
     err = once_per_device(reinterpret_cast<const void*>(kern), [](const void* k) {
         return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, RtShape<NP>::SMEM_BYTES);
     });
     if (err != cudaSuccess) return err;
-    const int npairs = (int)((a.T + 2 * RT_BM - 1) / (2 * RT_BM));
-    const int grid = 2 * (npairs < sms / 2 ? npairs : sms / 2);
+    const int grid = router_tc_grid(a.T, sms);
     return launch_k(kern, dim3((unsigned)grid), dim3(RT_THREADS), S::SMEM_BYTES, s, 2, mx, mw, p);
 }
 
 }  // namespace
+
+int router_tc_grid(int64_t T, int sms) {
+    const int64_t npairs = (T + 2 * RT_BM - 1) / (2 * RT_BM);
+    return 2 * (int)(npairs < sms / 2 ? npairs : sms / 2);
+}
 
 // At least 32 padded experts: the pair MMA's N (3 NP merged, NP per part) is
 // then a multiple of 32.
