@@ -42,6 +42,8 @@ def _load():
         lib.oracle_router.restype = None
         lib.oracle_aux.argtypes = [i64, i32, i32, P, P, f64, P, P, P]
         lib.oracle_aux.restype = None
+        lib.oracle_z_loss.argtypes = [i64, i32, P]
+        lib.oracle_z_loss.restype = f64
         lib.oracle_capacity.argtypes = [i64, i32, i32, f64]
         lib.oracle_capacity.restype = i32
         lib.oracle_dispatch.argtypes = [i64, i32, i32, i32, P, P, P, P, P, P]
@@ -121,6 +123,17 @@ def route(x, w_r, b_r=None, k=1):
     lib.oracle_router(T, d, N, k, _ptr(x), xd, _ptr(w_r), _ptr(b), _ptr(logits), _ptr(probs),
                       _ptr(idx), _ptr(gate))
     return dict(logits=logits, probs=probs, idx=idx, gate=gate)
+
+
+def z_loss(logits):
+    """Router z-loss: the mean over tokens of (log sum_i exp h_i)^2 over the
+    fp32 router logits (CMU 10-423 Lecture 16, section 4.2, "router z-loss";
+    the page's formula is not legible, its experiment reports the router's
+    logsumexp^2 -- this is that reading, unweighted)."""
+    lib = _load()
+    logits = np.ascontiguousarray(logits, dtype=np.float32)
+    T, N = logits.shape
+    return float(lib.oracle_z_loss(T, N, _ptr(logits)))
 
 
 def aux_loss(idx, probs, alpha=1e-2):

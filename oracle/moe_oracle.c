@@ -156,6 +156,31 @@ void oracle_router(int64_t T, int32_t d, int32_t N, int32_t k,
     }
 }
 
+/* ---- Router z-loss --------------------------------------------------------
+ * CMU 10-423 Lecture 16, section 4.2 ("router z-loss", Zoph et al. 2022): a
+ * penalty on large router logits; the page's formula is not legible, and its
+ * experiment reports the router's "logsumexp^2".  Reading taken:
+ *   z = (1/T) sum_t ( log sum_i exp(h_{t,i}) )^2
+ * over the fp32 router logits h (the values oracle_router writes), without the
+ * weight (0.001 in OLMoE), which the caller applies.  log-sum-exp is taken as
+ * m + log sum_i exp(h_i - m), m = max_i h_i, in double.  T = 0 gives 0. */
+double oracle_z_loss(int64_t T, int32_t N, const float* logits) {
+    if (T <= 0) return 0.0;
+    double acc = 0.0;
+    for (int64_t t = 0; t < T; ++t) {
+        const float* h = logits + (size_t)t * N;
+        double m = (double)h[0];
+        for (int32_t i = 1; i < N; ++i) {
+            if ((double)h[i] > m) m = (double)h[i];
+        }
+        double s = 0.0;
+        for (int32_t i = 0; i < N; ++i) s += exp((double)h[i] - m);
+        const double lse = m + log(s);
+        acc += lse * lse;
+    }
+    return acc / (double)T;
+}
+
 /* ---- Load-balancing loss -------------------------------------------------
  * f_i = #{t : top-1 choice of t is i} / T   (pre-capacity, argmax indicator)
  * P_i = sum_t p_{t,i} / T

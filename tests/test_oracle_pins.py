@@ -176,6 +176,45 @@ def test_aux_empty_batch():
 
 # ------------------------------------------------------------- capacity -----
 
+# ---------------------------------------------------------------- z-loss ----
+
+def test_z_loss_uniform_router_closed_form():
+    # equal logits c on N experts: log sum exp = c + ln N for every token
+    for N, c in [(1, 0.0), (8, 0.0), (64, 0.0), (8, 1.5), (128, -3.25)]:
+        logits = np.full((5, N), c, np.float32)
+        assert oracle.z_loss(logits) == pytest.approx((c + math.log(N)) ** 2, rel=1e-15, abs=1e-15)
+
+
+def test_z_loss_matches_library_logsumexp():
+    from scipy.special import logsumexp
+    rng = np.random.default_rng(3)
+    logits = (rng.standard_normal((37, 11)) * 4.0).astype(np.float32)
+    want = np.mean(logsumexp(logits.astype(np.float64), axis=1) ** 2)
+    assert oracle.z_loss(logits) == pytest.approx(want, rel=1e-13)
+
+
+def test_z_loss_large_logits_and_shift():
+    # max-shifted evaluation: huge logits do not overflow; a shift by c moves
+    # every token's log-sum-exp by c; permuting experts changes nothing
+    logits = np.array([[1000.0, 999.0, -5.0], [-1000.0, -1000.0, -1000.0]], np.float32)
+    l0 = 1000.0 + math.log(1.0 + math.exp(-1.0) + math.exp(-1005.0))
+    l1 = -1000.0 + math.log(3.0)
+    assert oracle.z_loss(logits) == pytest.approx((l0 * l0 + l1 * l1) / 2, rel=1e-14)
+    # one token at a time, logits >= 4 so every log-sum-exp is positive:
+    # sqrt(z) is the log-sum-exp, and a shift by c adds c to it
+    rng = np.random.default_rng(5)
+    h = (4.0 + rng.random((9, 6))).astype(np.float32)
+    c = np.float32(2.0)
+    for t in range(9):
+        one = h[t:t + 1]
+        assert math.sqrt(oracle.z_loss(one + c)) == pytest.approx(math.sqrt(oracle.z_loss(one)) + 2.0, rel=1e-12)
+    assert oracle.z_loss(h[:, ::-1].copy()) == pytest.approx(oracle.z_loss(h), rel=1e-14)
+
+
+def test_z_loss_empty_batch():
+    assert oracle.z_loss(np.zeros((0, 4), np.float32)) == 0.0
+
+
 def test_capacity_exercise(golden):
     g = golden("capacity_exercise.txt")
     C = oracle.capacity(g["T"], g["N"], g["k"], g["cf"])
