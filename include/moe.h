@@ -117,6 +117,19 @@ int32_t moe_route(const moe_config* cfg, const void* x, const float* w_r, const 
                   double* f, double* P, double* aux,
                   void* ws, size_t ws_bytes, void* stream);
 
+/* moe_route plus the router z-loss (CMU 10-423 Lecture 16, section 4.2,
+ * "router z-loss", Zoph et al. 2022: a penalty on large router logits; the
+ * page's formula is not legible and its experiment reports the router's
+ * logsumexp^2, so z is read as the mean over tokens of
+ * (log sum_e exp h_{t,e})^2 over the fp32 logits h, unweighted -- the caller
+ * applies its coefficient, 0.001 in OLMoE).  Out: z_loss [1] fp64 (nullable);
+ * 0 for T = 0.  Per-token values are summed in fp64 in a fixed order.  The
+ * other arguments and outputs are those of moe_route. */
+int32_t moe_route_z(const moe_config* cfg, const void* x, const float* w_r, const float* b_r,
+                    int32_t* idx, float* gate, float* probs,
+                    double* f, double* P, double* aux, double* z_loss,
+                    void* ws, size_t ws_bytes, void* stream);
+
 /* Capacity-limited dispatch (row A3 and the gather of A4).
  * In:  x [T, d] (dtype; nullable when xe is NULL), idx [T, k], gate [T, k].
  * Out: pos [T, k] int32 (claim number of the assignment on its expert: all

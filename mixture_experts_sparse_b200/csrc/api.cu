@@ -56,7 +56,7 @@ namespace {
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
 struct Layout {
-    size_t hdr, part_cnt, part_psum, w_split, scan_state;
+    size_t hdr, part_cnt, part_psum, part_z, w_split, scan_state;
     size_t idx, gate, pos, drop, counts, kept, offsets, f, P, aux;
     size_t row_token, row_gate, xe, h, ye;
     size_t total;
@@ -85,6 +85,7 @@ Layout layout_of(const moe_config& c) {
     const size_t nbr = (size_t)router_partial_rows(c.T, c.n_experts);
     L.part_cnt = take(4 * nbr * N);
     L.part_psum = take(4 * nbr * N);
+    L.part_z = take(8 * nbr);
     L.w_split = take(c.dtype == MOE_BF16 ? 2 * 3 * (size_t)router_tc_padded_experts(c.n_experts) * c.d_model : 0);
     const size_t nbs = (size_t)scan_blocks(c.T);
     L.scan_state = take(4 * (nbs * k * N > 8 ? nbs * k * N : 8));
@@ -199,7 +200,7 @@ const char* moe_status_string(int32_t status) {
 // to a later aux_reduce_block over their partials.
 static int32_t route_impl(const moe_config* cfg, const void* x, const float* w_r, const float* b_r, int32_t* idx,
                           float* gate, float* probs, double* f, double* P, double* aux, void* ws, size_t ws_bytes,
-                          void* stream, bool defer) {
+                          void* stream, bool defer, double* z = nullptr) {
     int32_t st = validate(cfg);
     if (st != MOE_OK) return st;
     if (!req(w_r) || !opt(b_r) || !opt(probs) || !opt(f) || !opt(P) || !opt(aux)) return MOE_ERR_INVALID_ARG;
@@ -220,6 +221,8 @@ static int32_t route_impl(const moe_config* cfg, const void* x, const float* w_r
     a.probs = probs;
     a.part_cnt = at<int32_t>(ws, L.part_cnt);
     a.part_psum = at<float>(ws, L.part_psum);
+    a.part_z = at<double>(ws, L.part_z);
+    a.z = z;
     a.f = f;
     a.P = P;
     a.aux = aux;
@@ -235,6 +238,13 @@ int32_t moe_route(const moe_config* cfg, const void* x, const float* w_r, const 
                   float* gate, float* probs, double* f, double* P, double* aux, void* ws, size_t ws_bytes,
                   void* stream) {
     return route_impl(cfg, x, w_r, b_r, idx, gate, probs, f, P, aux, ws, ws_bytes, stream, false);
+}
+
+int32_t moe_route_z(const moe_config* cfg, const void* x, const float* w_r, const float* b_r, int32_t* idx,
+                    float* gate, float* probs, double* f, double* P, double* aux, double* z_loss, void* ws,
+                    size_t ws_bytes, void* stream) {
+    if (!opt(z_loss)) return MOE_ERR_INVALID_ARG;
+    return route_impl(cfg, x, w_r, b_r, idx, gate, probs, f, P, aux, ws, ws_bytes, stream, false, z_loss);
 }
 
 static int32_t dispatch_impl(const moe_config* cfg, const void* x, const int32_t* idx, const float* gate,

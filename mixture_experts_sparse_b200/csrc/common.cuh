@@ -117,9 +117,23 @@ struct AuxArgs {
     const int32_t* part_cnt; const float* part_psum;
     int G; int N; int64_t T; float alpha;   // G = 0: nothing to reduce
     double* f; double* P; double* aux;      // each nullable
+    const double* part_z; double* z;        // router z-loss: per-CTA sums of lse^2 -> mean (z nullable)
 };
 constexpr int kAuxThreads = 192;
 constexpr int kAuxScratch = 2 * kAuxThreads + 128;   // doubles of shared memory
+
+// Router z-loss (CMU 10-423 Lecture 16, section 4.2, read as the mean over
+// tokens of the squared log-sum-exp of the router logits) from per-CTA sums:
+// called by one full warp; lane j adds partials j, j + 32, ... in order, then a
+// fixed shuffle tree; z = total / T (0 for T = 0).
+__device__ inline void z_reduce_warp(const double* part_z, int G, int64_t T, double* z) {
+    const int lane = threadIdx.x & 31;
+    double acc = 0.0;
+    for (int g = lane; g < G; g += 32) acc += __ldcg(part_z + g);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) *z = T > 0 ? acc / (double)T : 0.0;
+}
 
 // Called by every thread of one block of at least kAuxThreads threads.
 __device__ inline void aux_reduce_block(const AuxArgs& a, double* scratch) {
@@ -175,6 +189,7 @@ __device__ inline void aux_reduce_block(const AuxArgs& a, double* scratch) {
         for (int q = 0; q < N; ++q) s += sfp[q];
         if (a.aux) *a.aux = (double)a.alpha * (double)N * s;
     }
+    if (a.z && tid < 32) z_reduce_warp(a.part_z, G, a.T, a.z);
 }
 
 // ---- launchers implemented in the .cu files ---------------------------------
@@ -184,6 +199,7 @@ struct RouterArgs {
     int32_t* idx; float* gate; float* probs;
     int32_t* part_cnt; float* part_psum;   // [nblk, N]
     double* f; double* P; double* aux; float alpha;
+    double* part_z; double* z;             // router z-loss (z nullable; part_z [nblk] when z is set)
     void* w_split;                         // bf16 [3, NP, d] scratch (tensor-core router)
     int32_t* ticket;                       // finished-CTA counter of the tensor-core router
     int32_t* status;
@@ -195,7 +211,8 @@ int router_partial_rows(int64_t T, int N);         // partial rows any router pa
 int router_tc_padded_experts(int N);
 cudaError_t launch_router(const RouterArgs& a, cudaStream_t s);
 cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t s);
-cudaError_t launch_aux_finalize(const int32_t* part_cnt, const float* part_psum, int nblk, int N, int64_t T,
+cudaError_t launch_aux_finalize(const double* part_z, double* z, const int32_t* part_cnt, const float* part_psum,
+                                int nblk, int N, int64_t T,
                                 float alpha, double* f, double* P, double* aux, cudaStream_t s);
 
 // Number of claims numbered base, base+1, ..., base+count-1 that fall below C.

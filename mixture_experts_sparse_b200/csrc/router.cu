@@ -48,7 +48,7 @@ __global__ void __launch_bounds__(kThreads)
 router_kernel(const XT* __restrict__ x, const float* __restrict__ w_r, const float* __restrict__ b_r,
               int64_t T, int d, int N, int k,
               int32_t* __restrict__ idx, float* __restrict__ gate, float* __restrict__ probs,
-              int32_t* __restrict__ part_cnt, float* __restrict__ part_psum) {
+              int32_t* __restrict__ part_cnt, float* __restrict__ part_psum, double* __restrict__ part_z) {
     using S = RouterShape<TE, EG>;
     constexpr int VEC = 16 / sizeof(XT);          // elements per 16-byte load
     constexpr int PARTS = kDK / VEC;              // 16-byte loads per row chunk
@@ -63,6 +63,7 @@ router_kernel(const XT* __restrict__ x, const float* __restrict__ w_r, const flo
     float* lg = smem;               // [TB][NP + 1] after the main loop
     __shared__ int s_cnt[128];
     __shared__ float s_part[kThreads];
+    __shared__ double s_zw[kThreads / 32];   // per warp: sum of lse^2 over its tokens
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int eg = warp % EG, tg = warp / EG;
@@ -163,6 +164,7 @@ router_kernel(const XT* __restrict__ x, const float* __restrict__ w_r, const flo
     constexpr int MPL = (S::NP + 31) / 32;
     const int64_t rem_t = T - t0;
     const int tb_valid = rem_t < (int64_t)S::TB ? (int)rem_t : S::TB;
+    double zacc = 0.0;   // lane 0: sum over this warp's tokens of log-sum-exp^2
     for (int tok = warp; tok < tb_valid; tok += kThreads / 32) {
         float* row = lg + tok * (S::NP + 1);
         float v[MPL];
@@ -229,6 +231,8 @@ router_kernel(const XT* __restrict__ x, const float* __restrict__ w_r, const flo
             }
         }
         if (lane == 0) {
+            const float lse = m + logf(s);   // log sum_e exp(h_e)
+            zacc += (double)lse * (double)lse;
             atomicAdd(&s_cnt[bi], 1);
             if (k == 1) {
                 idx[t] = bi;
@@ -242,7 +246,13 @@ router_kernel(const XT* __restrict__ x, const float* __restrict__ w_r, const flo
             }
         }
     }
+    if (lane == 0) s_zw[warp] = zacc;
     __syncthreads();
+    if (part_z && tid == 0) {
+        double zs = 0.0;
+        for (int w = 0; w < kThreads / 32; ++w) zs += s_zw[w];
+        part_z[blockIdx.x] = zs;
+    }
 
     // ---- block partials in a fixed order: sum_t p[t][e], count of top-1 == e ----
     int npow = 8;
@@ -269,7 +279,8 @@ router_kernel(const XT* __restrict__ x, const float* __restrict__ w_r, const flo
 
 // f_i, P_i, aux from the per-block partials; fp64, fixed reduction order.
 __global__ void __launch_bounds__(1024)
-aux_finalize_kernel(const int32_t* __restrict__ part_cnt, const float* __restrict__ part_psum,
+aux_finalize_kernel(const double* __restrict__ part_z, double* __restrict__ z,
+                    const int32_t* __restrict__ part_cnt, const float* __restrict__ part_psum,
                     int nblk, int N, int64_t T, float alpha,
                     double* __restrict__ f, double* __restrict__ P, double* __restrict__ aux) {
     __shared__ double sp[1024];
@@ -322,6 +333,7 @@ aux_finalize_kernel(const int32_t* __restrict__ part_cnt, const float* __restric
         for (int q = 0; q < N; ++q) s += sfp[q];
         *aux = (double)alpha * (double)N * s;
     }
+    if (z && tid < 32) z_reduce_warp(part_z, nblk, T, z);
 }
 
 template <typename XT, int TE, int EG>
@@ -337,10 +349,11 @@ cudaError_t launch_router_t(const RouterArgs& a, cudaStream_t s) {
     if (err != cudaSuccess) return err;
     if (nblk > 0) {
         err = launch_k(kern, dim3((unsigned)nblk), dim3(kThreads), smem, s, 1, reinterpret_cast<const XT*>(a.x), a.w_r,
-                       a.b_r, a.T, a.d, a.N, a.k, a.idx, a.gate, a.probs, a.part_cnt, a.part_psum);
+                       a.b_r, a.T, a.d, a.N, a.k, a.idx, a.gate, a.probs, a.part_cnt, a.part_psum,
+                       a.z ? a.part_z : nullptr);
         if (err != cudaSuccess) return err;
     }
-    return launch_aux_finalize(a.part_cnt, a.part_psum, nblk, a.N, a.T, a.alpha, a.f, a.P, a.aux, s);
+    return launch_aux_finalize(a.part_z, a.z, a.part_cnt, a.part_psum, nblk, a.N, a.T, a.alpha, a.f, a.P, a.aux, s);
 }
 
 template <typename XT>
@@ -369,10 +382,11 @@ int router_partial_rows(int64_t T, int N) {
     return tc_rows > simt_rows ? tc_rows : simt_rows;
 }
 
-cudaError_t launch_aux_finalize(const int32_t* part_cnt, const float* part_psum, int nblk, int N, int64_t T,
-                                float alpha, double* f, double* P, double* aux, cudaStream_t s) {
-    return launch_k(aux_finalize_kernel, dim3(1), dim3(1024), 0, s, 1, part_cnt, part_psum, nblk, N, T, alpha, f, P,
-                    aux);
+cudaError_t launch_aux_finalize(const double* part_z, double* z, const int32_t* part_cnt, const float* part_psum,
+                                int nblk, int N, int64_t T, float alpha, double* f, double* P, double* aux,
+                                cudaStream_t s) {
+    return launch_k(aux_finalize_kernel, dim3(1), dim3(1024), 0, s, 1, part_z, z, part_cnt, part_psum, nblk, N, T,
+                    alpha, f, P, aux);
 }
 
 // bf16 activations: the tensor-core router (exact three-way split of W_r);

@@ -88,6 +88,8 @@ struct RtParams {
     int32_t* ticket;      // finished-CTA counter, 0 between calls
     int32_t* status;
     int defer_aux;        // 1: the partials are reduced later (aux_reduce_block elsewhere)
+    double* part_z;       // [Gp] per-CTA sums of lse^2 (null: no z-loss)
+    double* z;
     long long limit_ns;
 };
 
@@ -149,6 +151,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     __shared__ int s_abort;
     __shared__ int s_hist[NP];
     __shared__ float s_bias[NP];   // b_r, 0 without a bias, -inf for padding experts
+    __shared__ double s_z[128];    // per epilogue thread: sum of lse^2 over its tokens
     __shared__ int s_last;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -294,6 +297,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         const uint32_t tempty_leader0 = map_to_rank(smem_u32(&tempty_bar[0]), 0);
         const uint32_t tempty_leader1 = map_to_rank(smem_u32(&tempty_bar[1]), 0);
         int it = 0;
+        double zacc = 0.0;   // sum over this thread's tokens of log-sum-exp^2
         for (int tile = first_tile; tile < ntiles; tile += tile_step, ++it) {
             const int acc = p.nbuf == 2 ? (it & 1) : 0;
             const uint32_t acc_par = (uint32_t)(p.nbuf == 2 ? ((it >> 1) & 1) : (it & 1));
@@ -344,6 +348,8 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             const float s = tree_sum(v);
             const float inv = valid ? 1.f / s : 0.f;
             if (valid) {
+                const float lse = m + logf(s);   // log sum_e exp(h_e)
+                zacc += (double)lse * (double)lse;
                 if (k == 1) {
                     p.idx[t] = i1;
                     p.gate[t] = inv;   // p_{i*} = exp(0) / s
@@ -365,8 +371,14 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             for (int e = 0; e < NP; ++e) prow[e] += v[e] * inv;   // this thread's tokens, in tile order
         }
         // ---- this CTA's partials, expert-major: part[e][blockIdx.x] ----
-        named_bar(1, 128);
         const int et = tid - 64;   // 0..127 across the four epilogue warps
+        s_z[et] = zacc;
+        named_bar(1, 128);
+        if (et == 0 && p.part_z) {   // fixed order: warp quadrant, then lane
+            double zs = 0.0;
+            for (int r = 0; r < 128; ++r) zs += s_z[r];
+            p.part_z[blockIdx.x] = zs;
+        }
         const int Gp = ((int)gridDim.x + 3) & ~3;
         if (et < N) {
             float ps = 0.f;   // fixed order: warp quadrant, then lane
@@ -395,7 +407,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    const AuxArgs aa{p.part_cnt, p.part_psum, (int)gridDim.x, p.N, p.T, p.alpha, p.f, p.P, p.aux};
+    const AuxArgs aa{p.part_cnt, p.part_psum, (int)gridDim.x, p.N, p.T, p.alpha, p.f, p.P, p.aux, p.part_z, p.z};
     aux_reduce_block(aa, reinterpret_cast<double*>(smem));   // pipeline buffers are free now
     if (tid == 0) *p.ticket = 0;                             // ready for the next call
 }
@@ -473,6 +485,8 @@ cudaError_t run_router_tc(const RouterArgs& a, cudaStream_t s, int sms) {
     p.ticket = a.ticket;
     p.status = a.status;
     p.defer_aux = a.defer_aux ? 1 : 0;
+    p.part_z = a.z ? a.part_z : nullptr;
+    p.z = a.z;
     p.limit_ns = kWaitLimitNs;
     auto kern = router_tc_kernel<NP>;
     err = once_per_device(reinterpret_cast<const void*>(kern), [](const void* k) {
@@ -499,7 +513,7 @@ cudaError_t launch_router_tc(const RouterArgs& a, cudaStream_t s) {
     cudaError_t err = device_sm_count(&sms);
     if (err != cudaSuccess) return err;
     if (a.T == 0)   // no tokens: f, P and the aux loss are zero
-        return launch_aux_finalize(a.part_cnt, a.part_psum, 0, a.N, a.T, a.alpha, a.f, a.P, a.aux, s);
+        return launch_aux_finalize(a.part_z, a.z, a.part_cnt, a.part_psum, 0, a.N, a.T, a.alpha, a.f, a.P, a.aux, s);
     const int np = router_tc_padded_experts(a.N);
     if (np == 32) return run_router_tc<32>(a, s, sms);
     if (np == 64) return run_router_tc<64>(a, s, sms);

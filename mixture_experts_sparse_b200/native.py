@@ -39,6 +39,7 @@ _SIGS = {
     "moe_status_string": ([ctypes.c_int32], ctypes.c_char_p),
     "moe_workspace_init": ([_P, ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_route": ([ctypes.POINTER(MoeConfig)] + [_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_route_z": ([ctypes.POINTER(MoeConfig)] + [_P] * 11 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_dispatch": ([ctypes.POINTER(MoeConfig)] + [_P] * 12 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_expert_ffn": ([ctypes.POINTER(MoeConfig)] + [_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_combine": ([ctypes.POINTER(MoeConfig)] + [_P] * 8, ctypes.c_int32),
@@ -134,6 +135,11 @@ def moe_status_string(status):
 def moe_route(cfg, x, w_r, b_r, idx, gate, probs, f, P, aux, ws, stream=None):
     return lib().moe_route(ctypes.byref(cfg), _p(x), _p(w_r), _p(b_r), _p(idx), _p(gate), _p(probs),
                            _p(f), _p(P), _p(aux), _p(ws), _nbytes(ws), _s(stream))
+
+
+def moe_route_z(cfg, x, w_r, b_r, idx, gate, probs, f, P, aux, z_loss, ws, stream=None):
+    return lib().moe_route_z(ctypes.byref(cfg), _p(x), _p(w_r), _p(b_r), _p(idx), _p(gate), _p(probs),
+                             _p(f), _p(P), _p(aux), _p(z_loss), _p(ws), _nbytes(ws), _s(stream))
 
 
 def moe_dispatch(cfg, x, idx, gate, pos, drop, counts, kept, offsets, row_token, row_gate, xe, ws,

@@ -279,6 +279,12 @@ def test_workload_full_size(name):
     # every token with no kept assignment is exactly zero, at any size
     all_drop = dd["drop"].all(axis=1)
     assert np.all(got[all_drop] == 0.0)
+    # router z-loss at full size, against the oracle's logits
+    z = torch.empty(1, dtype=torch.float64, device="cuda")
+    x = to_device(L["x"])
+    nat.check(nat.moe_route_z(layer.cfg, x, layer.w["w_r"], layer.w["b_r"], layer.idx, layer.gate, None, None,
+                              None, None, z, layer.ws))
+    assert_rel(z.item(), oracle.z_loss(r["logits"]), REL_PROB, "z-loss")
 
 
 def test_mixtral_literal_capacity():
