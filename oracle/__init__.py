@@ -47,6 +47,7 @@ def _load():
         lib.oracle_capacity.argtypes = [i64, i32, i32, f64]
         lib.oracle_capacity.restype = i32
         lib.oracle_dispatch.argtypes = [i64, i32, i32, i32, P, P, P, P, P, P]
+        lib.oracle_dispatch_ordered.argtypes = [i64, i32, i32, i32, P, P, P, P, P, P, P]
         lib.oracle_dispatch.restype = None
         lib.oracle_expert_ffn.argtypes = [i32, i32, i32, P, i32, sz, P, P, P, P, P, P, i32,
                                           sz, sz, sz, sz, P, P]
@@ -157,10 +158,25 @@ def capacity(T, N, k, cf):
     return int(_load().oracle_capacity(int(T), int(N), int(k), float(cf)))
 
 
-def dispatch(idx, N, C):
+def priority_order(gate):
+    """Batch-priority claim order: tokens by descending priority score, ties to
+    the lower token index.  CS25 Lecture 05 notes, section "from language MoE
+    to Vision MoE": with a capacity factor below 1, priority routing first
+    scores each token's importance and lets the high-priority tokens take the
+    expert slots.  The score read here is the token's first-choice gate
+    gate[t, 0] (the router's weight for its first choice), compared as fp32."""
+    g0 = np.ascontiguousarray(np.asarray(gate, np.float32)[:, 0])
+    T = g0.shape[0]
+    return np.lexsort((np.arange(T), -g0.astype(np.float64))).astype(np.int64)
+
+
+def dispatch(idx, N, C, priority=None):
     """Capacity-limited slot claim: rank-major, then token order (CS25 Lecture 05
     notes, capacity-aware dispatch; CMU 10-423 Lecture 16 section 6.1, GShard
-    rule).  Returns dict(pos, drop, counts[k,N], kept[N], offsets[N+1])."""
+    rule), or with priority=gate [T, k] the batch-priority order of
+    priority_order(gate) (CS25 Lecture 05 notes, section "from language MoE to
+    Vision MoE": priority routing).  Returns dict(pos, drop, counts[k,N], kept[N],
+    offsets[N+1])."""
     lib = _load()
     idx = np.ascontiguousarray(idx, dtype=np.int32)
     T, k = idx.shape
@@ -169,8 +185,13 @@ def dispatch(idx, N, C):
     counts = np.empty((k, N), np.int32)
     kept = np.empty(N, np.int32)
     offsets = np.empty(N + 1, np.int32)
-    lib.oracle_dispatch(T, N, k, int(C), _ptr(idx), _ptr(pos), _ptr(drop), _ptr(counts),
-                        _ptr(kept), _ptr(offsets))
+    if priority is None:
+        lib.oracle_dispatch(T, N, k, int(C), _ptr(idx), _ptr(pos), _ptr(drop), _ptr(counts),
+                            _ptr(kept), _ptr(offsets))
+    else:
+        order = np.ascontiguousarray(priority_order(priority))
+        lib.oracle_dispatch_ordered(T, N, k, int(C), _ptr(idx), _ptr(order), _ptr(pos), _ptr(drop),
+                                    _ptr(counts), _ptr(kept), _ptr(offsets))
     return dict(pos=pos, drop=drop, counts=counts, kept=kept, offsets=offsets)
 
 
@@ -252,14 +273,15 @@ def expert_rows(x, weights, rows_token, rows_expert, act=RELU):
     return ye
 
 
-def forward(x, w_r, b_r, weights, k, C, act=RELU, alpha=1e-2, out_dtype=F32, tokens=None):
-    """The whole layer, step by step: route, aux loss, slot claim, experts,
-    combine.  tokens=None evaluates every token.  Returns a dict with every
-    intermediate and the outputs for the evaluated tokens."""
+def forward(x, w_r, b_r, weights, k, C, act=RELU, alpha=1e-2, out_dtype=F32, tokens=None, priority=False):
+    """The whole layer, step by step: route, aux loss, slot claim (token order,
+    or batch priority), experts, combine.  tokens=None evaluates every token.
+    Returns a dict with every intermediate and the outputs for the evaluated
+    tokens."""
     routing = route(x, w_r, b_r, k)
     f, P, aux = aux_loss(routing["idx"], routing["probs"], alpha)
     N = np.asarray(w_r).shape[0]
-    disp = dispatch(routing["idx"], N, C)
+    disp = dispatch(routing["idx"], N, C, priority=routing["gate"] if priority else None)
     T = np.asarray(x).shape[0]
     if tokens is None:
         tokens = np.arange(T, dtype=np.int64)

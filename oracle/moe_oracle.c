@@ -238,20 +238,26 @@ int32_t oracle_capacity(int64_t T, int32_t N, int32_t k, double cf) {
 }
 
 /* ---- Capacity-limited slot claim -------------------------------------------
- * For r = 0..k-1, for t = 0..T-1 in order: e = idx[t, r]; the assignment takes
- * claim number pos[t, r] = (claims on e so far); it is kept iff pos < C.
+ * For r = 0..k-1, for the tokens in claim order: e = idx[t, r]; the assignment
+ * takes claim number pos[t, r] = (claims on e so far); it is kept iff pos < C.
+ * The claim order is token order (CS25 Lecture 05 notes, capacity-aware
+ * dispatch), or, with batch priority (CS25 Lecture 05 notes, "from language
+ * MoE to Vision MoE": high-priority tokens take the slots first), `order`: a
+ * permutation of 0..T-1 listing the tokens from the highest priority down,
+ * built by the caller.
  * counts[r, e] = claims of rank r on e (pre-capacity); kept[e] =
  * min(sum_r counts[r, e], C); offsets[e] = sum_{e' < e} kept[e'], offsets[N] =
  * total kept rows.  The compact expert-major row of a kept (t, r) is
  * offsets[e] + pos[t, r]. */
-void oracle_dispatch(int64_t T, int32_t N, int32_t k, int32_t C, const int32_t* idx,
-                     int32_t* pos, uint8_t* drop, int32_t* counts, int32_t* kept,
-                     int32_t* offsets) {
+void oracle_dispatch_ordered(int64_t T, int32_t N, int32_t k, int32_t C, const int32_t* idx,
+                             const int64_t* order, int32_t* pos, uint8_t* drop, int32_t* counts,
+                             int32_t* kept, int32_t* offsets) {
     int64_t claims[1024];
     for (int32_t e = 0; e < N; ++e) claims[e] = 0;
     for (int32_t r = 0; r < k; ++r) {
         for (int32_t e = 0; e < N; ++e) counts[r * N + e] = 0;
-        for (int64_t t = 0; t < T; ++t) {
+        for (int64_t q = 0; q < T; ++q) {
+            int64_t t = order ? order[q] : q;
             int32_t e = idx[t * k + r];
             int64_t p = claims[e];
             claims[e] = p + 1;
@@ -268,6 +274,12 @@ void oracle_dispatch(int64_t T, int32_t N, int32_t k, int32_t C, const int32_t* 
         acc += kept[e];
     }
     offsets[N] = (int32_t)acc;
+}
+
+void oracle_dispatch(int64_t T, int32_t N, int32_t k, int32_t C, const int32_t* idx,
+                     int32_t* pos, uint8_t* drop, int32_t* counts, int32_t* kept,
+                     int32_t* offsets) {
+    oracle_dispatch_ordered(T, N, k, C, idx, (const int64_t*)0, pos, drop, counts, kept, offsets);
 }
 
 /* ---- One expert on one token -----------------------------------------------

@@ -316,6 +316,63 @@ def test_dispatch_brute_force(k):
                     np.testing.assert_array_equal(d["offsets"], np.concatenate([[0], np.cumsum(d["kept"])]))
 
 
+# ------------------------------------------------------- batch priority ----
+
+def _rand_routing(T, N, k, seed):
+    rng = np.random.default_rng(seed)
+    idx = np.stack([rng.permutation(N)[:k] for _ in range(T)]).astype(np.int32)
+    gate = rng.random((T, k)).astype(np.float32)
+    return idx, gate
+
+
+@pytest.mark.parametrize("k", [1, 2])
+def test_priority_with_equal_or_decreasing_scores_is_token_order(k):
+    # equal scores (ties to the lower index) and scores decreasing in t both
+    # give exactly the token-order claim, for every capacity
+    T, N = 40, 5
+    idx, gate = _rand_routing(T, N, k, 11)
+    flat = np.full((T, k), 0.25, np.float32)
+    dec = np.repeat(np.linspace(1.0, 0.1, T, dtype=np.float32)[:, None], k, axis=1)
+    for C in (0, 3, 8, 40):
+        ref = oracle.dispatch(idx, N, C)
+        for pr in (flat, dec):
+            got = oracle.dispatch(idx, N, C, priority=pr)
+            for key in ref:
+                np.testing.assert_array_equal(got[key], ref[key], err_msg=key)
+
+
+@pytest.mark.parametrize("k", [1, 2])
+def test_priority_increasing_scores_is_reversed_token_order(k):
+    # scores increasing in t claim in reversed token order: the same as the
+    # token-order dispatch of the reversed batch, read back reversed
+    T, N = 33, 4
+    idx, _ = _rand_routing(T, N, k, 12)
+    inc = np.repeat(np.linspace(0.1, 1.0, T, dtype=np.float32)[:, None], k, axis=1)
+    for C in (0, 2, 5, 33):
+        rev = oracle.dispatch(idx[::-1].copy(), N, C)
+        got = oracle.dispatch(idx, N, C, priority=inc)
+        np.testing.assert_array_equal(got["pos"], rev["pos"][::-1])
+        np.testing.assert_array_equal(got["drop"], rev["drop"][::-1])
+        for key in ("counts", "kept", "offsets"):
+            np.testing.assert_array_equal(got[key], rev[key])
+
+
+def test_priority_top1_keeps_the_highest_scores_per_expert():
+    # top-1: an expert keeps exactly its C claimants with the largest scores
+    # (ties to the lower index), whatever their positions in the batch
+    T, N, C = 200, 6, 9
+    idx, gate = _rand_routing(T, N, 1, 13)
+    gate[::7, 0] = gate[3, 0]                   # plant ties
+    got = oracle.dispatch(idx, N, C, priority=gate)
+    for e in range(N):
+        ts = np.nonzero(idx[:, 0] == e)[0]
+        ranked = sorted(ts, key=lambda t: (-float(gate[t, 0]), t))
+        kept = set(ranked[:C])
+        assert set(ts[got["drop"][ts, 0] == 0]) == kept
+        for n, t in enumerate(ranked):
+            assert got["pos"][t, 0] == n
+
+
 def test_gshard_rank_major_example():
     # CMU 10-423 Lecture 16 section 6.1 (b): 3 devices of capacity 3; first choices are
     # placed before second choices, so a token's second choice can find its expert full.
