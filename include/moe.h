@@ -72,7 +72,17 @@ typedef enum { MOE_RELU = 0, MOE_SWIGLU = 1 } moe_act;
 
 /* Layer shape.  Limits: 0 <= T < 2^28; 1 <= n_experts <= 128; top_k in {1, 2}
  * with top_k <= n_experts; capacity >= 0 (the explicit C; see moe_capacity);
- * d_model, d_ff >= 1; for MOE_BF16, d_model and d_ff multiples of 16. */
+ * d_model, d_ff >= 1; for MOE_BF16, d_model and d_ff multiples of 16.
+ * priority selects the order in which assignments claim expert slots:
+ *   MOE_ORDER_TOKEN (0): token order (CS25 Lecture 05 notes, capacity-aware
+ *     dispatch); every rank-0 claim before any rank-1 claim.
+ *   MOE_ORDER_PRIORITY (1): batch priority (CS25 Lecture 05 notes, section on
+ *     Vision MoE: with capacity short, the tokens with the highest priority
+ *     score take the slots first): tokens by descending first-choice gate
+ *     gate[t, 0], ties to the lower token index; still rank-major.  pos is
+ *     the claim number in that order.  Not available for the sharded
+ *     dispatch or moe_dispatch_noalloc (MOE_ERR_UNSUPPORTED). */
+typedef enum { MOE_ORDER_TOKEN = 0, MOE_ORDER_PRIORITY = 1 } moe_claim_order;
 typedef struct {
     int32_t T;
     int32_t d_model;
@@ -83,6 +93,7 @@ typedef struct {
     int32_t dtype;   /* moe_dtype */
     int32_t act;     /* moe_act */
     float alpha;     /* load-balancing loss weight */
+    int32_t priority;  /* moe_claim_order */
 } moe_config;
 
 /* Expert capacity C = floor(k * T * cf / N), computed exactly from the binary

@@ -59,6 +59,7 @@ struct Layout {
     size_t hdr, part_cnt, part_psum, part_z, w_split, scan_state;
     size_t idx, gate, pos, drop, counts, kept, offsets, f, P, aux;
     size_t row_token, row_gate, xe, h, ye;
+    size_t prio_hist, prio_cursor, prio_list, prio_perm, prio_idx, prio_pos, prio_range;   // batch priority only
     size_t total;
     int64_t rows;   // min(k T, N C): compact rows the buffers hold
 };
@@ -104,6 +105,15 @@ Layout layout_of(const moe_config& c) {
     L.xe = take(esz * R * (size_t)c.d_model);
     L.h = take(esz * R * (size_t)c.d_ff);
     L.ye = take(esz * R * (size_t)c.d_model);
+    if (c.priority == MOE_ORDER_PRIORITY) {   // batch-priority claim order scratch
+        L.prio_hist = take(4 * (size_t)(kPrioBuckets + 1));
+        L.prio_cursor = take(4 * (size_t)kPrioBuckets);
+        L.prio_list = take(4 * T);
+        L.prio_perm = take(4 * T);
+        L.prio_idx = take(4 * T * k);
+        L.prio_pos = take(4 * T * k);
+        L.prio_range = take(8);
+    }
     L.total = off;
     return L;
 }
@@ -118,6 +128,7 @@ int32_t validate(const moe_config* c) {
     if (c->act != MOE_RELU && c->act != MOE_SWIGLU) return MOE_ERR_INVALID_ARG;
     if (c->top_k > c->n_experts) return MOE_ERR_INVALID_ARG;
     if (!std::isfinite(c->alpha)) return MOE_ERR_INVALID_ARG;
+    if (c->priority != MOE_ORDER_TOKEN && c->priority != MOE_ORDER_PRIORITY) return MOE_ERR_INVALID_ARG;
     if (c->T >= (1 << 28) || c->n_experts > 128 || c->top_k > 2) return MOE_ERR_UNSUPPORTED;
     if (c->dtype == MOE_BF16 && (c->d_model % 16 != 0 || c->d_ff % 16 != 0)) return MOE_ERR_UNSUPPORTED;
     if ((int64_t)c->d_model * c->d_ff >= ((int64_t)1 << 40)) return MOE_ERR_UNSUPPORTED;
@@ -281,6 +292,15 @@ static int32_t dispatch_impl(const moe_config* cfg, const void* x, const int32_t
     a.hdr = at<WsHeader>(ws, L.hdr);
     a.claim_base = claim_base;
     if (aux) a.aux = *aux;
+    if (cfg->priority == MOE_ORDER_PRIORITY) {
+        a.prio.hist = at<int32_t>(ws, L.prio_hist);
+        a.prio.cursor = at<int32_t>(ws, L.prio_cursor);
+        a.prio.list = at<int32_t>(ws, L.prio_list);
+        a.prio.perm = at<int32_t>(ws, L.prio_perm);
+        a.prio.idx_sorted = at<int32_t>(ws, L.prio_idx);
+        a.prio.pos_sorted = at<int32_t>(ws, L.prio_pos);
+        a.prio.range = at<uint32_t>(ws, L.prio_range);
+    }
     return cuda_status(launch_dispatch(a, s));
 }
 
@@ -304,6 +324,7 @@ int32_t moe_dispatch_shard(const moe_config* cfg, const void* x, const int32_t* 
                            size_t ws_bytes, void* stream) {
     int32_t st = validate(cfg);
     if (st != MOE_OK) return st;
+    if (cfg->priority != MOE_ORDER_TOKEN) return MOE_ERR_UNSUPPORTED;   // needs every shard's scores
     if (!req(claim_base) || !req(counts) || !req(kept) || !req(offsets) || !opt(xe) || !opt(x))
         return MOE_ERR_INVALID_ARG;
     if (cfg->T > 0 && (!req(idx) || !req(gate) || !req(pos) || !req(drop) || !req(row_token) || !req(row_gate)))

@@ -221,6 +221,18 @@ __host__ __device__ __forceinline__ int kept_after(int base, int count, int C) {
     return room <= 0 ? 0 : (room < count ? room : count);
 }
 
+// Batch-priority scratch (all device, workspace-held); perm == nullptr: token order.
+constexpr int kPrioBuckets = 1 << 16;
+struct PrioArgs {
+    int32_t* hist;        // [kPrioBuckets + 1] bucket counts, then their exclusive prefix
+    int32_t* cursor;      // [kPrioBuckets]
+    int32_t* list;        // [T] tokens grouped by bucket
+    int32_t* perm;        // [T] perm[place] = token
+    int32_t* idx_sorted;  // [T, k] expert choices in claim order
+    int32_t* pos_sorted;  // [T, k] claim numbers in claim order
+    uint32_t* range;      // [2] smallest and largest key of the batch
+};
+
 struct DispatchArgs {
     const void* x; int dtype; const int32_t* idx; const float* gate;
     int64_t T; int d; int N; int k; int C;
@@ -230,6 +242,7 @@ struct DispatchArgs {
     uint32_t* scan_state; WsHeader* hdr;
     const int32_t* claim_base;   // [k, N] claims made before this shard (sharded batch), or null
     AuxArgs aux;                 // G > 0: one extra block of the gather reduces the router partials
+    PrioArgs prio;               // batch priority (perm set) or token order
 };
 int scan_blocks(int64_t T);
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s);

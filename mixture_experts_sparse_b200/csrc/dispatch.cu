@@ -181,7 +181,8 @@ scatter_kernel(const XT* __restrict__ x, const int32_t* __restrict__ idx, const 
                int64_t T, int d, int N, int k, int C,
                const int32_t* __restrict__ claim_base, int32_t* __restrict__ pos, uint8_t* __restrict__ drop,
                const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets, int32_t* __restrict__ row_token,
-               float* __restrict__ row_gate, XT* __restrict__ xe, XT* __restrict__ zero_out, const AuxArgs aux) {
+               float* __restrict__ row_gate, XT* __restrict__ xe, XT* __restrict__ zero_out, const AuxArgs aux,
+               const int32_t* __restrict__ perm, const int32_t* __restrict__ pos_in) {
     pdl_wait();
     pdl_launch();
     // the extra block (the first, so it is scheduled at once and runs beside
@@ -194,12 +195,17 @@ scatter_kernel(const XT* __restrict__ x, const int32_t* __restrict__ idx, const 
     const int lane = threadIdx.x & 31;
     const int64_t a = (int64_t)(blockIdx.x - (aux.G > 0 ? 1 : 0)) * 8 + (threadIdx.x >> 5);
     if (a >= T * k) return;
-    const int64_t t = a / k;
-    const int r = (int)(a - t * k);
+    // a enumerates the assignments in claim order: position q of the claim
+    // order, rank r.  Batch priority: the token at position q is perm[q], and
+    // the scan's claim numbers are in pos_in (claim-order layout).
+    const int64_t q = a / k;
+    const int r = (int)(a - q * k);
+    const int64_t t = perm ? (int64_t)perm[q] : q;
+    const int64_t ao = t * k + r;               // the assignment in token order
     int row = -1;
     if (lane == 0) {
-        const int e = idx[a];
-        const int lp = pos[a];                  // claim number among this shard's rank-r claims on e
+        const int e = idx[ao];
+        const int lp = pos_in ? pos_in[a] : pos[a];   // claim number among this shard's rank-r claims on e
         int p, row_off;
         if (r == 0) {
             p = (claim_base ? claim_base[e] : 0) + lp;
@@ -210,12 +216,12 @@ scatter_kernel(const XT* __restrict__ x, const int32_t* __restrict__ idx, const 
             row_off = kept_after(base0, counts[e], C) + lp;
         }
         const bool keep = p < C;
-        pos[a] = p;
-        drop[a] = keep ? 0 : 1;
+        pos[ao] = p;
+        drop[ao] = keep ? 0 : 1;
         if (keep) {
             row = offsets[e] + row_off;
             row_token[row] = (int32_t)t;
-            row_gate[row] = gate[a];
+            row_gate[row] = gate[ao];
         }
     }
     row = __shfl_sync(0xffffffffu, row, 0);
@@ -238,6 +244,125 @@ scatter_kernel(const XT* __restrict__ x, const int32_t* __restrict__ idx, const 
         } else {
             for (int j = lane; j < d; j += 32) zero_out[t * (int64_t)d + j] = XT(0.f);
         }
+    }
+}
+
+// ---- batch priority: the claim order --------------------------------------
+// CS25 Lecture 05 notes, section on Vision MoE: with capacity short, priority
+// routing lets the tokens with the highest priority score take the expert
+// slots first.  The score is the token's first-choice gate; the claim order is
+// descending score, ties to the lower token index (rank-major as before).
+// Key: 0xFFFFFFFF - bits(gate) (gates are >= 0, so their bit patterns order
+// like their values), ascending.  The batch's key range [kmin, kmax] is cut
+// into kPrioBuckets equal intervals (a monotone bucket map).  A token's place
+// in the order is the number of tokens in lower buckets plus, within its
+// bucket, the number of tokens with a smaller key or the same key and a lower
+// index -- exact and independent of the order in which the bucket lists were
+// filled.  Cost: one pass per token over its bucket (quadratic only when most
+// scores fall into one interval, e.g. many equal scores).
+__device__ __forceinline__ uint32_t prio_key(const float* gate, int64_t t, int k) {
+    return 0xFFFFFFFFu - __float_as_uint(gate[t * k]);
+}
+// range[0] = kmin, range[1] = kmax of the batch
+__device__ __forceinline__ uint32_t prio_bucket(uint32_t key, const uint32_t* range) {
+    const uint32_t lo = range[0], width = ((range[1] - lo) >> 16) + 1u;
+    return (key - lo) / width;   // < kPrioBuckets
+}
+
+__global__ void __launch_bounds__(256)
+prio_range_kernel(const float* __restrict__ gate, int64_t T, int k, uint32_t* __restrict__ range) {
+    pdl_wait();
+    pdl_launch();
+    uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < T; t += (int64_t)gridDim.x * blockDim.x) {
+        const uint32_t u = prio_key(gate, t, k);
+        mn = min(mn, u);
+        mx = max(mx, u);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        mn = min(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    if ((threadIdx.x & 31) == 0) {
+        atomicMin(&range[0], mn);
+        atomicMax(&range[1], mx);
+    }
+}
+
+__global__ void __launch_bounds__(256)
+prio_hist_kernel(const float* __restrict__ gate, int64_t T, int k, const uint32_t* __restrict__ range,
+                 int32_t* __restrict__ hist) {
+    pdl_wait();
+    pdl_launch();
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < T; t += (int64_t)gridDim.x * blockDim.x)
+        atomicAdd(&hist[prio_bucket(prio_key(gate, t, k), range)], 1);
+}
+
+// exclusive prefix of the kPrioBuckets counts, in place; hist[kPrioBuckets] = T.
+// One block of 32 warps; warp w owns the contiguous chunk [w C, (w + 1) C) and
+// scans it 32 entries at a time (coalesced), carrying the running total.
+__global__ void __launch_bounds__(1024) prio_scan_kernel(int32_t* __restrict__ hist) {
+    pdl_wait();
+    pdl_launch();
+    __shared__ int32_t s_warp[32];
+    constexpr int CHUNK = kPrioBuckets / 32;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int32_t* h = hist + warp * CHUNK;
+    int32_t tot = 0;
+    for (int j = lane; j < CHUNK; j += 32) tot += h[j];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xffffffffu, tot, o);
+    if (lane == 0) s_warp[warp] = tot;
+    __syncthreads();
+    int32_t carry = 0;
+    for (int w = 0; w < warp; ++w) carry += s_warp[w];
+    for (int j0 = 0; j0 < CHUNK; j0 += 32) {
+        const int32_t c = h[j0 + lane];
+        int32_t incl = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int32_t v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += v;
+        }
+        h[j0 + lane] = carry + incl - c;
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (threadIdx.x == 1023) hist[kPrioBuckets] = carry;
+}
+
+// bucket lists: list[base[b] + n] = t, n in arrival order
+__global__ void __launch_bounds__(256)
+prio_fill_kernel(const float* __restrict__ gate, int64_t T, int k, const uint32_t* __restrict__ range,
+                 const int32_t* __restrict__ base, int32_t* __restrict__ cursor, int32_t* __restrict__ list) {
+    pdl_wait();
+    pdl_launch();
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < T; t += (int64_t)gridDim.x * blockDim.x) {
+        const uint32_t b = prio_bucket(prio_key(gate, t, k), range);
+        list[base[b] + atomicAdd(&cursor[b], 1)] = (int32_t)t;
+    }
+}
+
+// place of t in the claim order; perm[place] = t, idx_sorted[place] = idx[t]
+__global__ void __launch_bounds__(256)
+prio_rank_kernel(const float* __restrict__ gate, const int32_t* __restrict__ idx, int64_t T, int k,
+                 const uint32_t* __restrict__ range, const int32_t* __restrict__ base,
+                 const int32_t* __restrict__ list, int32_t* __restrict__ perm, int32_t* __restrict__ idx_sorted) {
+    pdl_wait();
+    pdl_launch();
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < T; t += (int64_t)gridDim.x * blockDim.x) {
+        const uint32_t u = prio_key(gate, t, k);
+        const uint32_t b = prio_bucket(u, range);
+        const int32_t lo = base[b], hi = base[b + 1];
+        int32_t c = 0;
+        for (int32_t j = lo; j < hi; ++j) {
+            const int64_t t2 = list[j];
+            const uint32_t u2 = prio_key(gate, t2, k);
+            c += (u2 < u || (u2 == u && t2 < t)) ? 1 : 0;
+        }
+        const int64_t place = (int64_t)lo + c;
+        perm[place] = (int32_t)t;
+        for (int r = 0; r < k; ++r) idx_sorted[place * k + r] = idx[t * k + r];
     }
 }
 
@@ -316,13 +441,46 @@ int scan_blocks(int64_t T) { return (int)((T + kScanTokens - 1) / kScanTokens); 
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
     const int nblk = scan_blocks(a.T);
     if (nblk == 0) return cudaSuccess;
+    cudaError_t err;
+    // claim order: token order, or batch priority (the scan then runs over the
+    // expert choices in claim order and the gather maps back through perm)
+    const int32_t* scan_idx = a.idx;
+    int32_t* scan_pos = a.pos;
+    const int32_t* perm = nullptr;
+    const int32_t* pos_in = nullptr;
+    if (a.prio.perm) {
+        const PrioArgs& q = a.prio;
+        if ((err = cudaMemsetAsync(q.hist, 0, sizeof(int32_t) * (kPrioBuckets + 1), s)) != cudaSuccess) return err;
+        if ((err = cudaMemsetAsync(q.cursor, 0, sizeof(int32_t) * kPrioBuckets, s)) != cudaSuccess) return err;
+        if ((err = cudaMemsetAsync(q.range, 0xFF, sizeof(uint32_t), s)) != cudaSuccess) return err;     // kmin
+        if ((err = cudaMemsetAsync(q.range + 1, 0, sizeof(uint32_t), s)) != cudaSuccess) return err;   // kmax
+        const unsigned pg = (unsigned)((a.T + 255) / 256 < 4096 ? (a.T + 255) / 256 : 4096);
+        if ((err = launch_k(prio_range_kernel, dim3(pg), dim3(256), 0, s, 1, a.gate, a.T, a.k, q.range)) != cudaSuccess)
+            return err;
+        if ((err = launch_k(prio_hist_kernel, dim3(pg), dim3(256), 0, s, 1, a.gate, a.T, a.k,
+                            static_cast<const uint32_t*>(q.range), q.hist)) != cudaSuccess)
+            return err;
+        if ((err = launch_k(prio_scan_kernel, dim3(1), dim3(1024), 0, s, 1, q.hist)) != cudaSuccess) return err;
+        if ((err = launch_k(prio_fill_kernel, dim3(pg), dim3(256), 0, s, 1, a.gate, a.T, a.k,
+                            static_cast<const uint32_t*>(q.range), static_cast<const int32_t*>(q.hist), q.cursor,
+                            q.list)) != cudaSuccess)
+            return err;
+        if ((err = launch_k(prio_rank_kernel, dim3(pg), dim3(256), 0, s, 1, a.gate, a.idx, a.T, a.k,
+                            static_cast<const uint32_t*>(q.range), static_cast<const int32_t*>(q.hist),
+                            static_cast<const int32_t*>(q.list), q.perm, q.idx_sorted)) != cudaSuccess)
+            return err;
+        scan_idx = q.idx_sorted;
+        scan_pos = q.pos_sorted;
+        perm = q.perm;
+        pos_in = q.pos_sorted;
+    }
     // fresh tickets and look-back flags for this call
-    cudaError_t err = cudaMemsetAsync(&a.hdr->scan_ticket, 0, 2 * sizeof(int32_t), s);
+    err = cudaMemsetAsync(&a.hdr->scan_ticket, 0, 2 * sizeof(int32_t), s);
     if (err != cudaSuccess) return err;
     err = cudaMemsetAsync(a.scan_state, 0, sizeof(uint32_t) * (size_t)nblk * a.k * a.N, s);
     if (err != cudaSuccess) return err;
-    err = launch_k(scan_kernel, dim3((unsigned)nblk), dim3(kScanThreads), 0, s, 1, a.idx, a.T, a.N, a.k, a.C, nblk,
-                   a.claim_base, a.pos, a.counts, a.kept, a.offsets, a.scan_state, a.hdr, kWaitLimitNs);
+    err = launch_k(scan_kernel, dim3((unsigned)nblk), dim3(kScanThreads), 0, s, 1, scan_idx, a.T, a.N, a.k, a.C, nblk,
+                   a.claim_base, scan_pos, a.counts, a.kept, a.offsets, a.scan_state, a.hdr, kWaitLimitNs);
     if (err != cudaSuccess) return err;
     const int64_t warps = a.T * a.k;
     const unsigned grid = (unsigned)((warps + 7) / 8) + (a.aux.G > 0 ? 1u : 0u);
@@ -330,10 +488,12 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
         return launch_k(scatter_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, 1,
                         reinterpret_cast<const __nv_bfloat16*>(a.x), a.idx, a.gate, a.T, a.d, a.N, a.k, a.C,
                         a.claim_base, a.pos, a.drop, a.counts, a.offsets, a.row_token, a.row_gate,
-                        reinterpret_cast<__nv_bfloat16*>(a.xe), reinterpret_cast<__nv_bfloat16*>(a.zero_out), a.aux);
+                        reinterpret_cast<__nv_bfloat16*>(a.xe), reinterpret_cast<__nv_bfloat16*>(a.zero_out), a.aux,
+                        perm, pos_in);
     return launch_k(scatter_kernel<float>, dim3(grid), dim3(256), 0, s, 1, reinterpret_cast<const float*>(a.x), a.idx,
                     a.gate, a.T, a.d, a.N, a.k, a.C, a.claim_base, a.pos, a.drop, a.counts, a.offsets, a.row_token,
-                    a.row_gate, reinterpret_cast<float*>(a.xe), reinterpret_cast<float*>(a.zero_out), a.aux);
+                    a.row_gate, reinterpret_cast<float*>(a.xe), reinterpret_cast<float*>(a.zero_out), a.aux, perm,
+                    pos_in);
 }
 
 cudaError_t launch_counts(const int32_t* idx, int64_t T, int N, int k, int32_t* counts, cudaStream_t s) {

@@ -34,9 +34,9 @@ class MoeLayer:
     """Weights, workspace and routing outputs of one layer on one GPU."""
 
     def __init__(self, T, d_model, d_ff, n_experts, top_k, capacity, dtype, act, weights, alpha=1e-2,
-                 device="cuda"):
+                 device="cuda", priority=False):
         import torch
-        self.cfg = nat.config(T, d_model, d_ff, n_experts, top_k, capacity, dtype, act, alpha)
+        self.cfg = nat.config(T, d_model, d_ff, n_experts, top_k, capacity, dtype, act, alpha, priority=priority)
         self.device = device
         self.w = {k: to_device(weights.get(k), device) for k in WEIGHT_KEYS}
         self.ws = nat.new_workspace(self.cfg, device)

@@ -22,7 +22,8 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe_b200
 class MoeConfig(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d_model", ctypes.c_int32), ("d_ff", ctypes.c_int32),
                 ("n_experts", ctypes.c_int32), ("top_k", ctypes.c_int32), ("capacity", ctypes.c_int32),
-                ("dtype", ctypes.c_int32), ("act", ctypes.c_int32), ("alpha", ctypes.c_float)]
+                ("dtype", ctypes.c_int32), ("act", ctypes.c_int32), ("alpha", ctypes.c_float),
+                ("priority", ctypes.c_int32)]
 
 
 class MoeError(RuntimeError):
@@ -72,10 +73,15 @@ def lib():
     return _lib
 
 
-def config(T, d_model, d_ff, n_experts, top_k, capacity, dtype="bf16", act="relu", alpha=1e-2):
+MOE_ORDER_TOKEN, MOE_ORDER_PRIORITY = 0, 1
+
+
+def config(T, d_model, d_ff, n_experts, top_k, capacity, dtype="bf16", act="relu", alpha=1e-2, priority=False):
+    """moe_config; priority=True selects the batch-priority claim order."""
     return MoeConfig(int(T), int(d_model), int(d_ff), int(n_experts), int(top_k), int(capacity),
                      MOE_BF16 if dtype in ("bf16", MOE_BF16) else MOE_F32,
-                     MOE_SWIGLU if act in ("swiglu", MOE_SWIGLU) else MOE_RELU, float(alpha))
+                     MOE_SWIGLU if act in ("swiglu", MOE_SWIGLU) else MOE_RELU, float(alpha),
+                     MOE_ORDER_PRIORITY if priority else MOE_ORDER_TOKEN)
 
 
 def _p(t):

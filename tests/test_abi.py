@@ -58,6 +58,13 @@ def test_workspace_bytes_and_validation():
     for cfg in bad:
         assert nat.moe_workspace_bytes(cfg) == 0
     assert nat.moe_workspace_bytes(nat.config(16, 760, 3072, 8, 1, 8, dtype="f32")) > 0
+    # the batch-priority claim order needs its sort scratch on top; an unknown
+    # claim order is rejected
+    prio = nat.config(4096, 768, 3072, 64, 1, 80, priority=True)
+    assert nat.moe_workspace_bytes(prio) >= ws + 4 * (2 * 65536 + 1 + 4 * 4096)
+    odd = nat.config(4096, 768, 3072, 64, 1, 80)
+    odd.priority = 2
+    assert nat.moe_workspace_bytes(odd) == 0
 
 
 def test_host_validation_rejects_before_launch():
