@@ -35,7 +35,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM traffic of the first grouped GEMM launch (dram__bytes_read.sum +
 # dram__bytes_write.sum) from one ncu capture, keyed by workload, valid only
 # for the kernel source it was measured on.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # python bench.py --steps 3 --warmup 3 --no-cpu-baseline, then under
+    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none
+    #     -k regex:grouped_gemm -s 6 -c 2 (first timed step): stage 1 read
+    # 402836224 B (W1 + xe, the compulsory set) and wrote 362386432 B (H, part
+    # of it still in L2 when the kernel ends)
+    "switch_base": {"bytes_per_launch": 402836224 + 362386432, "src_sha": "0f4a4cb5b69485fa"},
+}
 
 
 def peaks():
