@@ -48,6 +48,7 @@ def _load():
         lib.oracle_capacity.restype = i32
         lib.oracle_dispatch.argtypes = [i64, i32, i32, i32, P, P, P, P, P, P]
         lib.oracle_dispatch_ordered.argtypes = [i64, i32, i32, i32, P, P, P, P, P, P, P]
+        lib.oracle_dispatch_ntlb.argtypes = [i64, i32, i32, P, P, P, P, P, P, P, P, P]
         lib.oracle_dispatch.restype = None
         lib.oracle_expert_ffn.argtypes = [i32, i32, i32, P, i32, sz, P, P, P, P, P, P, i32,
                                           sz, sz, sz, sz, P, P]
@@ -193,6 +194,28 @@ def dispatch(idx, N, C, priority=None):
         lib.oracle_dispatch_ordered(T, N, k, int(C), _ptr(idx), _ptr(order), _ptr(pos), _ptr(drop),
                                     _ptr(counts), _ptr(kept), _ptr(offsets))
     return dict(pos=pos, drop=drop, counts=counts, kept=kept, offsets=offsets)
+
+
+def dispatch_ntlb(probs, gate0, C):
+    """No-Token-Left-Behind re-routing for top-1 (CS25 Lecture 05 notes, "No
+    Token Left Behind": a token whose expert is full goes on to its next
+    choices until it gets a slot).  Stages in token order; see the C source for
+    the reading.  Returns dict(expert, gate, pos, drop, counts[N], kept[N],
+    offsets[N+1])."""
+    lib = _load()
+    probs = np.ascontiguousarray(probs, dtype=np.float32)
+    T, N = probs.shape
+    gate0 = np.ascontiguousarray(np.asarray(gate0, np.float32).reshape(T))
+    expert = np.empty(T, np.int32)
+    gate = np.empty(T, np.float32)
+    pos = np.empty(T, np.int32)
+    drop = np.empty(T, np.uint8)
+    counts = np.empty(N, np.int32)
+    kept = np.empty(N, np.int32)
+    offsets = np.empty(N + 1, np.int32)
+    lib.oracle_dispatch_ntlb(T, N, int(C), _ptr(probs), _ptr(gate0), _ptr(expert), _ptr(gate), _ptr(pos),
+                             _ptr(drop), _ptr(counts), _ptr(kept), _ptr(offsets))
+    return dict(expert=expert, gate=gate, pos=pos, drop=drop, counts=counts, kept=kept, offsets=offsets)
 
 
 def expert_ffn(x_row, w1, b1, w2, b2, act=RELU, w3=None, b3=None):

@@ -276,6 +276,71 @@ void oracle_dispatch_ordered(int64_t T, int32_t N, int32_t k, int32_t C, const i
     offsets[N] = (int32_t)acc;
 }
 
+/* ---- No-Token-Left-Behind re-routing (top-1) -------------------------------
+ * CS25 Lecture 05 notes, "No Token Left Behind": when a token's top-1 expert is
+ * full, it is sent on to its second, third ... choice until it gets a slot.
+ * Reading: stage 0 is the token-order claim on the first choice; in stage s a
+ * token without a slot claims, in token order, on its (s+1)-th expert in the
+ * order of its router probabilities probs[t, :] (descending, ties to the lower
+ * index), its claim numbered after every claim already made on that expert;
+ * it is kept iff that number is below C.  Stages run until every token has a
+ * slot or all N choices were tried.  Outputs per token: expert[t] (the expert
+ * that kept it; its first choice if none did), gate[t] = probs[t, expert[t]]
+ * for a kept token (its first-choice gate if dropped), pos[t] (claim number on
+ * expert[t]; C for a dropped token), drop[t]; per expert: counts[e] = every
+ * claim made on e over all stages, kept[e] = min(counts[e], C), offsets as in
+ * oracle_dispatch.  A kept token's compact row is offsets[e] + pos[t]. */
+void oracle_dispatch_ntlb(int64_t T, int32_t N, int32_t C, const float* probs, const float* gate0,
+                          int32_t* expert, float* gate, int32_t* pos, uint8_t* drop, int32_t* counts,
+                          int32_t* kept, int32_t* offsets) {
+    int64_t claims[1024];
+    for (int32_t e = 0; e < N; ++e) claims[e] = 0;
+    for (int64_t t = 0; t < T; ++t) drop[t] = 1;
+    for (int32_t s = 0; s < N; ++s) {
+        int64_t left = 0;
+        for (int64_t t = 0; t < T; ++t) {
+            if (!drop[t]) continue;
+            /* the (s+1)-th expert of t: rank experts by probability, ties to the
+             * lower index, by counting for each e how many experts precede it */
+            const float* p = probs + (size_t)t * N;
+            int32_t e_s = -1;
+            for (int32_t e = 0; e < N && e_s < 0; ++e) {
+                int32_t ahead = 0;
+                for (int32_t j = 0; j < N; ++j) {
+                    if (p[j] > p[e] || (p[j] == p[e] && j < e)) ++ahead;
+                }
+                if (ahead == s) e_s = e;
+            }
+            int64_t c = claims[e_s];
+            claims[e_s] = c + 1;
+            if (s == 0) expert[t] = e_s;
+            if (c < (int64_t)C) {
+                drop[t] = 0;
+                expert[t] = e_s;
+                pos[t] = (int32_t)c;
+                gate[t] = p[e_s];
+            } else {
+                ++left;
+            }
+        }
+        if (left == 0) break;
+    }
+    for (int64_t t = 0; t < T; ++t) {
+        if (drop[t]) {
+            pos[t] = C;
+            gate[t] = gate0[t];
+        }
+    }
+    int64_t acc = 0;
+    for (int32_t e = 0; e < N; ++e) {
+        counts[e] = (int32_t)claims[e];
+        kept[e] = (int32_t)(claims[e] < (int64_t)C ? claims[e] : (int64_t)C);
+        offsets[e] = (int32_t)acc;
+        acc += kept[e];
+    }
+    offsets[N] = (int32_t)acc;
+}
+
 void oracle_dispatch(int64_t T, int32_t N, int32_t k, int32_t C, const int32_t* idx,
                      int32_t* pos, uint8_t* drop, int32_t* counts, int32_t* kept,
                      int32_t* offsets) {

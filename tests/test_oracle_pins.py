@@ -373,6 +373,67 @@ def test_priority_top1_keeps_the_highest_scores_per_expert():
             assert got["pos"][t, 0] == n
 
 
+# ------------------------------------------------- no token left behind ----
+
+def _probs(T, N, seed):
+    rng = np.random.default_rng(seed)
+    h = rng.standard_normal((T, N))
+    p = np.exp(h - h.max(axis=1, keepdims=True))
+    return (p / p.sum(axis=1, keepdims=True)).astype(np.float32)
+
+
+def test_ntlb_without_overflow_is_the_top1_dispatch():
+    # C >= T: nobody overflows, so stage 0 alone is the token-order top-1 claim
+    T, N = 60, 5
+    p = _probs(T, N, 21)
+    top1 = np.argmax(p, axis=1).astype(np.int32)            # no exact ties in random data
+    ref = oracle.dispatch(top1[:, None], N, T)
+    got = oracle.dispatch_ntlb(p, p[np.arange(T), top1], T)
+    np.testing.assert_array_equal(got["expert"], top1)
+    np.testing.assert_array_equal(got["pos"], ref["pos"][:, 0])
+    np.testing.assert_array_equal(got["drop"], ref["drop"][:, 0])
+    np.testing.assert_array_equal(got["offsets"], ref["offsets"])
+    np.testing.assert_array_equal(got["gate"], p[np.arange(T), top1])
+
+
+@pytest.mark.parametrize("C", [0, 1, 4, 7, 12, 30])
+def test_ntlb_drops_only_when_every_expert_is_full(C):
+    T, N = 30, 4
+    p = _probs(T, N, 22)
+    top1 = np.argmax(p, axis=1)
+    got = oracle.dispatch_ntlb(p, p[np.arange(T), top1], C)
+    kept = got["kept"]
+    assert int(kept.sum()) == min(T, N * C)                  # a slot left anywhere takes a token
+    assert int((got["drop"] == 0).sum()) == min(T, N * C)
+    assert np.all(kept <= C)
+    # stage 0 keeps exactly the token-order top-1 claims below C
+    ref = oracle.dispatch(top1[:, None].astype(np.int32), N, C)
+    first = ref["drop"][:, 0] == 0
+    np.testing.assert_array_equal(got["expert"][first], top1[first])
+    np.testing.assert_array_equal(got["pos"][first], ref["pos"][first, 0])
+    # a kept token's gate is its probability for the expert that kept it, and
+    # every expert it prefers to that one was already full when it tried it
+    for t in np.nonzero(got["drop"] == 0)[0]:
+        e = got["expert"][t]
+        assert got["gate"][t] == p[t, e]
+        assert got["pos"][t] < C
+    rows = got["offsets"][got["expert"][got["drop"] == 0]] + got["pos"][got["drop"] == 0]
+    assert sorted(rows.tolist()) == list(range(int(kept.sum())))   # compact rows tile exactly
+
+
+def test_ntlb_small_hand_example():
+    # 3 tokens, 2 experts, C = 1.  All prefer expert 0: token 0 takes it in
+    # stage 0; in stage 1 token 1 takes expert 1 and token 2 finds it full.
+    p = np.array([[0.9, 0.1], [0.8, 0.2], [0.7, 0.3]], np.float32)
+    got = oracle.dispatch_ntlb(p, p[:, 0], 1)
+    np.testing.assert_array_equal(got["expert"], [0, 1, 0])
+    np.testing.assert_array_equal(got["drop"], [0, 0, 1])
+    np.testing.assert_array_equal(got["pos"], [0, 0, 1])
+    np.testing.assert_array_equal(got["counts"], [3, 2])
+    np.testing.assert_array_equal(got["kept"], [1, 1])
+    np.testing.assert_allclose(got["gate"], [0.9, 0.2, 0.7])
+
+
 def test_gshard_rank_major_example():
     # CMU 10-423 Lecture 16 section 6.1 (b): 3 devices of capacity 3; first choices are
     # placed before second choices, so a token's second choice can find its expert full.
