@@ -80,9 +80,17 @@ typedef enum { MOE_RELU = 0, MOE_SWIGLU = 1 } moe_act;
  *     Vision MoE: with capacity short, the tokens with the highest priority
  *     score take the slots first): tokens by descending first-choice gate
  *     gate[t, 0], ties to the lower token index; still rank-major.  pos is
- *     the claim number in that order.  Not available for the sharded
- *     dispatch or moe_dispatch_noalloc (MOE_ERR_UNSUPPORTED). */
-typedef enum { MOE_ORDER_TOKEN = 0, MOE_ORDER_PRIORITY = 1 } moe_claim_order;
+ *     the claim number in that order.
+ *   MOE_ORDER_NTLB (2): No-Token-Left-Behind re-routing, top-1 only (CS25
+ *     Lecture 05 notes, "No Token Left Behind": a token whose expert is full
+ *     goes on to its next choices until it gets a slot); see
+ *     moe_dispatch_ntlb.  moe_forward runs it from the router probabilities
+ *     and returns in idx / gate the expert each token finally uses and its
+ *     probability.
+ * Orders other than MOE_ORDER_TOKEN are not available for the sharded
+ * dispatch or moe_dispatch_noalloc, and MOE_ORDER_NTLB not for moe_dispatch
+ * (MOE_ERR_UNSUPPORTED). */
+typedef enum { MOE_ORDER_TOKEN = 0, MOE_ORDER_PRIORITY = 1, MOE_ORDER_NTLB = 2 } moe_claim_order;
 typedef struct {
     int32_t T;
     int32_t d_model;
@@ -154,6 +162,26 @@ int32_t moe_dispatch(const moe_config* cfg, const void* x, const int32_t* idx, c
                      int32_t* pos, uint8_t* drop, int32_t* counts, int32_t* kept,
                      int32_t* offsets, int32_t* row_token, float* row_gate, void* xe,
                      void* ws, size_t ws_bytes, void* stream);
+
+/* No-Token-Left-Behind dispatch (top-1; cfg->priority must be MOE_ORDER_NTLB).
+ * Stage 0 is the token-order claim on each token's first expert; in stage s
+ * every token still without a slot claims, in token order, on its (s+1)-th
+ * expert by router probability (descending, ties to the lower index), its
+ * claim numbered after all earlier claims on that expert; it is kept iff the
+ * number is below C.  Stages run until all N choices were tried.
+ * In:  probs [T, N] fp32 (moe_route's full softmax), x [T, d] (nullable when
+ *      xe is NULL).
+ * Out: expert [T] int32 (the expert that kept the token; its first choice if
+ *      none did), gate [T] fp32 (probs[t, expert[t]]), pos [T] (claim number
+ *      on expert[t]; C if dropped), drop [T], counts [N] (claims on each
+ *      expert over all stages), kept [N] = min(counts, C), offsets [N + 1],
+ *      row_token / row_gate / xe as moe_dispatch (row offsets[e] + pos).
+ * Cost: N stages of four small kernels and two memsets. */
+int32_t moe_dispatch_ntlb(const moe_config* cfg, const void* x, const float* probs,
+                          int32_t* expert, float* gate, int32_t* pos, uint8_t* drop,
+                          int32_t* counts, int32_t* kept, int32_t* offsets,
+                          int32_t* row_token, float* row_gate, void* xe,
+                          void* ws, size_t ws_bytes, void* stream);
 
 /* ---- One routing group split over several shards (one per GPU) ------------
  * Capacity is defined per routing group, and claims follow token order over the

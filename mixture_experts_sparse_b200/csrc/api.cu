@@ -60,6 +60,8 @@ struct Layout {
     size_t idx, gate, pos, drop, counts, kept, offsets, f, P, aux;
     size_t row_token, row_gate, xe, h, ye;
     size_t prio_hist, prio_cursor, prio_list, prio_perm, prio_idx, prio_pos, prio_range;   // batch priority only
+    size_t ntlb_probs, ntlb_ch, ntlb_last, ntlb_first, ntlb_placed, ntlb_lp;               // re-routing only
+    size_t ntlb_claims, ntlb_st_counts, ntlb_st_kept, ntlb_st_offsets, ntlb_state;
     size_t total;
     int64_t rows;   // min(k T, N C): compact rows the buffers hold
 };
@@ -114,6 +116,19 @@ Layout layout_of(const moe_config& c) {
         L.prio_pos = take(4 * T * k);
         L.prio_range = take(8);
     }
+    if (c.priority == MOE_ORDER_NTLB) {   // No-Token-Left-Behind scratch
+        L.ntlb_probs = take(4 * T * N);
+        L.ntlb_ch = take(4 * T);
+        L.ntlb_last = take(4 * T);
+        L.ntlb_first = take(4 * T);
+        L.ntlb_placed = take(4 * T);
+        L.ntlb_lp = take(4 * T);
+        L.ntlb_claims = take(4 * (N + 1));
+        L.ntlb_st_counts = take(4 * (N + 1));
+        L.ntlb_st_kept = take(4 * (N + 1));
+        L.ntlb_st_offsets = take(4 * (N + 2));
+        L.ntlb_state = take(4 * nbs * (N + 1));
+    }
     L.total = off;
     return L;
 }
@@ -128,8 +143,10 @@ int32_t validate(const moe_config* c) {
     if (c->act != MOE_RELU && c->act != MOE_SWIGLU) return MOE_ERR_INVALID_ARG;
     if (c->top_k > c->n_experts) return MOE_ERR_INVALID_ARG;
     if (!std::isfinite(c->alpha)) return MOE_ERR_INVALID_ARG;
-    if (c->priority != MOE_ORDER_TOKEN && c->priority != MOE_ORDER_PRIORITY) return MOE_ERR_INVALID_ARG;
+    if (c->priority != MOE_ORDER_TOKEN && c->priority != MOE_ORDER_PRIORITY && c->priority != MOE_ORDER_NTLB)
+        return MOE_ERR_INVALID_ARG;
     if (c->T >= (1 << 28) || c->n_experts > 128 || c->top_k > 2) return MOE_ERR_UNSUPPORTED;
+    if (c->priority == MOE_ORDER_NTLB && c->top_k != 1) return MOE_ERR_UNSUPPORTED;   // re-routing is top-1
     if (c->dtype == MOE_BF16 && (c->d_model % 16 != 0 || c->d_ff % 16 != 0)) return MOE_ERR_UNSUPPORTED;
     if ((int64_t)c->d_model * c->d_ff >= ((int64_t)1 << 40)) return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
@@ -304,6 +321,68 @@ static int32_t dispatch_impl(const moe_config* cfg, const void* x, const int32_t
     return cuda_status(launch_dispatch(a, s));
 }
 
+// No-Token-Left-Behind dispatch from the router probabilities (top-1).
+static int32_t ntlb_impl(const moe_config* cfg, const void* x, const float* probs, int32_t* expert, float* gate,
+                         int32_t* pos, uint8_t* drop, int32_t* counts, int32_t* kept, int32_t* offsets,
+                         int32_t* row_token, float* row_gate, void* xe, void* zero_out, void* ws, cudaStream_t s,
+                         const AuxArgs* aux = nullptr) {
+    const Layout L = layout_of(*cfg);
+    if (cfg->T == 0) {
+        cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * cfg->n_experts, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(kept, 0, sizeof(int32_t) * cfg->n_experts, s);
+        if (e == cudaSuccess) e = cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (cfg->n_experts + 1), s);
+        return cuda_status(e);
+    }
+    NtlbArgs a{};
+    a.x = x;
+    a.dtype = cfg->dtype;
+    a.probs = probs;
+    a.T = cfg->T;
+    a.d = cfg->d_model;
+    a.N = cfg->n_experts;
+    a.C = cfg->capacity;
+    a.expert = expert;
+    a.gate = gate;
+    a.pos = pos;
+    a.drop = drop;
+    a.counts = counts;
+    a.kept = kept;
+    a.offsets = offsets;
+    a.row_token = row_token;
+    a.row_gate = row_gate;
+    a.xe = xe;
+    a.zero_out = zero_out;
+    a.ch = at<int32_t>(ws, L.ntlb_ch);
+    a.last = at<int32_t>(ws, L.ntlb_last);
+    a.first = at<int32_t>(ws, L.ntlb_first);
+    a.placed = at<int32_t>(ws, L.ntlb_placed);
+    a.lp = at<int32_t>(ws, L.ntlb_lp);
+    a.claims = at<int32_t>(ws, L.ntlb_claims);
+    a.st_counts = at<int32_t>(ws, L.ntlb_st_counts);
+    a.st_kept = at<int32_t>(ws, L.ntlb_st_kept);
+    a.st_offsets = at<int32_t>(ws, L.ntlb_st_offsets);
+    a.scan_state = at<uint32_t>(ws, L.ntlb_state);
+    a.hdr = at<WsHeader>(ws, L.hdr);
+    if (aux) a.aux = *aux;
+    return cuda_status(launch_dispatch_ntlb(a, s));
+}
+
+int32_t moe_dispatch_ntlb(const moe_config* cfg, const void* x, const float* probs, int32_t* expert, float* gate,
+                          int32_t* pos, uint8_t* drop, int32_t* counts, int32_t* kept, int32_t* offsets,
+                          int32_t* row_token, float* row_gate, void* xe, void* ws, size_t ws_bytes, void* stream) {
+    int32_t st = validate(cfg);
+    if (st != MOE_OK) return st;
+    if (cfg->priority != MOE_ORDER_NTLB) return MOE_ERR_INVALID_ARG;
+    if (!req(counts) || !req(kept) || !req(offsets) || !opt(xe) || !opt(x)) return MOE_ERR_INVALID_ARG;
+    if (cfg->T > 0 && (!req(probs) || !req(expert) || !req(gate) || !req(pos) || !req(drop) || !req(row_token) ||
+                       !req(row_gate)))
+        return MOE_ERR_INVALID_ARG;
+    if (xe && cfg->T > 0 && !req(x)) return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+    return ntlb_impl(cfg, x, probs, expert, gate, pos, drop, counts, kept, offsets, row_token, row_gate, xe, nullptr,
+                     ws, (cudaStream_t)stream);
+}
+
 int32_t moe_dispatch(const moe_config* cfg, const void* x, const int32_t* idx, const float* gate, int32_t* pos,
                      uint8_t* drop, int32_t* counts, int32_t* kept, int32_t* offsets, int32_t* row_token,
                      float* row_gate, void* xe, void* ws, size_t ws_bytes, void* stream) {
@@ -313,6 +392,7 @@ int32_t moe_dispatch(const moe_config* cfg, const void* x, const int32_t* idx, c
     if (cfg->T > 0 && (!req(idx) || !req(gate) || !req(pos) || !req(drop) || !req(row_token) || !req(row_gate)))
         return MOE_ERR_INVALID_ARG;
     if (xe && cfg->T > 0 && !req(x)) return MOE_ERR_INVALID_ARG;
+    if (cfg->priority == MOE_ORDER_NTLB) return MOE_ERR_UNSUPPORTED;   // needs the probabilities: moe_dispatch_ntlb
     if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
     return dispatch_impl(cfg, x, idx, gate, pos, drop, counts, kept, offsets, row_token, row_gate, xe, nullptr, ws,
                          (cudaStream_t)stream);
@@ -494,14 +574,20 @@ static int32_t forward_impl(const moe_config* cfg, const void* x, const float* w
         aa = AuxArgs{at<int32_t>(ws, L.part_cnt), at<float>(ws, L.part_psum), router_tc_grid(cfg->T, sms),
                      (int)cfg->n_experts, cfg->T, cfg->alpha, f, P, aux};
     }
-    st = route_impl(cfg, x, w_r, b_r, idx, gate, nullptr, f, P, aux, ws, ws_bytes, s, defer);
+    // re-routing needs every token's router probabilities
+    const bool ntlb = cfg->priority == MOE_ORDER_NTLB;
+    float* probs_ws = ntlb ? at<float>(ws, L.ntlb_probs) : nullptr;
+    st = route_impl(cfg, x, w_r, b_r, idx, gate, probs_ws, f, P, aux, ws, ws_bytes, s, defer);
     if (st != MOE_OK) return st;
     if (!mark(1)) return MOE_ERR_CUDA;
     // top-1 bf16: the second GEMM scatters gate * E(x) into out; dispatch zeroes
     // the rows of dropped tokens.  Otherwise expert outputs go through the combine.
     const bool fused = cfg->dtype == MOE_BF16 && cfg->top_k == 1;
-    st = dispatch_impl(cfg, x, idx, gate, pos, drop, counts, kept, offsets, row_token, row_gate, xe,
-                       fused ? out : nullptr, ws, s, nullptr, aa.G > 0 ? &aa : nullptr);
+    // re-routing overwrites idx and gate with the expert each token finally uses and its probability
+    st = ntlb ? ntlb_impl(cfg, x, probs_ws, idx, gate, pos, drop, counts, kept, offsets, row_token, row_gate, xe,
+                          fused ? out : nullptr, ws, s, aa.G > 0 ? &aa : nullptr)
+              : dispatch_impl(cfg, x, idx, gate, pos, drop, counts, kept, offsets, row_token, row_gate, xe,
+                              fused ? out : nullptr, ws, s, nullptr, aa.G > 0 ? &aa : nullptr);
     if (st != MOE_OK) return st;
     if (!mark(2)) return MOE_ERR_CUDA;
     st = ffn_impl(cfg, xe, offsets, w1, b1, w3, b3, w2, b2, ye, fused ? out : nullptr, row_token, row_gate, ws, s,

@@ -244,6 +244,22 @@ struct DispatchArgs {
     AuxArgs aux;                 // G > 0: one extra block of the gather reduces the router partials
     PrioArgs prio;               // batch priority (perm set) or token order
 };
+// No-Token-Left-Behind re-routing (top-1); all device, workspace-held scratch.
+struct NtlbArgs {
+    const void* x; int dtype; const float* probs;   // probs [T, N]
+    int64_t T; int d; int N; int C;
+    int32_t* expert; float* gate; int32_t* pos; uint8_t* drop;   // [T], token order
+    int32_t* counts; int32_t* kept; int32_t* offsets;            // [N], [N], [N + 1]
+    int32_t* row_token; float* row_gate; void* xe; void* zero_out;
+    int32_t* ch; int32_t* last; int32_t* first; int32_t* placed; int32_t* lp;   // [T] each
+    int32_t* claims;                                             // [N + 1]
+    int32_t* st_counts; int32_t* st_kept; int32_t* st_offsets;   // [N + 1], [N + 1], [N + 2]
+    uint32_t* scan_state;                                        // [scan_blocks(T) * (N + 1)]
+    WsHeader* hdr;
+    AuxArgs aux;
+};
+cudaError_t launch_dispatch_ntlb(const NtlbArgs& a, cudaStream_t s);
+
 int scan_blocks(int64_t T);
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s);
 cudaError_t launch_counts(const int32_t* idx, int64_t T, int N, int k, int32_t* counts, cudaStream_t s);

@@ -366,6 +366,108 @@ prio_rank_kernel(const float* __restrict__ gate, const int32_t* __restrict__ idx
     }
 }
 
+// ---- No-Token-Left-Behind re-routing (top-1) --------------------------------
+// CS25 Lecture 05 notes, "No Token Left Behind": a token whose expert is full
+// goes on to its second, third ... choice until it gets a slot.  Stage s: each
+// token still without a slot claims, in token order, on its (s+1)-th expert
+// (router probabilities descending, ties to the lower index), numbered after
+// every claim already made on that expert; kept iff that number is below C.
+// Per stage: ntlb_choose_kernel, the look-back scan over N + 1 experts (expert
+// N is the sink of tokens already placed), ntlb_place_kernel and
+// ntlb_claims_kernel; then ntlb_final_kernel, ntlb_offsets_kernel and the
+// gather.
+
+// expert a (probability pa) comes before expert b in a token's order
+__device__ __forceinline__ bool ntlb_before(float pa, int a, float pb, int b) {
+    return pa > pb || (pa == pb && a < b);
+}
+
+__global__ void __launch_bounds__(256)
+ntlb_choose_kernel(const float* __restrict__ probs, int64_t T, int N, int s, int32_t* __restrict__ placed,
+                   int32_t* __restrict__ last, int32_t* __restrict__ first, int32_t* __restrict__ ch) {
+    pdl_wait();
+    pdl_launch();
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < T; t += (int64_t)gridDim.x * blockDim.x) {
+        if (s == 0) placed[t] = 0;
+        else if (placed[t]) {
+            ch[t] = N;   // the sink: claims nothing
+            continue;
+        }
+        const float* p = probs + t * N;
+        const int le = s > 0 ? last[t] : -1;
+        const float lpv = s > 0 ? p[le] : 0.f;
+        int best = -1;
+        float bp = 0.f;
+        for (int e = 0; e < N; ++e) {   // the first expert after the previous choice
+            const float pe = p[e];
+            if (s > 0 && !ntlb_before(lpv, le, pe, e)) continue;
+            if (best < 0 || ntlb_before(pe, e, bp, best)) {
+                best = e;
+                bp = pe;
+            }
+        }
+        ch[t] = best;   // s < N: an untried expert is always left
+        last[t] = best;
+        if (s == 0) first[t] = best;
+    }
+}
+
+__global__ void __launch_bounds__(256)
+ntlb_place_kernel(const float* __restrict__ probs, int64_t T, int N, int C, const int32_t* __restrict__ ch,
+                  const int32_t* __restrict__ lp, const int32_t* __restrict__ claims, int32_t* __restrict__ placed,
+                  int32_t* __restrict__ expert, int32_t* __restrict__ pos, float* __restrict__ gate) {
+    pdl_wait();
+    pdl_launch();
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < T; t += (int64_t)gridDim.x * blockDim.x) {
+        const int e = ch[t];
+        if (e >= N) continue;
+        const int64_t c = (int64_t)claims[e] + lp[t];
+        if (c < (int64_t)C) {
+            placed[t] = 1;
+            expert[t] = e;
+            pos[t] = (int32_t)c;
+            gate[t] = probs[t * N + e];
+        }
+    }
+}
+
+__global__ void ntlb_claims_kernel(int N, const int32_t* __restrict__ st_counts, int32_t* __restrict__ claims) {
+    pdl_wait();
+    pdl_launch();
+    for (int e = threadIdx.x; e < N; e += blockDim.x) claims[e] += st_counts[e];
+}
+
+__global__ void __launch_bounds__(256)
+ntlb_final_kernel(const float* __restrict__ probs, int64_t T, int N, int C, const int32_t* __restrict__ placed,
+                  const int32_t* __restrict__ first, int32_t* __restrict__ expert, float* __restrict__ gate,
+                  int32_t* __restrict__ pos) {
+    pdl_wait();
+    pdl_launch();
+    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < T; t += (int64_t)gridDim.x * blockDim.x) {
+        if (placed[t]) continue;
+        const int e = first[t];   // dropped: its first choice, claim number C
+        expert[t] = e;
+        pos[t] = C;
+        gate[t] = probs[t * N + e];
+    }
+}
+
+__global__ void ntlb_offsets_kernel(int N, int C, const int32_t* __restrict__ claims, int32_t* __restrict__ counts,
+                                    int32_t* __restrict__ kept, int32_t* __restrict__ offsets) {
+    pdl_wait();
+    pdl_launch();
+    if (threadIdx.x != 0) return;
+    int32_t acc = 0;
+    for (int e = 0; e < N; ++e) {
+        const int32_t c = claims[e];
+        counts[e] = c;
+        kept[e] = c < C ? c : C;
+        offsets[e] = acc;
+        acc += kept[e];
+    }
+    offsets[N] = acc;
+}
+
 // Claims per (rank, expert) of this shard: counts[r][e] (int atomics, so the
 // result is exact and order-independent).
 __global__ void __launch_bounds__(256)
@@ -494,6 +596,58 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
                     a.gate, a.T, a.d, a.N, a.k, a.C, a.claim_base, a.pos, a.drop, a.counts, a.offsets, a.row_token,
                     a.row_gate, reinterpret_cast<float*>(a.xe), reinterpret_cast<float*>(a.zero_out), a.aux, perm,
                     pos_in);
+}
+
+cudaError_t launch_dispatch_ntlb(const NtlbArgs& a, cudaStream_t s) {
+    const int nblk = scan_blocks(a.T);
+    if (nblk == 0) return cudaSuccess;
+    const int N = a.N;
+    const unsigned g = (unsigned)((a.T + 255) / 256 < 4096 ? (a.T + 255) / 256 : 4096);
+    cudaError_t err = cudaMemsetAsync(a.claims, 0, sizeof(int32_t) * (N + 1), s);
+    if (err != cudaSuccess) return err;
+    for (int st = 0; st < N; ++st) {
+        if ((err = launch_k(ntlb_choose_kernel, dim3(g), dim3(256), 0, s, 1, a.probs, a.T, N, st, a.placed, a.last,
+                            a.first, a.ch)) != cudaSuccess)
+            return err;
+        if ((err = cudaMemsetAsync(&a.hdr->scan_ticket, 0, 2 * sizeof(int32_t), s)) != cudaSuccess) return err;
+        if ((err = cudaMemsetAsync(a.scan_state, 0, sizeof(uint32_t) * (size_t)nblk * (N + 1), s)) != cudaSuccess)
+            return err;
+        // this stage's claim numbers per expert in token order (no capacity: C = INT32_MAX)
+        if ((err = launch_k(scan_kernel, dim3((unsigned)nblk), dim3(kScanThreads), 0, s, 1,
+                            static_cast<const int32_t*>(a.ch), a.T, N + 1, 1, 0x7fffffff, nblk,
+                            static_cast<const int32_t*>(nullptr), a.lp, a.st_counts, a.st_kept, a.st_offsets,
+                            a.scan_state, a.hdr, kWaitLimitNs)) != cudaSuccess)
+            return err;
+        if ((err = launch_k(ntlb_place_kernel, dim3(g), dim3(256), 0, s, 1, a.probs, a.T, N, a.C,
+                            static_cast<const int32_t*>(a.ch), static_cast<const int32_t*>(a.lp),
+                            static_cast<const int32_t*>(a.claims), a.placed, a.expert, a.pos, a.gate)) != cudaSuccess)
+            return err;
+        if ((err = launch_k(ntlb_claims_kernel, dim3(1), dim3(128), 0, s, 1, N,
+                            static_cast<const int32_t*>(a.st_counts), a.claims)) != cudaSuccess)
+            return err;
+    }
+    if ((err = launch_k(ntlb_final_kernel, dim3(g), dim3(256), 0, s, 1, a.probs, a.T, N, a.C,
+                        static_cast<const int32_t*>(a.placed), static_cast<const int32_t*>(a.first), a.expert,
+                        a.gate, a.pos)) != cudaSuccess)
+        return err;
+    if ((err = launch_k(ntlb_offsets_kernel, dim3(1), dim3(32), 0, s, 1, N, a.C,
+                        static_cast<const int32_t*>(a.claims), a.counts, a.kept, a.offsets)) != cudaSuccess)
+        return err;
+    // the gather, from the final experts and claim numbers (rank 0, no claim base)
+    const unsigned grid = (unsigned)((a.T + 7) / 8) + (a.aux.G > 0 ? 1u : 0u);
+    const int32_t* none = nullptr;
+    if (a.dtype == MOE_BF16)
+        return launch_k(scatter_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, 1,
+                        reinterpret_cast<const __nv_bfloat16*>(a.x), static_cast<const int32_t*>(a.expert),
+                        static_cast<const float*>(a.gate), a.T, a.d, N, 1, a.C, none, a.pos, a.drop,
+                        static_cast<const int32_t*>(a.counts), static_cast<const int32_t*>(a.offsets), a.row_token,
+                        a.row_gate, reinterpret_cast<__nv_bfloat16*>(a.xe),
+                        reinterpret_cast<__nv_bfloat16*>(a.zero_out), a.aux, none, none);
+    return launch_k(scatter_kernel<float>, dim3(grid), dim3(256), 0, s, 1, reinterpret_cast<const float*>(a.x),
+                    static_cast<const int32_t*>(a.expert), static_cast<const float*>(a.gate), a.T, a.d, N, 1, a.C,
+                    none, a.pos, a.drop, static_cast<const int32_t*>(a.counts),
+                    static_cast<const int32_t*>(a.offsets), a.row_token, a.row_gate, reinterpret_cast<float*>(a.xe),
+                    reinterpret_cast<float*>(a.zero_out), a.aux, none, none);
 }
 
 cudaError_t launch_counts(const int32_t* idx, int64_t T, int N, int k, int32_t* counts, cudaStream_t s) {

@@ -85,7 +85,8 @@ extern "C" int32_t moe_dispatch_noalloc(const moe_config* cfg, const void* x, co
         (c.dtype != MOE_F32 && c.dtype != MOE_BF16) || (c.act != MOE_RELU && c.act != MOE_SWIGLU) ||
         c.top_k > c.n_experts)
         return MOE_ERR_INVALID_ARG;
-    if (c.priority != MOE_ORDER_TOKEN && c.priority != MOE_ORDER_PRIORITY) return MOE_ERR_INVALID_ARG;
+    if (c.priority != MOE_ORDER_TOKEN && c.priority != MOE_ORDER_PRIORITY && c.priority != MOE_ORDER_NTLB)
+        return MOE_ERR_INVALID_ARG;
     if (c.n_experts > 128 || c.top_k > 2 || (c.dtype == MOE_BF16 && (c.d_model % 16 != 0 || c.d_ff % 16 != 0)))
         return MOE_ERR_UNSUPPORTED;
     if (c.priority != MOE_ORDER_TOKEN) return MOE_ERR_UNSUPPORTED;   // its scratch has no room for the sort

@@ -41,6 +41,7 @@ _SIGS = {
     "moe_workspace_init": ([_P, ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_route": ([ctypes.POINTER(MoeConfig)] + [_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_route_z": ([ctypes.POINTER(MoeConfig)] + [_P] * 11 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_dispatch_ntlb": ([ctypes.POINTER(MoeConfig)] + [_P] * 13 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_dispatch": ([ctypes.POINTER(MoeConfig)] + [_P] * 12 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_expert_ffn": ([ctypes.POINTER(MoeConfig)] + [_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_combine": ([ctypes.POINTER(MoeConfig)] + [_P] * 8, ctypes.c_int32),
@@ -73,15 +74,16 @@ def lib():
     return _lib
 
 
-MOE_ORDER_TOKEN, MOE_ORDER_PRIORITY = 0, 1
+MOE_ORDER_TOKEN, MOE_ORDER_PRIORITY, MOE_ORDER_NTLB = 0, 1, 2
 
 
 def config(T, d_model, d_ff, n_experts, top_k, capacity, dtype="bf16", act="relu", alpha=1e-2, priority=False):
-    """moe_config; priority=True selects the batch-priority claim order."""
+    """moe_config.  priority: False/MOE_ORDER_TOKEN, True/MOE_ORDER_PRIORITY
+    (batch priority) or MOE_ORDER_NTLB (No-Token-Left-Behind re-routing)."""
+    order = MOE_ORDER_PRIORITY if priority is True else (MOE_ORDER_TOKEN if priority is False else int(priority))
     return MoeConfig(int(T), int(d_model), int(d_ff), int(n_experts), int(top_k), int(capacity),
                      MOE_BF16 if dtype in ("bf16", MOE_BF16) else MOE_F32,
-                     MOE_SWIGLU if act in ("swiglu", MOE_SWIGLU) else MOE_RELU, float(alpha),
-                     MOE_ORDER_PRIORITY if priority else MOE_ORDER_TOKEN)
+                     MOE_SWIGLU if act in ("swiglu", MOE_SWIGLU) else MOE_RELU, float(alpha), order)
 
 
 def _p(t):
@@ -146,6 +148,13 @@ def moe_route(cfg, x, w_r, b_r, idx, gate, probs, f, P, aux, ws, stream=None):
 def moe_route_z(cfg, x, w_r, b_r, idx, gate, probs, f, P, aux, z_loss, ws, stream=None):
     return lib().moe_route_z(ctypes.byref(cfg), _p(x), _p(w_r), _p(b_r), _p(idx), _p(gate), _p(probs),
                              _p(f), _p(P), _p(aux), _p(z_loss), _p(ws), _nbytes(ws), _s(stream))
+
+
+def moe_dispatch_ntlb(cfg, x, probs, expert, gate, pos, drop, counts, kept, offsets, row_token, row_gate, xe, ws,
+                      stream=None):
+    return lib().moe_dispatch_ntlb(ctypes.byref(cfg), _p(x), _p(probs), _p(expert), _p(gate), _p(pos), _p(drop),
+                                   _p(counts), _p(kept), _p(offsets), _p(row_token), _p(row_gate), _p(xe), _p(ws),
+                                   _nbytes(ws), _s(stream))
 
 
 def moe_dispatch(cfg, x, idx, gate, pos, drop, counts, kept, offsets, row_token, row_gate, xe, ws,

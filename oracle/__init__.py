@@ -296,14 +296,27 @@ def expert_rows(x, weights, rows_token, rows_expert, act=RELU):
     return ye
 
 
-def forward(x, w_r, b_r, weights, k, C, act=RELU, alpha=1e-2, out_dtype=F32, tokens=None, priority=False):
+def forward(x, w_r, b_r, weights, k, C, act=RELU, alpha=1e-2, out_dtype=F32, tokens=None, priority=False,
+            ntlb=False):
     """The whole layer, step by step: route, aux loss, slot claim (token order,
-    or batch priority), experts, combine.  tokens=None evaluates every token.
-    Returns a dict with every intermediate and the outputs for the evaluated
-    tokens."""
+    batch priority, or No-Token-Left-Behind re-routing for top-1), experts,
+    combine.  tokens=None evaluates every token.  Returns a dict with every
+    intermediate and the outputs for the evaluated tokens; with ntlb the
+    experts and gates used are in disp["expert"] / disp["gate"]."""
     routing = route(x, w_r, b_r, k)
     f, P, aux = aux_loss(routing["idx"], routing["probs"], alpha)
     N = np.asarray(w_r).shape[0]
+    if ntlb:
+        assert k == 1
+        disp = dispatch_ntlb(routing["probs"], routing["gate"][:, 0], C)
+        used = dict(idx=disp["expert"][:, None], gate=disp["gate"][:, None])
+        T = np.asarray(x).shape[0]
+        if tokens is None:
+            tokens = np.arange(T, dtype=np.int64)
+        out_exact, out_rounded = layer_tokens(x, weights, used, dict(drop=disp["drop"][:, None]), tokens, act,
+                                              out_dtype)
+        return dict(routing=routing, f=f, P=P, aux=aux, disp=disp, tokens=np.asarray(tokens),
+                    out_exact=out_exact, out=out_rounded)
     disp = dispatch(routing["idx"], N, C, priority=routing["gate"] if priority else None)
     T = np.asarray(x).shape[0]
     if tokens is None:

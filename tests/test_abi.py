@@ -63,8 +63,12 @@ def test_workspace_bytes_and_validation():
     prio = nat.config(4096, 768, 3072, 64, 1, 80, priority=True)
     assert nat.moe_workspace_bytes(prio) >= ws + 4 * (2 * 65536 + 1 + 4 * 4096)
     odd = nat.config(4096, 768, 3072, 64, 1, 80)
-    odd.priority = 2
+    odd.priority = 3
     assert nat.moe_workspace_bytes(odd) == 0
+    # re-routing keeps every token's probabilities and its stage state; top-1 only
+    ntlb = nat.config(4096, 768, 3072, 64, 1, 80, priority=nat.MOE_ORDER_NTLB)
+    assert nat.moe_workspace_bytes(ntlb) >= ws + 4 * 4096 * 64
+    assert nat.moe_workspace_bytes(nat.config(4096, 768, 3072, 64, 2, 80, priority=nat.MOE_ORDER_NTLB)) == 0
 
 
 def test_host_validation_rejects_before_launch():

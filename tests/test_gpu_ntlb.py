@@ -1,0 +1,109 @@
+"""No-Token-Left-Behind re-routing (moe_dispatch_ntlb, moe_config.priority =
+MOE_ORDER_NTLB) through the C ABI against the oracle (CS25 Lecture 05 notes,
+"No Token Left Behind": a token whose expert is full goes on to its next
+choices until it gets a slot; top-1).  Needs a B200.
+
+Dispatch level: both sides get the oracle's router probabilities, so every
+output is identical.  Layer level: the GPU router's probabilities differ from
+the oracle's in the last bits, so a token whose next choices are near-tied may
+take another expert; the test requires agreement on almost every token,
+checks the GPU result is a valid re-routing (a token drops only when every
+expert is full; compact rows tile exactly), and compares outputs wherever
+expert and keep/drop agree."""
+import numpy as np
+import pytest
+
+import oracle
+from gpu_helpers import assert_close_out, widen_out
+from mixture_experts_sparse_b200 import inputs
+from mixture_experts_sparse_b200 import native as nat
+from mixture_experts_sparse_b200.layer import MoeLayer, to_device, to_host_bits
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+
+def _gpu_ntlb(L, probs, T, d, N, C):
+    cfg = nat.config(T, d, 64, N, 1, C, priority=nat.MOE_ORDER_NTLB)
+    ws = nat.new_workspace(cfg)
+    R = max(1, min(T, N * C))
+    dev = dict(device="cuda")
+    out = dict(expert=torch.full((T,), -7, dtype=torch.int32, **dev),
+               gate=torch.full((T,), -1.0, dtype=torch.float32, **dev),
+               pos=torch.full((T,), -7, dtype=torch.int32, **dev),
+               drop=torch.full((T,), 9, dtype=torch.uint8, **dev),
+               counts=torch.empty(N, dtype=torch.int32, **dev),
+               kept=torch.empty(N, dtype=torch.int32, **dev),
+               offsets=torch.empty(N + 1, dtype=torch.int32, **dev),
+               row_token=torch.full((R,), -1, dtype=torch.int32, **dev),
+               row_gate=torch.empty(R, dtype=torch.float32, **dev),
+               xe=torch.zeros(R, d, dtype=torch.bfloat16, **dev))
+    nat.check(nat.moe_dispatch_ntlb(cfg, to_device(L["x"]), to_device(probs), out["expert"], out["gate"], out["pos"],
+                                    out["drop"], out["counts"], out["kept"], out["offsets"], out["row_token"],
+                                    out["row_gate"], out["xe"], ws))
+    torch.cuda.synchronize()
+    nat.check(nat.moe_read_device_status(ws))
+    return {key: (to_host_bits(v) if key == "xe" else v.cpu().numpy()) for key, v in out.items()}
+
+
+@pytest.mark.parametrize("T,N,cf,bias,ties", [(4099, 7, 1.0, 0.8, False), (3000, 16, 1.25, 1.5, False),
+                                              (2000, 8, 0.5, 0.0, False), (1000, 1, 0.5, 0.0, False),
+                                              (1500, 6, 1.0, 1.0, True), (700, 5, 0.0, 0.5, False)])
+def test_ntlb_dispatch_exact(T, N, cf, bias, ties):
+    d = 128
+    rb = np.linspace(bias, 0.0, N).astype(np.float32) if bias else None
+    L = inputs.make_layer(T=T, d_model=d, d_ff=64, n_experts=N, top_k=1, dtype="bf16", seed=T + N, router_bias=rb)
+    r = oracle.route(L["x"], L["w_r"], L["b_r"], 1)
+    probs = r["probs"]
+    if ties:   # few distinct values: many equal probabilities, ties to the lower expert index
+        probs = (np.round(probs * 8.0) / 8.0).astype(np.float32)
+    C = nat.moe_capacity(T, N, 1, cf)
+    first = np.array([min(range(N), key=lambda e: (-float(probs[t, e]), e)) for t in range(T)])
+    want = oracle.dispatch_ntlb(probs, probs[np.arange(T), first], C)
+    got = _gpu_ntlb(L, probs, T, d, N, C)
+    for key in ("expert", "gate", "pos", "drop", "counts", "kept", "offsets"):
+        np.testing.assert_array_equal(got[key], want[key], err_msg=key)
+    nrows = int(want["offsets"][-1])
+    kept_t = np.nonzero(want["drop"] == 0)[0]
+    rows = want["offsets"][want["expert"][kept_t]] + want["pos"][kept_t]
+    want_t = np.full(nrows, -1)
+    want_t[rows] = kept_t
+    np.testing.assert_array_equal(got["row_token"][:nrows], want_t)
+    np.testing.assert_array_equal(got["row_gate"][:nrows], want["gate"][want_t])
+    np.testing.assert_array_equal(got["xe"][:nrows], L["x"][want_t])
+
+
+@pytest.mark.parametrize("case", [(3000, 128, 256, 8, 1.0, "relu", "bf16", 1.0), (900, 64, 128, 5, 1.25, "relu", "f32", 0.8)],
+                         ids=lambda c: "T%d_N%d_%s" % (c[0], c[3], c[6]))
+def test_ntlb_layer_against_oracle(case):
+    T, d, dff, N, cf, act, dtype, bias = case
+    L = inputs.make_layer(T=T, d_model=d, d_ff=dff, n_experts=N, top_k=1, act=act, dtype=dtype, seed=9,
+                          biases=(dtype == "f32"), router_bias=np.linspace(bias, 0.0, N).astype(np.float32))
+    C = nat.moe_capacity(T, N, 1, cf)
+    layer = MoeLayer(T, d, dff, N, 1, C, dtype, act, L, priority=nat.MOE_ORDER_NTLB)
+    nat.check(layer.forward(to_device(L["x"])))
+    torch.cuda.synchronize()
+    nat.check(nat.moe_read_device_status(layer.ws))
+    res = oracle.forward(L["x"], L["w_r"], L["b_r"], {key: L[key] for key in ("w1", "b1", "w3", "b3", "w2", "b2")},
+                         k=1, C=C, act=oracle.RELU, out_dtype=oracle.BF16 if dtype == "bf16" else oracle.F32,
+                         ntlb=True)
+    dd = res["disp"]
+    expert = layer.idx.cpu().numpy()[:, 0]
+    drop = layer.drop.cpu().numpy()[:, 0]
+    pos = layer.pos.cpu().numpy()[:, 0]
+    kept = layer.kept.cpu().numpy()
+    offsets = layer.offsets.cpu().numpy()
+    # a valid re-routing: drops only when every expert is full, rows tile exactly
+    assert int(kept.sum()) == min(T, N * C) and np.all(kept <= C)
+    assert int((drop == 0).sum()) == int(kept.sum())
+    rows = offsets[expert[drop == 0]] + pos[drop == 0]
+    assert sorted(rows.tolist()) == list(range(int(kept.sum())))
+    same = (expert == dd["expert"]) & (drop == dd["drop"])
+    assert same.mean() > 0.99, same.mean()
+    got = widen_out(layer.out) if dtype == "bf16" else layer.out.cpu().numpy().astype(np.float64)
+    assert_close_out(got[same], res["out_exact"][same], dtype)
+    # the aux loss is the router's (pre-capacity top-1), unchanged by re-routing
+    np.testing.assert_array_equal(layer.f.cpu().numpy(), res["f"])
