@@ -107,3 +107,38 @@ def test_ntlb_layer_against_oracle(case):
     assert_close_out(got[same], res["out_exact"][same], dtype)
     # the aux loss is the router's (pre-capacity top-1), unchanged by re-routing
     np.testing.assert_array_equal(layer.f.cpu().numpy(), res["f"])
+
+
+def test_ntlb_dispatch_time_at_switch_base_size():
+    # T = 65536 tokens, 64 experts, cf 1.0, skewed synthetic probabilities:
+    # time the re-routing dispatch (reported, not asserted beyond completion)
+    T, d, N = 65536, 768, 64
+    rng = np.random.default_rng(4)
+    h = rng.standard_normal((T, N)).astype(np.float32) + np.linspace(1.0, 0.0, N, dtype=np.float32)
+    p = np.exp(h - h.max(axis=1, keepdims=True))
+    probs = (p / p.sum(axis=1, keepdims=True)).astype(np.float32)
+    L = dict(x=rng.integers(0, 1 << 15, size=(T, d)).astype(np.uint16))
+    C = nat.moe_capacity(T, N, 1, 1.0)
+    cfg = nat.config(T, d, 64, N, 1, C, priority=nat.MOE_ORDER_NTLB)
+    ws = nat.new_workspace(cfg)
+    R = min(T, N * C)
+    dev = dict(device="cuda")
+    bufs = [torch.empty(T, dtype=torch.int32, **dev), torch.empty(T, dtype=torch.float32, **dev),
+            torch.empty(T, dtype=torch.int32, **dev), torch.empty(T, dtype=torch.uint8, **dev),
+            torch.empty(N, dtype=torch.int32, **dev), torch.empty(N, dtype=torch.int32, **dev),
+            torch.empty(N + 1, dtype=torch.int32, **dev), torch.empty(R, dtype=torch.int32, **dev),
+            torch.empty(R, dtype=torch.float32, **dev), torch.empty(R, d, dtype=torch.bfloat16, **dev)]
+    x, pr = to_device(L["x"]), to_device(probs)
+    nat.check(nat.moe_dispatch_ntlb(cfg, x, pr, *bufs, ws))
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    ev[0].record()
+    for _ in range(5):
+        nat.check(nat.moe_dispatch_ntlb(cfg, x, pr, *bufs, ws))
+    ev[1].record()
+    torch.cuda.synchronize()
+    nat.check(nat.moe_read_device_status(ws))
+    kept = bufs[5].cpu().numpy()
+    assert int(kept.sum()) == min(T, N * C)
+    print(f"\nre-routing dispatch at T={T}, N={N}, C={C}: {ev[0].elapsed_time(ev[1]) / 5 * 1e3:.1f} us, "
+          f"{int((bufs[3] == 0).sum())} tokens kept")
