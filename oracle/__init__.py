@@ -49,6 +49,7 @@ def _load():
         lib.oracle_dispatch.argtypes = [i64, i32, i32, i32, P, P, P, P, P, P]
         lib.oracle_dispatch_ordered.argtypes = [i64, i32, i32, i32, P, P, P, P, P, P, P]
         lib.oracle_dispatch_ntlb.argtypes = [i64, i32, i32, P, P, P, P, P, P, P, P, P]
+        lib.oracle_router_backward.argtypes = [i64, i32, i32, i32, P, i32, P, P, P, P, P, P, f64, P, P, P, P]
         lib.oracle_dispatch.restype = None
         lib.oracle_expert_ffn.argtypes = [i32, i32, i32, P, i32, sz, P, P, P, P, P, P, i32,
                                           sz, sz, sz, sz, P, P]
@@ -136,6 +137,32 @@ def z_loss(logits):
     logits = np.ascontiguousarray(logits, dtype=np.float32)
     T, N = logits.shape
     return float(lib.oracle_z_loss(T, N, _ptr(logits)))
+
+
+def router_backward(x, w_r, probs, idx, gate, f, dgate, alpha=1e-2):
+    """Router backward: gradients of sum dgate * gate + L_aux with respect to
+    the router logits, W_r, b_r and x (gate path of "From Switch Transformer to
+    GLaM"; load-balancing gradient through P_i with coefficient f_i, CMU 10-423
+    Lecture 16 section 4.2).  Returns dict(dh [T,N], dw [N,d], db [N], dx [T,d])
+    in fp64."""
+    lib = _load()
+    x, xd = _as_input(x)
+    T, d = x.shape
+    w_r = np.ascontiguousarray(w_r, dtype=np.float32)
+    N = w_r.shape[0]
+    probs = np.ascontiguousarray(probs, dtype=np.float32)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    k = idx.shape[1]
+    gate = np.ascontiguousarray(gate, dtype=np.float32)
+    f = np.ascontiguousarray(f, dtype=np.float64)
+    dgate = np.ascontiguousarray(dgate, dtype=np.float32)
+    dh = np.empty((T, N), np.float64)
+    dw = np.empty((N, d), np.float64)
+    db = np.empty(N, np.float64)
+    dx = np.empty((T, d), np.float64)
+    lib.oracle_router_backward(T, d, N, k, _ptr(x), xd, _ptr(w_r), _ptr(probs), _ptr(idx), _ptr(gate), _ptr(f),
+                               _ptr(dgate), float(alpha), _ptr(dh), _ptr(dw), _ptr(db), _ptr(dx))
+    return dict(dh=dh, dw=dw, db=db, dx=dx)
 
 
 def aux_loss(idx, probs, alpha=1e-2):

@@ -207,6 +207,63 @@ void oracle_aux(int64_t T, int32_t N, int32_t k, const int32_t* idx, const float
     *aux = alpha * (double)N * s;
 }
 
+/* ---- Router backward -------------------------------------------------------
+ * Gradient of L = sum_{t,r} dgate[t,r] g_{t,r}(h) + L_aux(h) with respect to the
+ * router logits h, the router weights and bias, and the router's input x.
+ *  - gate path ("From Switch Transformer to GLaM": y = p_{i*} E_{i*}(x) for
+ *    top-1; y = w1 E_{i1} + w2 E_{i2} with w the softmax over the two kept
+ *    logits for top-2; the expert choice itself has no gradient):
+ *      top-1: g = p_{i*}, dg/dh_j = p_{i*} (delta_{j i*} - p_j);
+ *      top-2: g1 = 1 / (1 + e^{h2 - h1}), g2 = 1 - g1; dg1/dh1 = -dg1/dh2 =
+ *             g1 g2, and g2 the opposite.
+ *  - load-balancing loss (CMU 10-423 Lecture 16, section 4.2: f_i is counted
+ *    and carries no gradient; the gradient flows through P_i with coefficient
+ *    f_i): dL_aux/dp_{t,i} = alpha N f_i / T, then through the softmax:
+ *    dh_{t,j} = p_{t,j} (a_j - sum_i p_{t,i} a_i), a_i = alpha N f_i / T.
+ *  - dW_r[i, :] = sum_t dh_{t,i} x_t, db_r[i] = sum_t dh_{t,i},
+ *    dx_t = sum_i dh_{t,i} W_r[i, :]  (h = W_r x + b_r).
+ * probs [T, N] and gate [T, k] are the forward's fp32 values; f [N] double.
+ * Outputs in double: dh [T, N], dw [N, d], db [N], dx [T, d]. */
+void oracle_router_backward(int64_t T, int32_t d, int32_t N, int32_t k,
+                            const void* x, int32_t x_dtype, const float* w_r,
+                            const float* probs, const int32_t* idx, const float* gate,
+                            const double* f, const float* dgate, double alpha,
+                            double* dh, double* dw, double* db, double* dx) {
+    double a[1024];
+    for (int32_t i = 0; i < N; ++i) a[i] = T > 0 ? alpha * (double)N * f[i] / (double)T : 0.0;
+    for (int32_t i = 0; i < N; ++i) {
+        db[i] = 0.0;
+        for (int32_t j = 0; j < d; ++j) dw[(size_t)i * d + j] = 0.0;
+    }
+    for (int64_t t = 0; t < T; ++t) {
+        const float* p = probs + (size_t)t * N;
+        double* g = dh + (size_t)t * N;
+        double spa = 0.0;
+        for (int32_t i = 0; i < N; ++i) spa += (double)p[i] * a[i];
+        for (int32_t j = 0; j < N; ++j) g[j] = (double)p[j] * (a[j] - spa);
+        if (k == 1) {
+            const int32_t is = idx[t];
+            const double gs = (double)gate[t], dg = (double)dgate[t];
+            for (int32_t j = 0; j < N; ++j) g[j] += dg * gs * ((j == is ? 1.0 : 0.0) - (double)p[j]);
+        } else {
+            const int32_t i1 = idx[t * 2], i2 = idx[t * 2 + 1];
+            const double g1 = (double)gate[t * 2], g2 = (double)gate[t * 2 + 1];
+            const double c = (double)dgate[t * 2] - (double)dgate[t * 2 + 1];
+            g[i1] += c * g1 * g2;
+            g[i2] -= c * g1 * g2;
+        }
+        for (int32_t i = 0; i < N; ++i) {
+            db[i] += g[i];
+            for (int32_t j = 0; j < d; ++j) dw[(size_t)i * d + j] += g[i] * load_elem(x, x_dtype, (size_t)t * d + j);
+        }
+        for (int32_t j = 0; j < d; ++j) {
+            double acc = 0.0;
+            for (int32_t i = 0; i < N; ++i) acc += g[i] * (double)w_r[(size_t)i * d + j];
+            dx[(size_t)t * d + j] = acc;
+        }
+    }
+}
+
 /* ---- Capacity --------------------------------------------------------------
  * C = floor(k * T * cf / N), exact.  cf is a binary double m * 2^e with m an
  * odd-or-zero 53-bit integer, so k T cf / N = k T m / (N 2^-e) is a rational

@@ -434,6 +434,73 @@ def test_ntlb_small_hand_example():
     np.testing.assert_allclose(got["gate"], [0.9, 0.2, 0.7])
 
 
+# ------------------------------------------------------ router backward ----
+
+def _fwd_loss(x, w, b, idx, f, dgate, alpha):
+    """sum dgate * gate + L_aux in fp64, with the expert selection and f held
+    fixed (the forward's definitions: softmax router, top-1 gate p_{i*} or the
+    softmax over the two kept logits, aux = alpha N sum f_i P_i)."""
+    h = x @ w.T + b
+    p = np.exp(h - h.max(axis=1, keepdims=True))
+    p /= p.sum(axis=1, keepdims=True)
+    T, N = p.shape
+    k = idx.shape[1]
+    if k == 1:
+        g = p[np.arange(T), idx[:, 0]][:, None]
+    else:
+        h1, h2 = h[np.arange(T), idx[:, 0]], h[np.arange(T), idx[:, 1]]
+        g1 = 1.0 / (1.0 + np.exp(h2 - h1))
+        g = np.stack([g1, 1.0 - g1], axis=1)
+    return float((dgate * g).sum() + alpha * N * (f * p.mean(axis=0)).sum()), p, g
+
+
+@pytest.mark.parametrize("k", [1, 2])
+def test_router_backward_matches_finite_differences(k):
+    rng = np.random.default_rng(40 + k)
+    T, N, d, alpha = 6, 5, 4, 0.3
+    x = rng.standard_normal((T, d))
+    w = rng.standard_normal((N, d)) * 0.7
+    b = rng.standard_normal(N) * 0.2
+    h = x @ w.T + b
+    idx = np.argsort(-h, axis=1, kind="stable")[:, :k].astype(np.int32)
+    f = rng.random(N)
+    f /= f.sum()
+    dgate = rng.standard_normal((T, k))
+    _, p, g = _fwd_loss(x, w, b, idx, f, dgate, alpha)
+    got = oracle.router_backward(x.astype(np.float32), w.astype(np.float32), p.astype(np.float32), idx,
+                                 g.astype(np.float32), f, dgate.astype(np.float32), alpha)
+    # the oracle reads x and W_r as fp32: differentiate at those values
+    x32, w32 = x.astype(np.float32).astype(np.float64), w.astype(np.float32).astype(np.float64)
+    dg32 = dgate.astype(np.float32).astype(np.float64)
+
+    def num_grad(fun, a, eps=1e-6):
+        out = np.zeros_like(a)
+        for i in np.ndindex(a.shape):
+            hi, lo = a.copy(), a.copy()
+            hi[i] += eps
+            lo[i] -= eps
+            out[i] = (fun(hi) - fun(lo)) / (2 * eps)
+        return out
+
+    L = lambda xx, ww, bb: _fwd_loss(xx, ww, bb, idx, f, dg32, alpha)[0]
+    np.testing.assert_allclose(got["dw"], num_grad(lambda ww: L(x32, ww, b), w32), rtol=2e-5, atol=1e-7)
+    np.testing.assert_allclose(got["db"], num_grad(lambda bb: L(x32, w32, bb), b.copy()), rtol=2e-5, atol=1e-7)
+    np.testing.assert_allclose(got["dx"], num_grad(lambda xx: L(xx, w32, b), x32), rtol=2e-5, atol=1e-7)
+
+
+def test_router_backward_uniform_f_has_no_aux_gradient():
+    # equal f_i: dL_aux/dp_{t,i} is the same for every expert, and the softmax
+    # Jacobian maps a constant vector to zero
+    rng = np.random.default_rng(44)
+    T, N, d = 7, 6, 5
+    x = rng.standard_normal((T, d)).astype(np.float32)
+    w = rng.standard_normal((N, d)).astype(np.float32)
+    r = oracle.route(x, w, None, 1)
+    got = oracle.router_backward(x, w, r["probs"], r["idx"], r["gate"], np.full(N, 1.0 / N), np.zeros((T, 1), np.float32),
+                                 alpha=0.5)
+    assert np.abs(got["dh"]).max() < 1e-7
+
+
 def test_gshard_rank_major_example():
     # CMU 10-423 Lecture 16 section 6.1 (b): 3 devices of capacity 3; first choices are
     # placed before second choices, so a token's second choice can find its expert full.
