@@ -149,6 +149,24 @@ int32_t moe_route_z(const moe_config* cfg, const void* x, const float* w_r, cons
                     double* f, double* P, double* aux, double* z_loss,
                     void* ws, size_t ws_bytes, void* stream);
 
+/* Router backward (fp32): gradients of L = sum_{t,r} dgate[t,r] gate[t,r] +
+ * L_aux with respect to the router logits, W_r, b_r and the router input x.
+ * Gate path ("From Switch Transformer to GLaM": top-1 gate p_{i*}, top-2 the
+ * softmax over the two kept logits; the expert choice has no gradient) and
+ * the load-balancing loss with f held constant (CMU 10-423 Lecture 16,
+ * section 4.2: dL_aux/dp_{t,i} = alpha N f_i / T, alpha = cfg->alpha).
+ * In:  x [T, d] (dtype), w_r [N, d], probs [T, N] (moe_route's full softmax),
+ *      idx, gate [T, k] (moe_route's), f [N] fp64 (moe_route's), dgate [T, k]
+ *      fp32 (dL/dgate: <dL/dout_t, E_{idx}(x_t)> for a kept assignment, 0
+ *      for a dropped one).
+ * Out: dh [T, N] fp32 (dL/dh); dw_r [N, d], db_r [N], dx [T, d] fp32 (each
+ *      nullable; dx is the router's part of dL/dx).  Sums over tokens run per
+ *      512-token chunk in fp32 and over chunks in fp64, in a fixed order. */
+int32_t moe_router_backward(const moe_config* cfg, const void* x, const float* w_r, const float* probs,
+                            const int32_t* idx, const float* gate, const double* f, const float* dgate,
+                            float* dh, float* dw_r, float* db_r, float* dx,
+                            void* ws, size_t ws_bytes, void* stream);
+
 /* Capacity-limited dispatch (row A3 and the gather of A4).
  * In:  x [T, d] (dtype; nullable when xe is NULL), idx [T, k], gate [T, k].
  * Out: pos [T, k] int32 (claim number of the assignment on its expert: all

@@ -62,6 +62,7 @@ struct Layout {
     size_t prio_hist, prio_cursor, prio_list, prio_perm, prio_idx, prio_pos, prio_range;   // batch priority only
     size_t ntlb_probs, ntlb_ch, ntlb_last, ntlb_first, ntlb_placed, ntlb_lp;               // re-routing only
     size_t ntlb_claims, ntlb_st_counts, ntlb_st_kept, ntlb_st_offsets, ntlb_state;
+    size_t bwd_part_dw, bwd_part_db;   // router backward partials
     size_t total;
     int64_t rows;   // min(k T, N C): compact rows the buffers hold
 };
@@ -107,6 +108,9 @@ Layout layout_of(const moe_config& c) {
     L.xe = take(esz * R * (size_t)c.d_model);
     L.h = take(esz * R * (size_t)c.d_ff);
     L.ye = take(esz * R * (size_t)c.d_model);
+    const size_t nch = (size_t)router_bwd_chunks(c.T);
+    L.bwd_part_dw = take(4 * nch * N * (size_t)c.d_model);
+    L.bwd_part_db = take(4 * nch * N);
     if (c.priority == MOE_ORDER_PRIORITY) {   // batch-priority claim order scratch
         L.prio_hist = take(4 * (size_t)(kPrioBuckets + 1));
         L.prio_cursor = take(4 * (size_t)kPrioBuckets);
@@ -381,6 +385,39 @@ int32_t moe_dispatch_ntlb(const moe_config* cfg, const void* x, const float* pro
     if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
     return ntlb_impl(cfg, x, probs, expert, gate, pos, drop, counts, kept, offsets, row_token, row_gate, xe, nullptr,
                      ws, (cudaStream_t)stream);
+}
+
+int32_t moe_router_backward(const moe_config* cfg, const void* x, const float* w_r, const float* probs,
+                            const int32_t* idx, const float* gate, const double* f, const float* dgate, float* dh,
+                            float* dw_r, float* db_r, float* dx, void* ws, size_t ws_bytes, void* stream) {
+    int32_t st = validate(cfg);
+    if (st != MOE_OK) return st;
+    if (!req(w_r) || !req(f) || !opt(dw_r) || !opt(db_r) || !opt(dx)) return MOE_ERR_INVALID_ARG;
+    if (cfg->T > 0 && (!req(x) || !req(probs) || !req(idx) || !req(gate) || !req(dgate) || !req(dh)))
+        return MOE_ERR_INVALID_ARG;
+    if ((st = check_ws(cfg, ws, ws_bytes)) != MOE_OK) return st;
+    const Layout L = layout_of(*cfg);
+    RouterBwdArgs a{};
+    a.x = x;
+    a.dtype = cfg->dtype;
+    a.w_r = w_r;
+    a.probs = probs;
+    a.idx = idx;
+    a.gate = gate;
+    a.f = f;
+    a.dgate = dgate;
+    a.alpha = cfg->alpha;
+    a.T = cfg->T;
+    a.d = cfg->d_model;
+    a.N = cfg->n_experts;
+    a.k = cfg->top_k;
+    a.dh = dh;
+    a.dw = dw_r;
+    a.db = db_r;
+    a.dx = dx;
+    a.part_dw = at<float>(ws, L.bwd_part_dw);
+    a.part_db = at<float>(ws, L.bwd_part_db);
+    return cuda_status(launch_router_backward(a, (cudaStream_t)stream));
 }
 
 int32_t moe_dispatch(const moe_config* cfg, const void* x, const int32_t* idx, const float* gate, int32_t* pos,

@@ -206,6 +206,17 @@ struct RouterArgs {
     bool defer_aux;                        // tensor-core router: leave f, P, aux to aux_reduce_block
 };
 int router_tc_grid(int64_t T, int sms);            // CTAs of the tensor-core router (= partial rows used)
+
+struct RouterBwdArgs {
+    const void* x; int dtype; const float* w_r;
+    const float* probs; const int32_t* idx; const float* gate; const double* f; const float* dgate;
+    float alpha; int64_t T; int d; int N; int k;
+    float* dh;                        // [T, N]
+    float* dw; float* db; float* dx;  // [N, d], [N], [T, d] (each nullable)
+    float* part_dw; float* part_db;   // [router_bwd_chunks(T), N, d], [.., N]
+};
+int router_bwd_chunks(int64_t T);
+cudaError_t launch_router_backward(const RouterBwdArgs& a, cudaStream_t s);
 int router_blocks(int64_t T, int N);               // partial rows the FP32-pipe router writes
 int router_partial_rows(int64_t T, int N);         // partial rows any router path writes
 int router_tc_padded_experts(int N);

@@ -1,0 +1,251 @@
+// Router backward on the FP32 pipe: gradients of sum_{t,r} dgate[t,r] g_{t,r}
+// + L_aux with respect to the router logits h, W_r, b_r and the router input x.
+//
+//  - gate path ("From Switch Transformer to GLaM": y = p_{i*} E_{i*}(x) for
+//    top-1, y = w1 E_{i1} + w2 E_{i2} with w the softmax over the two kept
+//    logits for top-2; the expert choice itself carries no gradient):
+//      top-1: dh_j += dgate p_{i*} (delta_{j i*} - p_j);
+//      top-2: dh_{i1} += (dg1 - dg2) g1 g2, dh_{i2} -= (dg1 - dg2) g1 g2.
+//  - load-balancing loss (CMU 10-423 Lecture 16, section 4.2: f_i is counted
+//    and carries no gradient, P_i = mean_t p_{t,i} carries coefficient f_i):
+//      dh_j += p_j (a_j - sum_i p_i a_i), a_i = alpha N f_i / T.
+//  - dW_r = dh^T x, db_r = sum_t dh_t (a contraction over tokens: per
+//    512-token chunk partials, then a fixed-order fp64 sum over chunks), and
+//    dx_t = dh_t W_r.
+// Kernels: router_bwd_dh_kernel (one warp per token), router_bwd_dw_kernel
+// (32 experts x 128 columns per block over one token chunk),
+// router_bwd_reduce_kernel, router_bwd_dx_kernel (64 tokens x 128 columns).
+// All sums run in a fixed order: results are bit-identical run to run.
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kBwdChunk = 512;   // tokens per dW_r partial
+
+__global__ void __launch_bounds__(256)
+router_bwd_dh_kernel(const float* __restrict__ probs, const int32_t* __restrict__ idx, const float* __restrict__ gate,
+                     const float* __restrict__ dgate, const double* __restrict__ f, float alpha, int64_t T, int N,
+                     int k, float* __restrict__ dh) {
+    pdl_wait();
+    pdl_launch();
+    const int lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (t >= T) return;
+    const float* p = probs + t * N;
+    float pv[4], av[4];
+    float spa = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int e = lane + 32 * q;
+        pv[q] = e < N ? p[e] : 0.f;
+        av[q] = e < N ? (float)((double)alpha * (double)N * f[e] / (double)T) : 0.f;
+        spa = fmaf(pv[q], av[q], spa);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) spa += __shfl_xor_sync(0xffffffffu, spa, o);
+    float gv[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) gv[q] = pv[q] * (av[q] - spa);
+    if (k == 1) {
+        const int is = idx[t];
+        const float c = dgate[t] * gate[t];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int e = lane + 32 * q;
+            gv[q] += c * ((e == is ? 1.f : 0.f) - pv[q]);
+        }
+    } else {
+        const int i1 = idx[2 * t], i2 = idx[2 * t + 1];
+        const float g1 = gate[2 * t], g2 = gate[2 * t + 1];
+        const float c = (dgate[2 * t] - dgate[2 * t + 1]) * g1 * g2;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int e = lane + 32 * q;
+            if (e == i1) gv[q] += c;
+            if (e == i2) gv[q] -= c;
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int e = lane + 32 * q;
+        if (e < N) dh[t * N + e] = gv[q];
+    }
+}
+
+// part_dw[chunk][n][c] = sum over the chunk's tokens of dh[t][n] x[t][c];
+// blocks with blockIdx.z == 0 also write part_db[chunk][n].
+template <typename XT>
+__global__ void __launch_bounds__(256)
+router_bwd_dw_kernel(const float* __restrict__ dh, const XT* __restrict__ x, int64_t T, int N, int d,
+                     float* __restrict__ part_dw, float* __restrict__ part_db) {
+    pdl_wait();
+    pdl_launch();
+    __shared__ float s_dh[32][33];    // [token][expert]
+    __shared__ float s_x[32][132];    // [token][column]
+    const int tid = threadIdx.x;
+    const int chunk = blockIdx.x, n0 = blockIdx.y * 32, c0 = blockIdx.z * 128;
+    const int64_t t_lo = (int64_t)chunk * kBwdChunk;
+    const int64_t t_hi = t_lo + kBwdChunk < T ? t_lo + kBwdChunk : T;
+    const int tn = tid >> 5, tc = tid & 31;   // thread: experts 4 tn .. 4 tn + 3, columns tc + 32 j
+    float acc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    float dbacc = 0.f;   // thread tid < 32: expert n0 + tid
+    for (int64_t t0 = t_lo; t0 < t_hi; t0 += 32) {
+        for (int q = tid; q < 32 * 32; q += 256) {
+            const int r = q >> 5, c = q & 31;
+            const int64_t t = t0 + r;
+            s_dh[r][c] = (t < t_hi && n0 + c < N) ? dh[t * N + n0 + c] : 0.f;
+        }
+        for (int q = tid; q < 32 * 128; q += 256) {
+            const int r = q >> 7, c = q & 127;
+            const int64_t t = t0 + r;
+            s_x[r][c] = (t < t_hi && c0 + c < d) ? Elem<XT>::to_f(x[t * d + c0 + c]) : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int r = 0; r < 32; ++r) {
+            float a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = s_dh[r][4 * tn + i];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) b[j] = s_x[r][tc + 32 * j];
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+        }
+        if (blockIdx.z == 0 && tid < 32)
+            for (int r = 0; r < 32; ++r) dbacc += s_dh[r][tid];
+        __syncthreads();
+    }
+    float* pw = part_dw + (int64_t)chunk * N * d;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int n = n0 + 4 * tn + i;
+        if (n >= N) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c = c0 + tc + 32 * j;
+            if (c < d) pw[(int64_t)n * d + c] = acc[i][j];
+        }
+    }
+    if (blockIdx.z == 0 && tid < 32 && n0 + tid < N) part_db[(int64_t)chunk * N + n0 + tid] = dbacc;
+}
+
+// dw[n][c] = sum over chunks, in order, of the partials (fp64 accumulation)
+__global__ void __launch_bounds__(256)
+router_bwd_reduce_kernel(const float* __restrict__ part_dw, const float* __restrict__ part_db, int nchunk, int N,
+                         int d, float* __restrict__ dw, float* __restrict__ db) {
+    pdl_wait();
+    pdl_launch();
+    const int64_t nd = (int64_t)N * d;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nd + N; i += (int64_t)gridDim.x * blockDim.x) {
+        double acc = 0.0;
+        if (i < nd) {
+            for (int c = 0; c < nchunk; ++c) acc += (double)part_dw[(int64_t)c * nd + i];
+            if (dw) dw[i] = (float)acc;
+        } else {
+            const int64_t n = i - nd;
+            for (int c = 0; c < nchunk; ++c) acc += (double)part_db[(int64_t)c * N + n];
+            if (db) db[n] = (float)acc;
+        }
+    }
+}
+
+// dx[t][c] = sum_n dh[t][n] W_r[n][c]
+__global__ void __launch_bounds__(256)
+router_bwd_dx_kernel(const float* __restrict__ dh, const float* __restrict__ w_r, int64_t T, int N, int d,
+                     float* __restrict__ dx) {
+    pdl_wait();
+    pdl_launch();
+    __shared__ float s_dh[64][33];   // [token][expert]
+    __shared__ float s_w[32][132];   // [expert][column]
+    const int tid = threadIdx.x;
+    const int64_t t0 = (int64_t)blockIdx.x * 64;
+    const int c0 = blockIdx.y * 128;
+    const int tt = tid >> 5, tc = tid & 31;   // thread: tokens 8 tt .. 8 tt + 7, columns tc + 32 j
+    float acc[8][4];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+    for (int n0 = 0; n0 < N; n0 += 32) {
+        for (int q = tid; q < 64 * 32; q += 256) {
+            const int r = q >> 5, c = q & 31;
+            const int64_t t = t0 + r;
+            s_dh[r][c] = (t < T && n0 + c < N) ? dh[t * N + n0 + c] : 0.f;
+        }
+        for (int q = tid; q < 32 * 128; q += 256) {
+            const int r = q >> 7, c = q & 127;
+            s_w[r][c] = (n0 + r < N && c0 + c < d) ? w_r[(int64_t)(n0 + r) * d + c0 + c] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int n = 0; n < 32; ++n) {
+            float b[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) b[j] = s_w[n][tc + 32 * j];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float a = s_dh[8 * tt + i][n];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(a, b[j], acc[i][j]);
+            }
+        }
+        __syncthreads();
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int64_t t = t0 + 8 * tt + i;
+        if (t >= T) continue;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c = c0 + tc + 32 * j;
+            if (c < d) dx[t * d + c] = acc[i][j];
+        }
+    }
+}
+
+}  // namespace
+
+int router_bwd_chunks(int64_t T) { return (int)((T + kBwdChunk - 1) / kBwdChunk); }
+
+cudaError_t launch_router_backward(const RouterBwdArgs& a, cudaStream_t s) {
+    if (a.T <= 0) {   // no tokens: every gradient is zero
+        cudaError_t e = cudaSuccess;
+        if (a.dw) e = cudaMemsetAsync(a.dw, 0, sizeof(float) * a.N * a.d, s);
+        if (e == cudaSuccess && a.db) e = cudaMemsetAsync(a.db, 0, sizeof(float) * a.N, s);
+        return e;
+    }
+    cudaError_t err = launch_k(router_bwd_dh_kernel, dim3((unsigned)((a.T + 7) / 8)), dim3(256), 0, s, 1, a.probs,
+                               a.idx, a.gate, a.dgate, a.f, a.alpha, a.T, a.N, a.k, a.dh);
+    if (err != cudaSuccess) return err;
+    if (a.dw || a.db) {
+        const int nchunk = router_bwd_chunks(a.T);
+        const dim3 g((unsigned)nchunk, (unsigned)((a.N + 31) / 32), (unsigned)((a.d + 127) / 128));
+        err = a.dtype == MOE_BF16
+                  ? launch_k(router_bwd_dw_kernel<__nv_bfloat16>, g, dim3(256), 0, s, 1,
+                             static_cast<const float*>(a.dh), reinterpret_cast<const __nv_bfloat16*>(a.x), a.T, a.N,
+                             a.d, a.part_dw, a.part_db)
+                  : launch_k(router_bwd_dw_kernel<float>, g, dim3(256), 0, s, 1, static_cast<const float*>(a.dh),
+                             reinterpret_cast<const float*>(a.x), a.T, a.N, a.d, a.part_dw, a.part_db);
+        if (err != cudaSuccess) return err;
+        const int64_t n = (int64_t)a.N * a.d + a.N;
+        const unsigned rg = (unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+        err = launch_k(router_bwd_reduce_kernel, dim3(rg), dim3(256), 0, s, 1, static_cast<const float*>(a.part_dw),
+                       static_cast<const float*>(a.part_db), nchunk, a.N, a.d, a.dw, a.db);
+        if (err != cudaSuccess) return err;
+    }
+    if (a.dx) {
+        const dim3 g((unsigned)((a.T + 63) / 64), (unsigned)((a.d + 127) / 128));
+        err = launch_k(router_bwd_dx_kernel, g, dim3(256), 0, s, 1, static_cast<const float*>(a.dh), a.w_r, a.T, a.N,
+                       a.d, a.dx);
+    }
+    return err;
+}
+
+}  // namespace moe

@@ -42,6 +42,7 @@ _SIGS = {
     "moe_route": ([ctypes.POINTER(MoeConfig)] + [_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_route_z": ([ctypes.POINTER(MoeConfig)] + [_P] * 11 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_dispatch_ntlb": ([ctypes.POINTER(MoeConfig)] + [_P] * 13 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_router_backward": ([ctypes.POINTER(MoeConfig)] + [_P] * 12 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_dispatch": ([ctypes.POINTER(MoeConfig)] + [_P] * 12 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_expert_ffn": ([ctypes.POINTER(MoeConfig)] + [_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_combine": ([ctypes.POINTER(MoeConfig)] + [_P] * 8, ctypes.c_int32),
@@ -148,6 +149,11 @@ def moe_route(cfg, x, w_r, b_r, idx, gate, probs, f, P, aux, ws, stream=None):
 def moe_route_z(cfg, x, w_r, b_r, idx, gate, probs, f, P, aux, z_loss, ws, stream=None):
     return lib().moe_route_z(ctypes.byref(cfg), _p(x), _p(w_r), _p(b_r), _p(idx), _p(gate), _p(probs),
                              _p(f), _p(P), _p(aux), _p(z_loss), _p(ws), _nbytes(ws), _s(stream))
+
+
+def moe_router_backward(cfg, x, w_r, probs, idx, gate, f, dgate, dh, dw_r, db_r, dx, ws, stream=None):
+    return lib().moe_router_backward(ctypes.byref(cfg), _p(x), _p(w_r), _p(probs), _p(idx), _p(gate), _p(f),
+                                     _p(dgate), _p(dh), _p(dw_r), _p(db_r), _p(dx), _p(ws), _nbytes(ws), _s(stream))
 
 
 def moe_dispatch_ntlb(cfg, x, probs, expert, gate, pos, drop, counts, kept, offsets, row_token, row_gate, xe, ws,
