@@ -50,6 +50,8 @@ def _load():
         lib.oracle_dispatch_ordered.argtypes = [i64, i32, i32, i32, P, P, P, P, P, P, P]
         lib.oracle_dispatch_ntlb.argtypes = [i64, i32, i32, P, P, P, P, P, P, P, P, P]
         lib.oracle_router_backward.argtypes = [i64, i32, i32, i32, P, i32, P, P, P, P, P, P, f64, P, P, P, P]
+        lib.oracle_expert_backward.argtypes = [i64, i32, i32, i32, i32, i32, P, i32, P, P, P, P, P, P, i32,
+                                               P, P, P, P, P, P, P, P, P, P, P, P, P]
         lib.oracle_dispatch.restype = None
         lib.oracle_expert_ffn.argtypes = [i32, i32, i32, P, i32, sz, P, P, P, P, P, P, i32,
                                           sz, sz, sz, sz, P, P]
@@ -163,6 +165,39 @@ def router_backward(x, w_r, probs, idx, gate, f, dgate, alpha=1e-2):
     lib.oracle_router_backward(T, d, N, k, _ptr(x), xd, _ptr(w_r), _ptr(probs), _ptr(idx), _ptr(gate), _ptr(f),
                                _ptr(dgate), float(alpha), _ptr(dh), _ptr(dw), _ptr(db), _ptr(dx))
     return dict(dh=dh, dw=dw, db=db, dx=dx)
+
+
+def expert_backward(x, weights, idx, gate, drop, dout, act=RELU):
+    """Expert-path backward of L = sum_t <dout_t, out_t>: dL/dgate, the expert
+    part of dL/dx and the expert weight and bias gradients ("From Switch
+    Transformer to GLaM" FFN; CMU 10-423 Lecture 16 section 2.3 SwiGLU).
+    weights: dict(w1, b1, w3, b3, w2, b2) as for layer_tokens.  Returns a dict
+    of fp64 arrays (dw3/db3 None for ReLU)."""
+    lib = _load()
+    x, xd = _as_input(x)
+    T, d = x.shape
+    w1, wd = _as_input(weights["w1"])
+    N, d_ff, _ = w1.shape
+    w2, _ = _as_input(weights["w2"])
+    w3, _ = _as_input(weights.get("w3"))
+    b1, _ = _as_input(weights.get("b1"))
+    b3, _ = _as_input(weights.get("b3"))
+    b2, _ = _as_input(weights.get("b2"))
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    k = idx.shape[1]
+    gate = np.ascontiguousarray(gate, dtype=np.float32)
+    drop = np.ascontiguousarray(drop, dtype=np.uint8)
+    dout = np.ascontiguousarray(dout, dtype=np.float32)
+    sw = act == SWIGLU
+    out = dict(dgate=np.empty((T, k)), dx=np.empty((T, d)), dw1=np.empty((N, d_ff, d)), db1=np.empty((N, d_ff)),
+               dw3=np.empty((N, d_ff, d)) if sw else None, db3=np.empty((N, d_ff)) if sw else None,
+               dw2=np.empty((N, d, d_ff)), db2=np.empty((N, d)))
+    scratch = np.empty(6 * d_ff, np.float64)
+    lib.oracle_expert_backward(T, d, d_ff, N, k, act, _ptr(x), xd, _ptr(w1), _ptr(b1), _ptr(w3), _ptr(b3), _ptr(w2),
+                               _ptr(b2), wd, _ptr(idx), _ptr(gate), _ptr(drop), _ptr(dout), _ptr(scratch),
+                               _ptr(out["dgate"]), _ptr(out["dx"]), _ptr(out["dw1"]), _ptr(out["db1"]),
+                               _ptr(out["dw3"]), _ptr(out["db3"]), _ptr(out["dw2"]), _ptr(out["db2"]))
+    return out
 
 
 def aux_loss(idx, probs, alpha=1e-2):

@@ -264,6 +264,111 @@ void oracle_router_backward(int64_t T, int32_t d, int32_t N, int32_t k,
     }
 }
 
+/* ---- Expert backward -------------------------------------------------------
+ * Gradients of L = sum_t <dout_t, out_t> through the kept assignments of the
+ * layer: out_t = sum_{kept r} g_{t,r} E_{e}(x_t) ("From Switch Transformer to
+ * GLaM": FFN(x) = W2 s(W1 x); CMU 10-423 Lecture 16, section 2.3: the SwiGLU
+ * expert silu(W1 x) * (W3 x)).  Per kept (t, r) with expert e and gate g:
+ *   u = W1 x + b1, (v = W3 x + b3), a = relu(u) | silu(u) v, y = W2 a + b2;
+ *   dgate[t,r] = <dout_t, y>;  dy = g dout_t;
+ *   dW2[e] += dy a^T, db2[e] += dy, da = W2^T dy;
+ *   ReLU:   du = da (u > 0);
+ *   SwiGLU: du = da v silu'(u), dv = da silu(u), silu'(u) = s(u)(1 + u(1 - s(u)));
+ *   dW1[e] += du x^T, db1[e] += du, (dW3[e] += dv x^T, db3[e] += dv);
+ *   dx_t += W1^T du (+ W3^T dv).
+ * Dropped assignments contribute nothing (dgate 0).  Weights as in
+ * oracle_expert_ffn; outputs in double, zero-initialised here: dgate [T,k],
+ * dx [T,d], dw1/dw3 [N,d_ff,d], db1/db3 [N,d_ff], dw2 [N,d,d_ff], db2 [N,d]
+ * (dw3/db3 only for SwiGLU; they may be NULL otherwise). */
+void oracle_expert_backward(int64_t T, int32_t d, int32_t d_ff, int32_t N, int32_t k, int32_t act,
+                            const void* x, int32_t x_dtype,
+                            const void* w1, const void* b1, const void* w3, const void* b3,
+                            const void* w2, const void* b2, int32_t w_dtype,
+                            const int32_t* idx, const float* gate, const uint8_t* drop, const float* dout,
+                            double* scratch, double* dgate, double* dx, double* dw1, double* db1,
+                            double* dw3, double* db3, double* dw2, double* db2) {
+    double* u = scratch;
+    double* v = u + d_ff;
+    double* a = v + d_ff;
+    double* da = a + d_ff;
+    double* du = da + d_ff;
+    double* dv = du + d_ff;
+    const int swiglu = act == ORACLE_SWIGLU;
+    for (int64_t t = 0; t < T; ++t)
+        for (int32_t j = 0; j < d; ++j) dx[(size_t)t * d + j] = 0.0;
+    for (size_t i = 0; i < (size_t)N * d_ff * d; ++i) {
+        dw1[i] = 0.0;
+        dw2[i] = 0.0;
+        if (swiglu) dw3[i] = 0.0;
+    }
+    for (size_t i = 0; i < (size_t)N * d_ff; ++i) {
+        db1[i] = 0.0;
+        if (swiglu) db3[i] = 0.0;
+    }
+    for (size_t i = 0; i < (size_t)N * d; ++i) db2[i] = 0.0;
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t r = 0; r < k; ++r) {
+            dgate[t * k + r] = 0.0;
+            if (drop[t * k + r]) continue;
+            const int32_t e = idx[t * k + r];
+            const double g = (double)gate[t * k + r];
+            const size_t o1 = (size_t)e * d_ff * d, ob1 = (size_t)e * d_ff, o2 = (size_t)e * d * d_ff,
+                         ob2 = (size_t)e * d;
+            for (int32_t j = 0; j < d_ff; ++j) {
+                double su = 0.0, sv = 0.0;
+                for (int32_t i = 0; i < d; ++i) {
+                    const double xi = load_elem(x, x_dtype, (size_t)t * d + i);
+                    su += load_elem(w1, w_dtype, o1 + (size_t)j * d + i) * xi;
+                    if (swiglu) sv += load_elem(w3, w_dtype, o1 + (size_t)j * d + i) * xi;
+                }
+                if (b1) su += load_elem(b1, w_dtype, ob1 + j);
+                if (swiglu && b3) sv += load_elem(b3, w_dtype, ob1 + j);
+                u[j] = su;
+                v[j] = sv;
+                a[j] = swiglu ? su / (1.0 + exp(-su)) * sv : (su > 0.0 ? su : 0.0);
+            }
+            double dg = 0.0;
+            for (int32_t n = 0; n < d; ++n) {
+                double y = 0.0;
+                for (int32_t j = 0; j < d_ff; ++j) y += load_elem(w2, w_dtype, o2 + (size_t)n * d_ff + j) * a[j];
+                if (b2) y += load_elem(b2, w_dtype, ob2 + n);
+                dg += (double)dout[(size_t)t * d + n] * y;
+            }
+            dgate[t * k + r] = dg;
+            for (int32_t j = 0; j < d_ff; ++j) da[j] = 0.0;
+            for (int32_t n = 0; n < d; ++n) {
+                const double dy = g * (double)dout[(size_t)t * d + n];
+                db2[ob2 + n] += dy;
+                for (int32_t j = 0; j < d_ff; ++j) {
+                    dw2[o2 + (size_t)n * d_ff + j] += dy * a[j];
+                    da[j] += load_elem(w2, w_dtype, o2 + (size_t)n * d_ff + j) * dy;
+                }
+            }
+            for (int32_t j = 0; j < d_ff; ++j) {
+                if (swiglu) {
+                    const double sg = 1.0 / (1.0 + exp(-u[j]));
+                    du[j] = da[j] * v[j] * sg * (1.0 + u[j] * (1.0 - sg));
+                    dv[j] = da[j] * u[j] * sg;
+                } else {
+                    du[j] = u[j] > 0.0 ? da[j] : 0.0;
+                    dv[j] = 0.0;
+                }
+                db1[ob1 + j] += du[j];
+                if (swiglu) db3[ob1 + j] += dv[j];
+                for (int32_t i = 0; i < d; ++i) {
+                    const double xi = load_elem(x, x_dtype, (size_t)t * d + i);
+                    dw1[o1 + (size_t)j * d + i] += du[j] * xi;
+                    dx[(size_t)t * d + i] += load_elem(w1, w_dtype, o1 + (size_t)j * d + i) * du[j];
+                    if (swiglu) {
+                        dw3[o1 + (size_t)j * d + i] += dv[j] * xi;
+                        dx[(size_t)t * d + i] += load_elem(w3, w_dtype, o1 + (size_t)j * d + i) * dv[j];
+                    }
+                }
+            }
+        }
+    }
+}
+
 /* ---- Capacity --------------------------------------------------------------
  * C = floor(k * T * cf / N), exact.  cf is a binary double m * 2^e with m an
  * odd-or-zero 53-bit integer, so k T cf / N = k T m / (N 2^-e) is a rational

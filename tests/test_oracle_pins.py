@@ -501,6 +501,67 @@ def test_router_backward_uniform_f_has_no_aux_gradient():
     assert np.abs(got["dh"]).max() < 1e-7
 
 
+# ------------------------------------------------------ expert backward ----
+
+@pytest.mark.parametrize("act", ["relu", "swiglu"])
+def test_expert_backward_matches_finite_differences(act):
+    rng = np.random.default_rng(50 if act == "relu" else 51)
+    T, d, d_ff, N, k = 4, 3, 5, 3, 2
+    f32 = lambda a: np.asarray(a, np.float32)
+    W = dict(w1=f32(rng.standard_normal((N, d_ff, d))), b1=f32(rng.standard_normal((N, d_ff)) * 0.3),
+             w2=f32(rng.standard_normal((N, d, d_ff))), b2=f32(rng.standard_normal((N, d)) * 0.3))
+    if act == "swiglu":
+        W.update(w3=f32(rng.standard_normal((N, d_ff, d))), b3=f32(rng.standard_normal((N, d_ff)) * 0.3))
+    x = f32(rng.standard_normal((T, d)))
+    idx = np.stack([rng.permutation(N)[:k] for _ in range(T)]).astype(np.int32)
+    gate = f32(rng.random((T, k)))
+    drop = np.zeros((T, k), np.uint8)
+    drop[1, 1] = 1                                           # a dropped assignment contributes nothing
+    dout = f32(rng.standard_normal((T, d)))
+    P64 = {key: v.astype(np.float64) for key, v in W.items()}
+
+    def loss(x_, g_, P):
+        L = 0.0
+        for t in range(T):
+            for r in range(k):
+                if drop[t, r]:
+                    continue
+                e = idx[t, r]
+                u = P["w1"][e] @ x_[t] + P["b1"][e]
+                if act == "relu":
+                    a = np.maximum(u, 0.0)
+                else:
+                    v = P["w3"][e] @ x_[t] + P["b3"][e]
+                    a = u / (1.0 + np.exp(-u)) * v
+                y = P["w2"][e] @ a + P["b2"][e]
+                L += g_[t, r] * float(dout[t].astype(np.float64) @ y)
+        return L
+
+    if act == "relu":   # finite differences need every preactivation away from the kink
+        for t in range(T):
+            for r in range(k):
+                u = P64["w1"][idx[t, r]] @ x[t].astype(np.float64) + P64["b1"][idx[t, r]]
+                assert np.abs(u).min() > 1e-3
+
+    def num(fun, a, eps=1e-6):
+        out = np.zeros_like(a)
+        for i in np.ndindex(a.shape):
+            hi, lo = a.copy(), a.copy()
+            hi[i] += eps
+            lo[i] -= eps
+            out[i] = (fun(hi) - fun(lo)) / (2 * eps)
+        return out
+
+    got = oracle.expert_backward(x, W, idx, gate, drop, dout, act=oracle.SWIGLU if act == "swiglu" else oracle.RELU)
+    x64, g64 = x.astype(np.float64), gate.astype(np.float64)
+    tol = dict(rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(got["dgate"], num(lambda g_: loss(x64, g_, P64), g64) * (1 - drop), **tol)
+    np.testing.assert_allclose(got["dx"], num(lambda x_: loss(x_, g64, P64), x64), **tol)
+    for key in W:
+        ref = num(lambda a_: loss(x64, g64, {**P64, key: a_}), P64[key])
+        np.testing.assert_allclose(got["d" + key], ref, err_msg=key, **tol)
+
+
 def test_gshard_rank_major_example():
     # CMU 10-423 Lecture 16 section 6.1 (b): 3 devices of capacity 3; first choices are
     # placed before second choices, so a token's second choice can find its expert full.
