@@ -26,6 +26,14 @@
  *               choice is i (before capacity), P_i = mean router probability
  *               (GLaM page, section "Load balancing"; alpha = 1e-2)
  *
+ * Beyond the forward: other slot-claim rules (moe_config.priority: batch
+ * priority, No-Token-Left-Behind re-routing; moe_dispatch_ntlb), the router
+ * z-loss (moe_route_z), one routing group split over several GPUs with one
+ * small exchange (moe_expert_counts, moe_claim_base, moe_dispatch_shard,
+ * moe_combine_shard, moe_aux_shards), the router backward
+ * (moe_router_backward), and a dispatch that needs no workspace
+ * (moe_dispatch_noalloc).
+ *
  * Conventions shared by every entry point
  *   - All array pointers are DEVICE pointers unless stated; the caller owns
  *     every buffer.  The library never allocates or frees memory.
