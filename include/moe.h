@@ -30,8 +30,8 @@
  * priority, No-Token-Left-Behind re-routing; moe_dispatch_ntlb), the router
  * z-loss (moe_route_z), one routing group split over several GPUs with one
  * small exchange (moe_expert_counts, moe_claim_base, moe_dispatch_shard,
- * moe_combine_shard, moe_aux_shards), the router backward
- * (moe_router_backward), and a dispatch that needs no workspace
+ * moe_combine_shard, moe_aux_shards), the router backward (moe_gate_grad,
+ * moe_router_backward), and a dispatch that needs no workspace
  * (moe_dispatch_noalloc).
  *
  * Conventions shared by every entry point
@@ -156,6 +156,17 @@ int32_t moe_route_z(const moe_config* cfg, const void* x, const float* w_r, cons
                     int32_t* idx, float* gate, float* probs,
                     double* f, double* P, double* aux, double* z_loss,
                     void* ws, size_t ws_bytes, void* stream);
+
+/* Gradient of L with respect to the gates, from the upstream dL/dout and the
+ * un-gated expert outputs (out_t = sum_r gate_{t,r} E_{idx[t,r]}(x_t)):
+ * dgate[t, r] = <dout_t, ye[offsets[idx[t,r]] + pos[t,r]]> for a kept
+ * assignment, 0 for a dropped one; fp32 accumulation.  In: dout [T, d]
+ * (dtype), ye [R, d] (dtype; moe_expert_ffn's output), idx, pos, drop [T, k],
+ * offsets [N + 1].  Out: dgate [T, k] fp32 -- the input of
+ * moe_router_backward. */
+int32_t moe_gate_grad(const moe_config* cfg, const void* dout, const void* ye, const int32_t* idx,
+                      const int32_t* pos, const uint8_t* drop, const int32_t* offsets, float* dgate,
+                      void* stream);
 
 /* Router backward (fp32): gradients of L = sum_{t,r} dgate[t,r] gate[t,r] +
  * L_aux with respect to the router logits, W_r, b_r and the router input x.

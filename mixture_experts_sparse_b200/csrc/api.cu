@@ -387,6 +387,29 @@ int32_t moe_dispatch_ntlb(const moe_config* cfg, const void* x, const float* pro
                      ws, (cudaStream_t)stream);
 }
 
+int32_t moe_gate_grad(const moe_config* cfg, const void* dout, const void* ye, const int32_t* idx,
+                      const int32_t* pos, const uint8_t* drop, const int32_t* offsets, float* dgate, void* stream) {
+    int32_t st = validate(cfg);
+    if (st != MOE_OK) return st;
+    if (cfg->T > 0 && (!req(dout) || !req(idx) || !req(pos) || !req(drop) || !req(offsets) || !req(dgate)))
+        return MOE_ERR_INVALID_ARG;
+    if (!opt(ye)) return MOE_ERR_INVALID_ARG;
+    if (cfg->T > 0 && compact_rows(*cfg) > 0 && !ye) return MOE_ERR_INVALID_ARG;
+    GateGradArgs a{};
+    a.dtype = cfg->dtype;
+    a.T = cfg->T;
+    a.d = cfg->d_model;
+    a.k = cfg->top_k;
+    a.dout = dout;
+    a.ye = ye;
+    a.idx = idx;
+    a.pos = pos;
+    a.drop = drop;
+    a.offsets = offsets;
+    a.dgate = dgate;
+    return cuda_status(launch_gate_grad(a, (cudaStream_t)stream));
+}
+
 int32_t moe_router_backward(const moe_config* cfg, const void* x, const float* w_r, const float* probs,
                             const int32_t* idx, const float* gate, const double* f, const float* dgate, float* dh,
                             float* dw_r, float* db_r, float* dx, void* ws, size_t ws_bytes, void* stream) {

@@ -71,6 +71,33 @@ combine_kernel(const XT* __restrict__ ye, const int32_t* __restrict__ idx, const
     }
 }
 
+// dL/dgate[t, r] = <dout_t, ye[offsets[idx[t,r]] + pos[t,r]]> for a kept
+// assignment, 0 for a dropped one: the gate's gradient for the router backward
+// (out_t = sum_r gate_{t,r} E(x_t), "From Switch Transformer to GLaM").  One
+// warp per assignment, fp32 accumulation, a fixed shuffle tree.
+template <typename XT>
+__global__ void __launch_bounds__(256)
+gate_grad_kernel(const XT* __restrict__ dout, const XT* __restrict__ ye, const int32_t* __restrict__ idx,
+                 const int32_t* __restrict__ pos, const uint8_t* __restrict__ drop,
+                 const int32_t* __restrict__ offsets, int64_t T, int d, int k, float* __restrict__ dgate) {
+    pdl_wait();
+    pdl_launch();
+    const int lane = threadIdx.x & 31;
+    const int64_t a = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (a >= T * k) return;
+    const int64_t t = a / k;
+    float acc = 0.f;
+    if (!drop[a]) {
+        const int64_t row = (int64_t)offsets[idx[a]] + pos[a];
+        const XT* g = dout + t * (int64_t)d;
+        const XT* y = ye + row * (int64_t)d;
+        for (int c = lane; c < d; c += 32) acc = fmaf(Elem<XT>::to_f(g[c]), Elem<XT>::to_f(y[c]), acc);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) dgate[a] = acc;
+}
+
 }  // namespace
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
@@ -83,6 +110,17 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
     return launch_k(combine_kernel<float>, dim3(grid), dim3(256), 0, s, 1, reinterpret_cast<const float*>(a.ye), a.idx,
                     a.pos, a.drop, a.gate, a.offsets, a.claim_base, a.counts, a.C, a.N, a.T, a.d, a.k,
                     reinterpret_cast<float*>(a.out));
+}
+
+cudaError_t launch_gate_grad(const GateGradArgs& a, cudaStream_t s) {
+    if (a.T <= 0) return cudaSuccess;
+    const unsigned grid = (unsigned)((a.T * a.k + 7) / 8);
+    if (a.dtype == MOE_BF16)
+        return launch_k(gate_grad_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, 1,
+                        reinterpret_cast<const __nv_bfloat16*>(a.dout), reinterpret_cast<const __nv_bfloat16*>(a.ye),
+                        a.idx, a.pos, a.drop, a.offsets, a.T, a.d, a.k, a.dgate);
+    return launch_k(gate_grad_kernel<float>, dim3(grid), dim3(256), 0, s, 1, reinterpret_cast<const float*>(a.dout),
+                    reinterpret_cast<const float*>(a.ye), a.idx, a.pos, a.drop, a.offsets, a.T, a.d, a.k, a.dgate);
 }
 
 }  // namespace moe

@@ -305,4 +305,11 @@ struct CombineArgs {
 };
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s);
 
+struct GateGradArgs {
+    int dtype; int64_t T; int d; int k;
+    const void* dout; const void* ye; const int32_t* idx; const int32_t* pos; const uint8_t* drop;
+    const int32_t* offsets; float* dgate;
+};
+cudaError_t launch_gate_grad(const GateGradArgs& a, cudaStream_t s);
+
 }  // namespace moe

@@ -43,6 +43,7 @@ _SIGS = {
     "moe_route_z": ([ctypes.POINTER(MoeConfig)] + [_P] * 11 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_dispatch_ntlb": ([ctypes.POINTER(MoeConfig)] + [_P] * 13 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_router_backward": ([ctypes.POINTER(MoeConfig)] + [_P] * 12 + [ctypes.c_size_t, _P], ctypes.c_int32),
+    "moe_gate_grad": ([ctypes.POINTER(MoeConfig)] + [_P] * 8, ctypes.c_int32),
     "moe_dispatch": ([ctypes.POINTER(MoeConfig)] + [_P] * 12 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_expert_ffn": ([ctypes.POINTER(MoeConfig)] + [_P] * 10 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_combine": ([ctypes.POINTER(MoeConfig)] + [_P] * 8, ctypes.c_int32),
@@ -149,6 +150,11 @@ def moe_route(cfg, x, w_r, b_r, idx, gate, probs, f, P, aux, ws, stream=None):
 def moe_route_z(cfg, x, w_r, b_r, idx, gate, probs, f, P, aux, z_loss, ws, stream=None):
     return lib().moe_route_z(ctypes.byref(cfg), _p(x), _p(w_r), _p(b_r), _p(idx), _p(gate), _p(probs),
                              _p(f), _p(P), _p(aux), _p(z_loss), _p(ws), _nbytes(ws), _s(stream))
+
+
+def moe_gate_grad(cfg, dout, ye, idx, pos, drop, offsets, dgate, stream=None):
+    return lib().moe_gate_grad(ctypes.byref(cfg), _p(dout), _p(ye), _p(idx), _p(pos), _p(drop), _p(offsets),
+                               _p(dgate), _s(stream))
 
 
 def moe_router_backward(cfg, x, w_r, probs, idx, gate, f, dgate, dh, dw_r, db_r, dx, ws, stream=None):
