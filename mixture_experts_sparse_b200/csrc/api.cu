@@ -632,7 +632,7 @@ static int32_t forward_impl(const moe_config* cfg, const void* x, const float* w
         int sms = 0;
         if (device_sm_count(&sms) != cudaSuccess) return MOE_ERR_CUDA;
         aa = AuxArgs{at<int32_t>(ws, L.part_cnt), at<float>(ws, L.part_psum), router_tc_grid(cfg->T, sms),
-                     (int)cfg->n_experts, cfg->T, cfg->alpha, f, P, aux};
+                     (int)cfg->n_experts, cfg->T, cfg->alpha, f, P, aux, nullptr, nullptr};
     }
     // re-routing needs every token's router probabilities
     const bool ntlb = cfg->priority == MOE_ORDER_NTLB;
