@@ -5,7 +5,8 @@ import pytest
 
 import oracle
 from gpu_helpers import (BF16_MAX_ABS, REL_PROB, act_code, assert_close_out, assert_rel, compare_routing,
-                         oracle_layer, rel_rms, run_layer, sample_tokens, widen_out, workload_inputs)
+                         oracle_layer, oracle_layer_threads, rel_rms, run_layer, sample_tokens, tile_cover_tokens,
+                         widen_out, workload_inputs)
 from mixture_experts_sparse_b200 import inputs
 from mixture_experts_sparse_b200 import native as nat
 from mixture_experts_sparse_b200.configs import WORKLOADS
@@ -269,9 +270,15 @@ def test_workload_full_size(name):
     layer, _ = run_layer(L, w.T, w.d_model, w.d_ff, w.n_experts, w.top_k, C, w.dtype, w.act, w.alpha)
     r = oracle.route(L["x"], L["w_r"], L["b_r"], w.top_k)
     dd = oracle.dispatch(r["idx"], w.n_experts, C)
-    tokens = None if w.T <= 1024 else sample_tokens(w.T, dd["drop"].astype(bool),
-                                                    n_random=24 if w.d_ff < 8192 else 8)
-    res = oracle_layer(L, w.top_k, C, w.act, w.dtype, w.alpha, tokens=tokens)
+    # sampled tokens (first/last/random/dropped) plus, for every expert, rows that
+    # put a checked row in every m-tile of both expert GEMMs, including the last
+    # row of every ragged tile (128-row slices; 256 for the costly Mixtral experts,
+    # the CTA-pair tile height)
+    tokens = None
+    if w.T > 1024:
+        tokens = np.union1d(sample_tokens(w.T, dd["drop"].astype(bool), n_random=24 if w.d_ff < 8192 else 8),
+                            tile_cover_tokens(r["idx"], dd, 256 if w.d_ff >= 8192 else 128))
+    res = oracle_layer_threads(L, w.top_k, C, w.act, w.dtype, w.alpha, tokens=tokens)
     compare_routing(layer, res)
     got = widen_out(layer.out)
     toks = res["tokens"]
@@ -297,8 +304,8 @@ def test_mixtral_literal_capacity():
     layer, _ = run_layer(L, w.T, w.d_model, w.d_ff, w.n_experts, w.top_k, C, w.dtype, w.act, w.alpha)
     r = oracle.route(L["x"], L["w_r"], L["b_r"], w.top_k)
     dd = oracle.dispatch(r["idx"], w.n_experts, C)
-    tokens = sample_tokens(w.T, dd["drop"].astype(bool), n_random=4)
-    res = oracle_layer(L, w.top_k, C, w.act, w.dtype, w.alpha, tokens=tokens)
+    tokens = np.union1d(sample_tokens(w.T, dd["drop"].astype(bool), n_random=4), tile_cover_tokens(r["idx"], dd, 256))
+    res = oracle_layer_threads(L, w.top_k, C, w.act, w.dtype, w.alpha, tokens=tokens)
     compare_routing(layer, res)
     assert_close_out(widen_out(layer.out)[res["tokens"]], res["out_exact"], w.dtype)
 
