@@ -30,17 +30,22 @@
  * priority, No-Token-Left-Behind re-routing; moe_dispatch_ntlb), the router
  * z-loss (moe_route_z), one routing group split over several GPUs with one
  * small exchange (moe_expert_counts, moe_claim_base, moe_dispatch_shard,
- * moe_combine_shard, moe_aux_shards), the router backward (moe_gate_grad,
- * moe_router_backward), and a dispatch that needs no workspace
+ * moe_combine_shard, moe_aux_shards), the experts spread over several GPUs
+ * with all-to-all dispatch and combine (moe_ep_*), the router backward
+ * (moe_gate_grad, moe_router_backward), and a dispatch that needs no workspace
  * (moe_dispatch_noalloc).
  *
  * Conventions shared by every entry point
  *   - All array pointers are DEVICE pointers unless stated; the caller owns
- *     every buffer.  The library never allocates or frees memory.
+ *     every buffer.  The library never allocates or frees memory; the one
+ *     exception is the fixed scratch array of moe_dispatch_noalloc (see its
+ *     declaration), a static object of the library itself.
  *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
  *     NULL = the legacy default stream).  Only moe_read_device_status
  *     synchronises.  Calls are stateless apart from the caller's workspace, so
- *     distinct workspaces may be used from distinct threads.
+ *     distinct workspaces may be used from distinct threads -- except
+ *     moe_dispatch_noalloc, whose calls share one library-wide scratch array
+ *     per GPU and must not overlap (see its declaration).
  *   - Layouts (row-major): x, out [T, d_model]; w_r [N, d_model] fp32; b_r [N]
  *     fp32; w1, w3 [N, d_ff, d_model]; w2 [N, d_model, d_ff] ("output x input",
  *     so every product is a row dot product); b1, b3 [N, d_ff]; b2 [N, d_model];
@@ -213,7 +218,8 @@ int32_t moe_dispatch(const moe_config* cfg, const void* x, const int32_t* idx, c
  *      on expert[t]; C if dropped), drop [T], counts [N] (claims on each
  *      expert over all stages), kept [N] = min(counts, C), offsets [N + 1],
  *      row_token / row_gate / xe as moe_dispatch (row offsets[e] + pos).
- * Cost: N stages of four small kernels and two memsets. */
+ * Cost: one cooperative kernel runs the stages (one grid barrier each) and
+ * stops after the first stage that leaves no token unplaced, then the gather. */
 int32_t moe_dispatch_ntlb(const moe_config* cfg, const void* x, const float* probs,
                           int32_t* expert, float* gate, int32_t* pos, uint8_t* drop,
                           int32_t* counts, int32_t* kept, int32_t* offsets,
@@ -325,6 +331,80 @@ int32_t moe_forward_events(const moe_config* cfg, const void* x, const float* w_
                            double* f, double* P, double* aux,
                            void* ws, size_t ws_bytes, void* stream, void* const* events);
 
+/* ---- Expert parallelism: the experts spread over several GPUs -------------
+ * "From Switch Transformer to GLaM", section All-to-All: the experts of a layer
+ * live on different devices; a dispatch all-to-all moves every token from the
+ * device that holds it to the device of its expert, the experts run there, and
+ * a combine all-to-all brings the outputs back.  CMU 10-423 Lecture 16,
+ * section 6.2 and exercise 4: this moves 2 * T_g * k * d * 2 B * (G - 1) / G
+ * per GPU per layer (bf16), about 235 MB for Mixtral-size layers on 8 GPUs.
+ *
+ * G GPUs (n_ranks), N experts, E = N / G per GPU: expert e lives on GPU e / E
+ * and each GPU holds only the weights of its own E experts.  Every GPU keeps
+ * its own batch of T tokens as its own routing group (its capacity C, its
+ * aux loss), so its output equals the one-GPU layer forward of its batch.
+ * One forward, per GPU g:
+ *   1. moe_route, then moe_dispatch with xe = NULL (slot claim and row maps;
+ *      the gather is fused into step 4);
+ *   2. all-gather every GPU's kept [N] into kept_all [G][N] (NCCL, 512 B);
+ *   3. moe_ep_layout;
+ *   4. moe_ep_dispatch: x rows into their experts' GPUs (peer stores);
+ *   5. barrier across the GPUs (e.g. a one-element NCCL all-reduce on the
+ *      stream): every GPU's rows have landed;
+ *   6. moe_ep_expert_ffn on the received rows: the second GEMM's epilogue
+ *      stores every result row straight into its source GPU's buffer;
+ *   7. barrier again; 8. top-2 only: moe_combine on the GPU's own ye.
+ * Peer buffers are reached through device pointers the caller maps (CUDA IPC);
+ * "pointer tables" below are DEVICE arrays of G device pointers, entry s
+ * addressing GPU s's buffer (this GPU's own entry its own buffer).  Only plain
+ * loads from local memory and plain stores to peer memory cross GPUs. */
+
+/* Receive rows each GPU must provide (recv_x [R, d], recv_rank / recv_row /
+ * recv_gate [R]): R = G * min(k T, E C) (k counted at most E); -1 if invalid
+ * (N not a multiple of n_ranks, or the config is invalid). */
+int64_t moe_ep_recv_rows(const moe_config* cfg, int32_t n_ranks);
+
+/* Workspace bytes of moe_ep_expert_ffn (0 if invalid). */
+size_t moe_ep_workspace_bytes(const moe_config* cfg, int32_t n_ranks);
+
+/* Where rows land.  In: kept_all [G][N] int32 (every GPU's moe_dispatch kept,
+ * GPU order).  Out: dst_start [N] (GPU `rank` as a source: its rows of expert
+ * e go to rows dst_start[e] ... of GPU e / E's receive buffer) and
+ * recv_offsets [E + 1] (GPU `rank` as a receiver: rows of its local expert j
+ * are [recv_offsets[j], recv_offsets[j + 1]), source GPU 0's rows first, each
+ * source's in its own claim order). */
+int32_t moe_ep_layout(int32_t n_ranks, int32_t rank, int32_t n_experts, const int32_t* kept_all,
+                      int32_t* dst_start, int32_t* recv_offsets, void* stream);
+
+/* Dispatch all-to-all with the gather fused in: for every kept row r of this
+ * GPU (moe_dispatch's offsets / row_token / row_gate), x[row_token[r]] is
+ * stored into row dst_start[e] + r - offsets[e] of recv_x[e / E], with its
+ * return address: recv_rank = rank, recv_row = the token (top-1) or r (top-2),
+ * recv_gate = row_gate[r].  Top-1: also zeroes out [T, d] rows of dropped
+ * tokens (drop [T, 1]); out is ignored for top-2.  cfg is this GPU's layer
+ * (its T, the total N, k, C, dtype).  recv_x, recv_rank, recv_row, recv_gate:
+ * pointer tables [G]. */
+int32_t moe_ep_dispatch(const moe_config* cfg, int32_t n_ranks, int32_t rank, const void* x,
+                        const int32_t* offsets, const int32_t* row_token, const float* row_gate,
+                        const uint8_t* drop, const int32_t* dst_start, void* const* recv_x,
+                        int32_t* const* recv_rank, int32_t* const* recv_row, float* const* recv_gate,
+                        void* out, void* stream);
+
+/* The local experts on the received rows, results sent back.  In: recv_x,
+ * recv_offsets [E + 1], recv_rank, recv_row, recv_gate (this GPU's receive
+ * buffers, filled by every GPU's moe_ep_dispatch); w1, w3 [E, d_ff, d], w2
+ * [E, d, d_ff], b1, b3 [E, d_ff], b2 [E, d] (nullable): this GPU's experts only.
+ * out_ptrs: pointer table [G]; top-1: every GPU's out [T, d], row recv_row
+ * receives recv_gate * E(x); top-2: every GPU's ye [min(k T, N C), d], row
+ * recv_row receives E(x) (then moe_combine on that GPU).  bf16: stored from the
+ * second GEMM's epilogue; fp32: after the expert FFN, by a copy kernel.
+ * ws: moe_ep_workspace_bytes(cfg, n_ranks) bytes, moe_workspace_init'ed. */
+int32_t moe_ep_expert_ffn(const moe_config* cfg, int32_t n_ranks, const void* recv_x, const int32_t* recv_offsets,
+                          const void* w1, const void* b1, const void* w3, const void* b3, const void* w2,
+                          const void* b2, const int32_t* recv_rank, const int32_t* recv_row,
+                          const float* recv_gate, void* const* out_ptrs, void* ws, size_t ws_bytes,
+                          void* stream);
+
 /* Synchronise `stream`, then return the device status latched in the
  * workspace: MOE_OK, or MOE_ERR_TIMEOUT if a bounded device-side wait gave up
  * during an earlier call on this workspace.  The outputs of such a call are
@@ -350,7 +430,9 @@ int32_t moe_read_device_status(void* ws, void* stream);
  * -- different streams, or different host threads on the same device -- race
  * and must be serialised by the caller.  The first call on each device looks up
  * the array's device address (cudaGetSymbolAddress) with that device current;
- * make that first call before any stream capture starts.
+ * make that first call before any stream capture starts.  The address is kept
+ * for the life of the process: do not reset the device (cudaDeviceReset)
+ * between calls.
  * Arguments are those of moe_dispatch, without ws/ws_bytes, plus
  * status: device int32 (nullable) that receives this call's device-side status
  * (MOE_OK, or MOE_ERR_TIMEOUT if the scan's bounded wait gave up). */

@@ -61,7 +61,7 @@ struct Layout {
     size_t row_token, row_gate, xe, h, ye;
     size_t prio_hist, prio_cursor, prio_list, prio_perm, prio_idx, prio_pos, prio_range;   // batch priority only
     size_t ntlb_probs, ntlb_ch, ntlb_last, ntlb_first, ntlb_placed, ntlb_lp;               // re-routing only
-    size_t ntlb_claims, ntlb_st_counts, ntlb_st_kept, ntlb_st_offsets, ntlb_state;
+    size_t ntlb_agg, ntlb_unplaced, ntlb_bar;
     size_t bwd_part_dw, bwd_part_db;   // router backward partials
     size_t total;
     int64_t rows;   // min(k T, N C): compact rows the buffers hold
@@ -127,11 +127,9 @@ Layout layout_of(const moe_config& c) {
         L.ntlb_first = take(4 * T);
         L.ntlb_placed = take(4 * T);
         L.ntlb_lp = take(4 * T);
-        L.ntlb_claims = take(4 * (N + 1));
-        L.ntlb_st_counts = take(4 * (N + 1));
-        L.ntlb_st_kept = take(4 * (N + 1));
-        L.ntlb_st_offsets = take(4 * (N + 2));
-        L.ntlb_state = take(4 * nbs * (N + 1));
+        L.ntlb_agg = take(4 * 2 * (size_t)kNtlbMaxBlocks * N);
+        L.ntlb_unplaced = take(4 * 2 * (size_t)kNtlbMaxBlocks);
+        L.ntlb_bar = take(4);
     }
     L.total = off;
     return L;
@@ -155,6 +153,12 @@ int32_t validate(const moe_config* c) {
     if ((int64_t)c->d_model * c->d_ff >= ((int64_t)1 << 40)) return MOE_ERR_UNSUPPORTED;
     return MOE_OK;
 }
+
+}  // namespace
+
+int32_t validate_config(const moe_config* c) { return validate(c); }
+
+namespace {
 
 int32_t check_ws(const moe_config* c, void* ws, size_t ws_bytes) {
     if (!ws || !aligned(ws)) return MOE_ERR_WORKSPACE;
@@ -361,11 +365,9 @@ static int32_t ntlb_impl(const moe_config* cfg, const void* x, const float* prob
     a.first = at<int32_t>(ws, L.ntlb_first);
     a.placed = at<int32_t>(ws, L.ntlb_placed);
     a.lp = at<int32_t>(ws, L.ntlb_lp);
-    a.claims = at<int32_t>(ws, L.ntlb_claims);
-    a.st_counts = at<int32_t>(ws, L.ntlb_st_counts);
-    a.st_kept = at<int32_t>(ws, L.ntlb_st_kept);
-    a.st_offsets = at<int32_t>(ws, L.ntlb_st_offsets);
-    a.scan_state = at<uint32_t>(ws, L.ntlb_state);
+    a.grid_agg = at<int32_t>(ws, L.ntlb_agg);
+    a.grid_unplaced = at<int32_t>(ws, L.ntlb_unplaced);
+    a.grid_bar = at<uint32_t>(ws, L.ntlb_bar);
     a.hdr = at<WsHeader>(ws, L.hdr);
     if (aux) a.aux = *aux;
     return cuda_status(launch_dispatch_ntlb(a, s));
@@ -689,6 +691,143 @@ int32_t moe_forward_events(const moe_config* cfg, const void* x, const float* w_
                            void* ws, size_t ws_bytes, void* stream, void* const* events) {
     return forward_impl(cfg, x, w_r, b_r, w1, b1, w3, b3, w2, b2, out, idx, gate, pos, drop, counts, kept, offsets,
                         f, P, aux, ws, ws_bytes, (cudaStream_t)stream, events);
+}
+
+// ---- expert parallelism --------------------------------------------------
+
+// The receiving GPU's view of a layer split over n_ranks GPUs: its E = N / G
+// experts, and up to min(k T, E C) rows from each of the G sources.
+static bool ep_recv_config(const moe_config* cfg, int32_t n_ranks, moe_config* out) {
+    if (!cfg || n_ranks < 1 || cfg->n_experts % n_ranks != 0) return false;
+    moe_config r = *cfg;
+    const int64_t T = (int64_t)cfg->T * n_ranks, C = (int64_t)cfg->capacity * n_ranks;
+    if (T >= (int64_t)1 << 28 || C > 2147483647) return false;
+    r.T = (int32_t)T;
+    r.n_experts = cfg->n_experts / n_ranks;
+    r.capacity = (int32_t)C;
+    r.top_k = cfg->top_k > r.n_experts ? r.n_experts : cfg->top_k;   // only sizes depend on it here
+    *out = r;
+    return true;
+}
+
+static int32_t ep_check(const moe_config* cfg, int32_t n_ranks, int32_t rank) {
+    int32_t st = validate(cfg);
+    if (st != MOE_OK) return st;
+    if (n_ranks < 1 || rank < 0 || rank >= n_ranks) return MOE_ERR_INVALID_ARG;
+    if (cfg->n_experts % n_ranks != 0) return MOE_ERR_UNSUPPORTED;   // whole experts per GPU
+    if (cfg->priority != MOE_ORDER_TOKEN) return MOE_ERR_UNSUPPORTED;
+    moe_config r;
+    if (!ep_recv_config(cfg, n_ranks, &r) || validate(&r) != MOE_OK) return MOE_ERR_UNSUPPORTED;
+    return MOE_OK;
+}
+
+int64_t moe_ep_recv_rows(const moe_config* cfg, int32_t n_ranks) {
+    moe_config r;
+    if (ep_check(cfg, n_ranks, 0) != MOE_OK || !ep_recv_config(cfg, n_ranks, &r)) return -1;
+    return compact_rows(r);
+}
+
+size_t moe_ep_workspace_bytes(const moe_config* cfg, int32_t n_ranks) {
+    moe_config r;
+    if (ep_check(cfg, n_ranks, 0) != MOE_OK || !ep_recv_config(cfg, n_ranks, &r)) return 0;
+    return layout_of(r).total;
+}
+
+int32_t moe_ep_layout(int32_t n_ranks, int32_t rank, int32_t n_experts, const int32_t* kept_all, int32_t* dst_start,
+                      int32_t* recv_offsets, void* stream) {
+    if (n_ranks < 1 || rank < 0 || rank >= n_ranks || n_experts < 1) return MOE_ERR_INVALID_ARG;
+    if (n_experts > 128 || n_experts % n_ranks != 0) return MOE_ERR_UNSUPPORTED;
+    if (!req(kept_all) || !req(dst_start) || !req(recv_offsets)) return MOE_ERR_INVALID_ARG;
+    return cuda_status(launch_ep_layout(n_ranks, rank, n_experts, kept_all, dst_start, recv_offsets,
+                                        (cudaStream_t)stream));
+}
+
+int32_t moe_ep_dispatch(const moe_config* cfg, int32_t n_ranks, int32_t rank, const void* x, const int32_t* offsets,
+                        const int32_t* row_token, const float* row_gate, const uint8_t* drop,
+                        const int32_t* dst_start, void* const* recv_x, int32_t* const* recv_rank,
+                        int32_t* const* recv_row, float* const* recv_gate, void* out, void* stream) {
+    int32_t st = ep_check(cfg, n_ranks, rank);
+    if (st != MOE_OK) return st;
+    if (!req(offsets) || !req(dst_start) || !req(recv_x) || !req(recv_rank) || !req(recv_row) || !req(recv_gate) ||
+        !opt(out))
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->T > 0 && (!req(x) || !req(row_token) || !req(row_gate) || !req(drop))) return MOE_ERR_INVALID_ARG;
+    if (cfg->T > 0 && cfg->top_k == 1 && !out) return MOE_ERR_INVALID_ARG;   // dropped tokens' rows are zeroed
+    EpDispatchArgs a{};
+    a.dtype = cfg->dtype;
+    a.T = cfg->T;
+    a.d = cfg->d_model;
+    a.N = cfg->n_experts;
+    a.k = cfg->top_k;
+    a.G = n_ranks;
+    a.rank = rank;
+    a.R_cap = compact_rows(*cfg);
+    a.x = x;
+    a.offsets = offsets;
+    a.row_token = row_token;
+    a.row_gate = row_gate;
+    a.dst_start = dst_start;
+    a.drop = drop;
+    a.out = cfg->top_k == 1 ? out : nullptr;
+    a.recv_x = recv_x;
+    a.recv_rank = recv_rank;
+    a.recv_row = recv_row;
+    a.recv_gate = recv_gate;
+    return cuda_status(launch_ep_dispatch(a, (cudaStream_t)stream));
+}
+
+int32_t moe_ep_expert_ffn(const moe_config* cfg, int32_t n_ranks, const void* recv_x, const int32_t* recv_offsets,
+                          const void* w1, const void* b1, const void* w3, const void* b3, const void* w2,
+                          const void* b2, const int32_t* recv_rank, const int32_t* recv_row, const float* recv_gate,
+                          void* const* out_ptrs, void* ws, size_t ws_bytes, void* stream) {
+    int32_t st = ep_check(cfg, n_ranks, 0);
+    if (st != MOE_OK) return st;
+    moe_config r;
+    ep_recv_config(cfg, n_ranks, &r);
+    if (!req(recv_x) || !req(recv_offsets) || !req(w1) || !req(w2) || !opt(b1) || !opt(b2) || !opt(b3) ||
+        !req(recv_rank) || !req(recv_row) || !req(out_ptrs) || !opt(recv_gate))
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->act == MOE_SWIGLU ? !req(w3) : !opt(w3)) return MOE_ERR_INVALID_ARG;
+    if (cfg->top_k == 1 && !recv_gate) return MOE_ERR_INVALID_ARG;   // top-1 results leave gated
+    if ((st = check_ws(&r, ws, ws_bytes)) != MOE_OK) return st;
+    const Layout L = layout_of(r);
+    if (L.rows <= 0) return MOE_OK;
+    cudaStream_t s = (cudaStream_t)stream;
+    // top-1: gate * E(x) into the source's out row of the token; top-2: E(x)
+    // into the source's compact row (the source's combine applies the gates)
+    const float* g = cfg->top_k == 1 ? recv_gate : nullptr;
+    if (cfg->dtype == MOE_BF16) {
+        FfnArgs a{};
+        a.dtype = r.dtype;
+        a.act = r.act;
+        a.N = r.n_experts;
+        a.d = r.d_model;
+        a.d_ff = r.d_ff;
+        a.C = (int)(L.rows < r.capacity ? L.rows : r.capacity);
+        a.R_cap = L.rows;
+        a.xe = recv_x;
+        a.offsets = recv_offsets;
+        a.w1 = w1;
+        a.b1 = b1;
+        a.w3 = w3;
+        a.b3 = b3;
+        a.w2 = w2;
+        a.b2 = b2;
+        a.h = at<void>(ws, L.h);
+        a.ye = at<void>(ws, L.ye);
+        a.row_token = recv_row;
+        a.row_gate = g;
+        a.scatter_ptrs = out_ptrs;
+        a.row_rank = recv_rank;
+        a.hdr = at<WsHeader>(ws, L.hdr);
+        return cuda_status(launch_expert_ffn(a, s));
+    }
+    // fp32: the FP32-pipe expert FFN into the workspace, then the rows go back
+    st = ffn_impl(&r, recv_x, recv_offsets, w1, b1, w3, b3, w2, b2, at<void>(ws, L.ye), nullptr, nullptr, nullptr,
+                  ws, s);
+    if (st != MOE_OK) return st;
+    return cuda_status(launch_ep_return(r.dtype, at<void>(ws, L.ye), recv_offsets, r.n_experts, r.d_model, L.rows,
+                                        recv_rank, recv_row, g, out_ptrs, s));
 }
 
 int32_t moe_read_device_status(void* ws, void* stream) {

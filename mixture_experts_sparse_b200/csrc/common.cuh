@@ -9,6 +9,14 @@
 
 namespace moe {
 
+// Tokens per block of the dispatch scan (dispatch.cu); the look-back state
+// holds one word per (scan block, rank, expert).
+constexpr int kScanTokens = 1024;
+
+// Argument checks every entry point that takes a moe_config runs first
+// (MOE_OK or the status to return); defined in api.cu.
+int32_t validate_config(const moe_config* c);
+
 // ---- workspace header (first 256 bytes of every workspace) ----------------
 struct WsHeader {
     int32_t status;        // latched moe_status of device-side failures
@@ -263,12 +271,13 @@ struct NtlbArgs {
     int32_t* counts; int32_t* kept; int32_t* offsets;            // [N], [N], [N + 1]
     int32_t* row_token; float* row_gate; void* xe; void* zero_out;
     int32_t* ch; int32_t* last; int32_t* first; int32_t* placed; int32_t* lp;   // [T] each
-    int32_t* claims;                                             // [N + 1]
-    int32_t* st_counts; int32_t* st_kept; int32_t* st_offsets;   // [N + 1], [N + 1], [N + 2]
-    uint32_t* scan_state;                                        // [scan_blocks(T) * (N + 1)]
+    int32_t* grid_agg;        // [2][kNtlbMaxBlocks][N] per-block stage claims
+    int32_t* grid_unplaced;   // [2][kNtlbMaxBlocks]
+    uint32_t* grid_bar;       // grid barrier counter
     WsHeader* hdr;
     AuxArgs aux;
 };
+constexpr int kNtlbMaxBlocks = 256;   // blocks of the cooperative re-routing kernel
 cudaError_t launch_dispatch_ntlb(const NtlbArgs& a, cudaStream_t s);
 
 int scan_blocks(int64_t T);
@@ -289,10 +298,27 @@ struct FfnArgs {
     void* ye;                     // [R, d] (used when scatter_out == nullptr)
     void* scatter_out;            // top-1 fused: out[row_token[r]] = row_gate[r] * E(x)
     const int32_t* row_token; const float* row_gate;
+    // expert parallelism: row r's result goes to GPU row_rank[r]: scatter_ptrs
+    // [row_rank[r]] + row_token[r] * d, times row_gate[r] (nullable: 1)
+    void* const* scatter_ptrs; const int32_t* row_rank;
     WsHeader* hdr;
     void* mid_event;              // optional cudaEvent_t recorded between the two stages
 };
 cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t s);
+
+// Expert parallelism (ep.cu)
+struct EpDispatchArgs {
+    int dtype; int64_t T; int d; int N; int k; int G; int rank; int64_t R_cap;
+    const void* x; const int32_t* offsets; const int32_t* row_token; const float* row_gate;
+    const int32_t* dst_start; const uint8_t* drop; void* out;
+    void* const* recv_x; int32_t* const* recv_rank; int32_t* const* recv_row; float* const* recv_gate;
+};
+cudaError_t launch_ep_layout(int G, int rank, int N, const int32_t* kept_all, int32_t* dst_start,
+                             int32_t* recv_offsets, cudaStream_t s);
+cudaError_t launch_ep_dispatch(const EpDispatchArgs& a, cudaStream_t s);
+cudaError_t launch_ep_return(int dtype, const void* ye, const int32_t* recv_offsets, int E, int d, int64_t R_cap,
+                             const int32_t* recv_rank, const int32_t* recv_row, const float* recv_gate,
+                             void* const* out_ptrs, cudaStream_t s);
 
 struct CombineArgs {
     int dtype; int64_t T; int d; int k;

@@ -26,8 +26,7 @@ namespace moe {
 namespace {
 
 constexpr int kScanThreads = 256;
-constexpr int kScanTokens = 1024;          // tokens per scan block (8 warps x 128)
-constexpr int kWarpTokens = kScanTokens / 8;
+constexpr int kWarpTokens = kScanTokens / 8;   // kScanTokens (common.cuh) = 8 warps x 128 tokens
 constexpr uint32_t kFlagAgg = 1u << 30;    // block aggregate published
 constexpr uint32_t kFlagPre = 2u << 30;    // inclusive prefix published
 constexpr uint32_t kValMask = (1u << 30) - 1u;
@@ -372,100 +371,226 @@ prio_rank_kernel(const float* __restrict__ gate, const int32_t* __restrict__ idx
 // token still without a slot claims, in token order, on its (s+1)-th expert
 // (router probabilities descending, ties to the lower index), numbered after
 // every claim already made on that expert; kept iff that number is below C.
-// Per stage: ntlb_choose_kernel, the look-back scan over N + 1 experts (expert
-// N is the sink of tokens already placed), ntlb_place_kernel and
-// ntlb_claims_kernel; then ntlb_final_kernel, ntlb_offsets_kernel and the
-// gather.
+//
+// One cooperative launch runs every stage (its blocks are co-resident, so they
+// may wait on one another).  Block b owns the contiguous tokens [b TB, (b+1) TB).
+// Per stage: (1) each block picks the next expert of its unplaced tokens and
+// ranks them per expert in token order (warp match + running counts over
+// 1024-token pieces), and publishes its per-expert claim counts; (2) one grid
+// barrier; (3) every block sums the counts of the blocks before it (exclusive
+// prefix) and of all blocks (the stage's claims), places its tokens whose claim
+// number claims_before[e] + prefix[e] + rank is below C, and publishes how many
+// of its tokens are still unplaced.  The next stage's barrier makes those counts
+// visible: when none is left, every block stops (the remaining stages would
+// claim nothing).  Dropped tokens then report their first choice with pos = C,
+// and block 0 writes counts / kept / offsets.  Scratch is double-buffered by
+// stage parity, so a block never overwrites counts a slower block still reads.
 
 // expert a (probability pa) comes before expert b in a token's order
 __device__ __forceinline__ bool ntlb_before(float pa, int a, float pb, int b) {
     return pa > pb || (pa == pb && a < b);
 }
 
-__global__ void __launch_bounds__(256)
-ntlb_choose_kernel(const float* __restrict__ probs, int64_t T, int N, int s, int32_t* __restrict__ placed,
-                   int32_t* __restrict__ last, int32_t* __restrict__ first, int32_t* __restrict__ ch) {
-    pdl_wait();
-    pdl_launch();
-    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < T; t += (int64_t)gridDim.x * blockDim.x) {
-        if (s == 0) placed[t] = 0;
-        else if (placed[t]) {
-            ch[t] = N;   // the sink: claims nothing
-            continue;
+// The first expert after `le` (probability lpv) in the token's order; le < 0:
+// the token's first choice.
+__device__ __forceinline__ int ntlb_next(const float* __restrict__ p, int N, int le, float lpv) {
+    int best = -1;
+    float bp = 0.f;
+    for (int e = 0; e < N; ++e) {
+        const float pe = __ldg(p + e);
+        if (le >= 0 && !ntlb_before(lpv, le, pe, e)) continue;
+        if (best < 0 || ntlb_before(pe, e, bp, best)) {
+            best = e;
+            bp = pe;
         }
-        const float* p = probs + t * N;
-        const int le = s > 0 ? last[t] : -1;
-        const float lpv = s > 0 ? p[le] : 0.f;
-        int best = -1;
-        float bp = 0.f;
-        for (int e = 0; e < N; ++e) {   // the first expert after the previous choice
-            const float pe = p[e];
-            if (s > 0 && !ntlb_before(lpv, le, pe, e)) continue;
-            if (best < 0 || ntlb_before(pe, e, bp, best)) {
-                best = e;
-                bp = pe;
+    }
+    return best;
+}
+
+struct NtlbGrid {
+    const float* probs; int64_t T; int N; int C; int64_t TB;
+    int32_t* expert; float* gate; int32_t* pos;
+    int32_t* counts; int32_t* kept; int32_t* offsets;
+    int32_t* ch; int32_t* last; int32_t* first; int32_t* placed; int32_t* lp;
+    int32_t* agg;        // [2][gridDim.x][N] per-block claims of the stage
+    int32_t* unplaced;   // [2][gridDim.x]
+    uint32_t* bar;       // grid barrier arrivals (0 at launch)
+    int32_t* status;
+    long long limit_ns;
+};
+
+// Grid-wide barrier of a cooperative launch (bounded: on expiry the status is
+// latched and false returned, and the caller stops).
+__device__ bool ntlb_grid_sync(uint32_t* bar, uint32_t target, long long limit_ns, int32_t* status, int* s_ok) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        atomicAdd(bar, 1u);
+        const long long t0 = global_ns();
+        int ok = 1;
+        for (unsigned i = 0; ld_relaxed(bar) < target; ++i) {
+            if ((i & 63u) == 63u && global_ns() - t0 > limit_ns) {
+                latch_status(status, MOE_ERR_TIMEOUT);
+                ok = 0;
+                break;
             }
         }
-        ch[t] = best;   // s < N: an untried expert is always left
-        last[t] = best;
-        if (s == 0) first[t] = best;
+        __threadfence();
+        *s_ok = ok;
     }
+    __syncthreads();
+    return *s_ok != 0;
 }
 
-__global__ void __launch_bounds__(256)
-ntlb_place_kernel(const float* __restrict__ probs, int64_t T, int N, int C, const int32_t* __restrict__ ch,
-                  const int32_t* __restrict__ lp, const int32_t* __restrict__ claims, int32_t* __restrict__ placed,
-                  int32_t* __restrict__ expert, int32_t* __restrict__ pos, float* __restrict__ gate) {
+__global__ void __launch_bounds__(kScanThreads) ntlb_grid_kernel(const NtlbGrid a) {
     pdl_wait();
     pdl_launch();
-    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < T; t += (int64_t)gridDim.x * blockDim.x) {
-        const int e = ch[t];
-        if (e >= N) continue;
-        const int64_t c = (int64_t)claims[e] + lp[t];
-        if (c < (int64_t)C) {
-            placed[t] = 1;
-            expert[t] = e;
-            pos[t] = (int32_t)c;
-            gate[t] = probs[t * N + e];
+    __shared__ int32_t s_claims[128];      // claims on each expert before this stage
+    __shared__ int32_t s_cnt[128];         // this block's claims in this stage, so far
+    __shared__ int32_t s_base[128];        // s_cnt before the current 1024-token piece
+    __shared__ int32_t s_wcnt[8][128];     // per warp, then per-warp exclusive offsets
+    __shared__ int32_t s_excl[128];        // claims of earlier blocks in this stage
+    __shared__ int32_t s_red[kScanThreads / 32];
+    __shared__ int s_ok;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int N = a.N, G = (int)gridDim.x, b = (int)blockIdx.x;
+    const int64_t t_lo = (int64_t)b * a.TB;
+    const int64_t t_hi = min(a.T, t_lo + a.TB);
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int e = tid; e < N; e += kScanThreads) {
+        s_claims[e] = 0;
+        s_cnt[e] = 0;
+    }
+    for (int q = tid; q < 8 * 128; q += kScanThreads) (&s_wcnt[0][0])[q] = 0;
+    __syncthreads();
+    uint32_t nbar = 0;
+    bool ok = true;
+    for (int s = 0; s < N && ok; ++s) {
+        const int par = s & 1;
+        // (1) next choice and the rank among this block's claims on it, token order
+        for (int64_t base = t_lo; base < t_hi; base += kScanTokens) {
+            int rk[kWarpTokens / 32], ex[kWarpTokens / 32];
+#pragma unroll
+            for (int it = 0; it < kWarpTokens / 32; ++it) {
+                const int64_t t = base + warp * kWarpTokens + it * 32 + lane;
+                int e = -1;
+                if (t < t_hi) {
+                    const float* p = a.probs + t * N;
+                    if (s == 0) {
+                        e = ntlb_next(p, N, -1, 0.f);
+                        a.placed[t] = 0;
+                        a.first[t] = e;
+                        a.last[t] = e;
+                    } else if (!a.placed[t]) {
+                        const int le = a.last[t];
+                        e = ntlb_next(p, N, le, __ldg(p + le));   // s < N: an untried expert is left
+                        a.last[t] = e;
+                    }
+                    a.ch[t] = e;
+                }
+                const unsigned peers = __match_any_sync(0xffffffffu, e);
+                ex[it] = e;
+                rk[it] = e >= 0 ? s_wcnt[warp][e] + __popc(peers & lt_mask) : 0;
+                __syncwarp();
+                if (e >= 0 && lane == __ffs(peers) - 1) s_wcnt[warp][e] += __popc(peers);
+                __syncwarp();
+            }
+            __syncthreads();
+            for (int e = tid; e < N; e += kScanThreads) {   // warp offsets inside the piece
+                int run = s_cnt[e];
+                s_base[e] = run;
+                for (int w = 0; w < 8; ++w) {
+                    const int v = s_wcnt[w][e];
+                    s_wcnt[w][e] = run;
+                    run += v;
+                }
+                s_cnt[e] = run;
+            }
+            __syncthreads();
+#pragma unroll
+            for (int it = 0; it < kWarpTokens / 32; ++it) {
+                const int64_t t = base + warp * kWarpTokens + it * 32 + lane;
+                if (t < t_hi && ex[it] >= 0) a.lp[t] = s_wcnt[warp][ex[it]] + rk[it];
+            }
+            __syncthreads();
+            for (int q = tid; q < 8 * N; q += kScanThreads) s_wcnt[q / N][q % N] = 0;
+            __syncthreads();
         }
+        for (int e = tid; e < N; e += kScanThreads) {
+            a.agg[((int64_t)par * G + b) * N + e] = s_cnt[e];
+            s_cnt[e] = 0;
+        }
+        // (2) every block's counts of this stage (and unplaced counts of the last) are visible
+        nbar += (uint32_t)G;
+        if (!ntlb_grid_sync(a.bar, nbar, a.limit_ns, a.status, &s_ok)) {
+            ok = false;
+            break;
+        }
+        if (s > 0) {   // nothing was left unplaced after the previous stage: done
+            int left = 0;
+            for (int q = tid; q < G; q += kScanThreads) left += __ldcg(a.unplaced + (int64_t)(par ^ 1) * G + q);
+            left = __syncthreads_or(left != 0);
+            if (!left) break;
+        }
+        // (3) claim numbers and placement
+        for (int e = tid; e < N; e += kScanThreads) {
+            int ex_ = 0, tot = 0;
+            const int32_t* col = a.agg + (int64_t)par * G * N + e;
+            for (int q = 0; q < G; ++q) {
+                const int v = __ldcg(col + (int64_t)q * N);
+                ex_ += q < b ? v : 0;
+                tot += v;
+            }
+            s_excl[e] = ex_;
+            s_base[e] = tot;
+        }
+        __syncthreads();
+        int left = 0;
+        for (int64_t t = t_lo + tid; t < t_hi; t += kScanThreads) {
+            if (a.placed[t]) continue;
+            const int e = a.ch[t];
+            const int64_t c = (int64_t)s_claims[e] + s_excl[e] + a.lp[t];
+            if (c < (int64_t)a.C) {
+                a.placed[t] = 1;
+                a.expert[t] = e;
+                a.pos[t] = (int32_t)c;
+                a.gate[t] = a.probs[t * N + e];
+            } else {
+                ++left;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) left += __shfl_xor_sync(0xffffffffu, left, o);
+        if (lane == 0) s_red[warp] = left;
+        __syncthreads();
+        if (tid == 0) {
+            int sum = 0;
+            for (int w = 0; w < kScanThreads / 32; ++w) sum += s_red[w];
+            a.unplaced[(int64_t)par * G + b] = sum;
+        }
+        for (int e = tid; e < N; e += kScanThreads) s_claims[e] += s_base[e];
+        __syncthreads();
     }
-}
-
-__global__ void ntlb_claims_kernel(int N, const int32_t* __restrict__ st_counts, int32_t* __restrict__ claims) {
-    pdl_wait();
-    pdl_launch();
-    for (int e = threadIdx.x; e < N; e += blockDim.x) claims[e] += st_counts[e];
-}
-
-__global__ void __launch_bounds__(256)
-ntlb_final_kernel(const float* __restrict__ probs, int64_t T, int N, int C, const int32_t* __restrict__ placed,
-                  const int32_t* __restrict__ first, int32_t* __restrict__ expert, float* __restrict__ gate,
-                  int32_t* __restrict__ pos) {
-    pdl_wait();
-    pdl_launch();
-    for (int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; t < T; t += (int64_t)gridDim.x * blockDim.x) {
-        if (placed[t]) continue;
-        const int e = first[t];   // dropped: its first choice, claim number C
-        expert[t] = e;
-        pos[t] = C;
-        gate[t] = probs[t * N + e];
+    if (!ok) return;
+    // dropped: first choice, claim number C
+    for (int64_t t = t_lo + tid; t < t_hi; t += kScanThreads) {
+        if (a.placed[t]) continue;
+        const int e = a.first[t];
+        a.expert[t] = e;
+        a.pos[t] = a.C;
+        a.gate[t] = a.probs[t * N + e];
     }
-}
-
-__global__ void ntlb_offsets_kernel(int N, int C, const int32_t* __restrict__ claims, int32_t* __restrict__ counts,
-                                    int32_t* __restrict__ kept, int32_t* __restrict__ offsets) {
-    pdl_wait();
-    pdl_launch();
-    if (threadIdx.x != 0) return;
-    int32_t acc = 0;
-    for (int e = 0; e < N; ++e) {
-        const int32_t c = claims[e];
-        counts[e] = c;
-        kept[e] = c < C ? c : C;
-        offsets[e] = acc;
-        acc += kept[e];
+    if (b == 0 && tid == 0) {   // every block holds the same claim totals
+        int32_t acc = 0;
+        for (int e = 0; e < N; ++e) {
+            const int32_t c = s_claims[e];
+            a.counts[e] = c;
+            a.kept[e] = c < a.C ? c : a.C;
+            a.offsets[e] = acc;
+            acc += a.kept[e];
+        }
+        a.offsets[N] = acc;
     }
-    offsets[N] = acc;
 }
 
 // Claims per (rank, expert) of this shard: counts[r][e] (int atomics, so the
@@ -598,44 +723,58 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
                     pos_in);
 }
 
+int ntlb_grid_blocks(int64_t T, int sms) {
+    const int64_t want = (T + 255) / 256;
+    int64_t g = want < sms ? want : sms;
+    if (g > kNtlbMaxBlocks) g = kNtlbMaxBlocks;
+    return (int)(g < 1 ? 1 : g);
+}
+
 cudaError_t launch_dispatch_ntlb(const NtlbArgs& a, cudaStream_t s) {
-    const int nblk = scan_blocks(a.T);
-    if (nblk == 0) return cudaSuccess;
-    const int N = a.N;
-    const unsigned g = (unsigned)((a.T + 255) / 256 < 4096 ? (a.T + 255) / 256 : 4096);
-    cudaError_t err = cudaMemsetAsync(a.claims, 0, sizeof(int32_t) * (N + 1), s);
+    if (a.T <= 0) return cudaSuccess;
+    int sms = 0;
+    cudaError_t err = device_sm_count(&sms);
     if (err != cudaSuccess) return err;
-    for (int st = 0; st < N; ++st) {
-        if ((err = launch_k(ntlb_choose_kernel, dim3(g), dim3(256), 0, s, 1, a.probs, a.T, N, st, a.placed, a.last,
-                            a.first, a.ch)) != cudaSuccess)
-            return err;
-        if ((err = cudaMemsetAsync(&a.hdr->scan_ticket, 0, 2 * sizeof(int32_t), s)) != cudaSuccess) return err;
-        if ((err = cudaMemsetAsync(a.scan_state, 0, sizeof(uint32_t) * (size_t)nblk * (N + 1), s)) != cudaSuccess)
-            return err;
-        // this stage's claim numbers per expert in token order (no capacity: C = INT32_MAX)
-        if ((err = launch_k(scan_kernel, dim3((unsigned)nblk), dim3(kScanThreads), 0, s, 1,
-                            static_cast<const int32_t*>(a.ch), a.T, N + 1, 1, 0x7fffffff, nblk,
-                            static_cast<const int32_t*>(nullptr), a.lp, a.st_counts, a.st_kept, a.st_offsets,
-                            a.scan_state, a.hdr, kWaitLimitNs)) != cudaSuccess)
-            return err;
-        if ((err = launch_k(ntlb_place_kernel, dim3(g), dim3(256), 0, s, 1, a.probs, a.T, N, a.C,
-                            static_cast<const int32_t*>(a.ch), static_cast<const int32_t*>(a.lp),
-                            static_cast<const int32_t*>(a.claims), a.placed, a.expert, a.pos, a.gate)) != cudaSuccess)
-            return err;
-        if ((err = launch_k(ntlb_claims_kernel, dim3(1), dim3(128), 0, s, 1, N,
-                            static_cast<const int32_t*>(a.st_counts), a.claims)) != cudaSuccess)
-            return err;
-    }
-    if ((err = launch_k(ntlb_final_kernel, dim3(g), dim3(256), 0, s, 1, a.probs, a.T, N, a.C,
-                        static_cast<const int32_t*>(a.placed), static_cast<const int32_t*>(a.first), a.expert,
-                        a.gate, a.pos)) != cudaSuccess)
-        return err;
-    if ((err = launch_k(ntlb_offsets_kernel, dim3(1), dim3(32), 0, s, 1, N, a.C,
-                        static_cast<const int32_t*>(a.claims), a.counts, a.kept, a.offsets)) != cudaSuccess)
-        return err;
+    // co-residency: the cooperative launch fails rather than run a grid that does not fit
+    const int G = ntlb_grid_blocks(a.T, sms);
+    NtlbGrid g{};
+    g.probs = a.probs;
+    g.T = a.T;
+    g.N = a.N;
+    g.C = a.C;
+    g.TB = (a.T + G - 1) / G;
+    g.expert = a.expert;
+    g.gate = a.gate;
+    g.pos = a.pos;
+    g.counts = a.counts;
+    g.kept = a.kept;
+    g.offsets = a.offsets;
+    g.ch = a.ch;
+    g.last = a.last;
+    g.first = a.first;
+    g.placed = a.placed;
+    g.lp = a.lp;
+    g.agg = a.grid_agg;
+    g.unplaced = a.grid_unplaced;
+    g.bar = a.grid_bar;
+    g.status = &a.hdr->status;
+    g.limit_ns = kWaitLimitNs;
+    if ((err = cudaMemsetAsync(a.grid_bar, 0, sizeof(uint32_t), s)) != cudaSuccess) return err;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)G);
+    cfg.blockDim = dim3(kScanThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if ((err = cudaLaunchKernelEx(&cfg, ntlb_grid_kernel, g)) != cudaSuccess) return err;
     // the gather, from the final experts and claim numbers (rank 0, no claim base)
     const unsigned grid = (unsigned)((a.T + 7) / 8) + (a.aux.G > 0 ? 1u : 0u);
     const int32_t* none = nullptr;
+    const int N = a.N;
     if (a.dtype == MOE_BF16)
         return launch_k(scatter_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, 1,
                         reinterpret_cast<const __nv_bfloat16*>(a.x), static_cast<const int32_t*>(a.expert),

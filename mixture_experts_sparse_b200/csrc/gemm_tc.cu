@@ -6,6 +6,8 @@
 //   stage 1, SwiGLU : H = silu(A W1[e]^T + b1[e]) * (A W3[e]^T + b3[e])
 //   stage 2         : Y = H W2[e]^T + b2[e]            (compact rows), or
 //   stage 2, scatter: out[row_token[r]] = row_gate[r] * (H W2[e]^T + b2[e])[r]
+//                     (expert parallelism: out is that of GPU row_rank[r], reached
+//                     through a peer pointer; row_gate may be absent)
 // which is the expert FFN of "From Switch Transformer to GLaM" (FFN(x) =
 // W2 s(W1 x)), the Mixtral SwiGLU expert of CMU 10-423 Lecture 16 section 2.3,
 // and the gate-scaled top-1 combine y = p_{i*} E_{i*}(x) of the GLaM page.
@@ -82,7 +84,9 @@ struct GemmParams {
     const __nv_bfloat16* bias3;
     __nv_bfloat16* out;
     const int32_t* row_token;
-    const float* row_gate;
+    const float* row_gate;        // scatter: nullable (no gate)
+    void* const* out_ptrs;        // scatter to several GPUs: row r goes to out_ptrs[row_rank[r]]
+    const int32_t* row_rank;
     int32_t* status;
     long long limit_ns;
 };
@@ -339,10 +343,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const int64_t grow = (int64_t)ti.row0 + r_in_tile;
             int64_t orow = grow;
             float g = 1.f;
+            __nv_bfloat16* obase = p.out;   // this row's destination tensor
             if (EPI == EPI_SCATTER && valid) {
                 orow = p.row_token[grow];
-                g = p.row_gate[grow];
+                if (p.row_gate) g = p.row_gate[grow];
+                if (p.row_rank) obase = reinterpret_cast<__nv_bfloat16*>(p.out_ptrs[p.row_rank[grow]]);
             }
+            __nv_bfloat16* my_dst = valid ? obase + orow * (int64_t)p.out_ld : nullptr;
             const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
             const __nv_bfloat16* bias_e = p.bias ? p.bias + (int64_t)ti.e * p.n_dim : nullptr;
             const __nv_bfloat16* bias3_e = p.bias3 ? p.bias3 + (int64_t)ti.e * p.n_dim : nullptr;
@@ -352,9 +359,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 #pragma unroll
             for (int k4 = 0; k4 < 8; ++k4) {
                 const int r = 4 * k4 + (lane >> 3);
-                const bool rv = __shfl_sync(0xffffffffu, valid, r);
-                const long long ro = __shfl_sync(0xffffffffu, (long long)orow, r);
-                dst_row[k4] = rv ? p.out + ro * (int64_t)p.out_ld : nullptr;
+                dst_row[k4] = reinterpret_cast<__nv_bfloat16*>(
+                    __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my_dst), r));
             }
 #pragma unroll 1
             for (int c = 0; c < BN_OUT / CW; ++c) {
@@ -585,10 +591,12 @@ cudaError_t launch_expert_ffn_tc(const FfnArgs& a, cudaStream_t s) {
     p2.bias = reinterpret_cast<const __nv_bfloat16*>(a.b2);
     p2.status = &a.hdr->status;
     p2.limit_ns = kWaitLimitNs;
-    if (a.scatter_out) {
+    if (a.scatter_out || a.scatter_ptrs) {
         p2.out = reinterpret_cast<__nv_bfloat16*>(a.scatter_out);
         p2.row_token = a.row_token;
         p2.row_gate = a.row_gate;
+        p2.out_ptrs = a.scatter_ptrs;
+        p2.row_rank = a.row_rank;
         return run_gemm_any<EPI_SCATTER>(mA2, mB2, mB2, p2, s);
     }
     p2.out = reinterpret_cast<__nv_bfloat16*>(a.ye);

@@ -21,7 +21,9 @@
 //     serialised by the caller.
 //   - The device address of the array is looked up once per device, on the
 //     first call made with that device current; make that first call before
-//     any stream capture begins.
+//     any stream capture begins.  The address is kept for the life of the
+//     process, which assumes the device's primary context lives as long (no
+//     cudaDeviceReset between calls).
 // The kernels launched are those of moe_dispatch.
 #include <mutex>
 
@@ -31,9 +33,8 @@ namespace moe {
 namespace {
 
 constexpr int64_t kNoAllocMaxTokens = int64_t(1) << 18;
-constexpr int kScanTokensPerBlock = 1024;   // the dispatch scan's block size
-constexpr size_t kNoAllocFlagWords =
-    (size_t)((kNoAllocMaxTokens + kScanTokensPerBlock - 1) / kScanTokensPerBlock) * 2 * 128;
+// one look-back word per (scan block, rank, expert) at the largest T, k and N
+constexpr size_t kNoAllocFlagWords = (size_t)((kNoAllocMaxTokens + kScanTokens - 1) / kScanTokens) * 2 * 128;
 constexpr size_t kNoAllocBytes = sizeof(WsHeader) + kNoAllocFlagWords * sizeof(uint32_t);
 
 }  // namespace
@@ -79,16 +80,9 @@ extern "C" int32_t moe_dispatch_noalloc(const moe_config* cfg, const void* x, co
                                         int32_t* offsets, int32_t* row_token, float* row_gate, void* xe,
                                         int32_t* status, void* stream) {
     using namespace moe;
-    if (!cfg) return MOE_ERR_INVALID_ARG;
+    const int32_t st = validate_config(cfg);   // the checks every entry point makes
+    if (st != MOE_OK) return st;
     const moe_config& c = *cfg;
-    if (c.T < 0 || c.d_model < 1 || c.d_ff < 1 || c.n_experts < 1 || c.top_k < 1 || c.capacity < 0 ||
-        (c.dtype != MOE_F32 && c.dtype != MOE_BF16) || (c.act != MOE_RELU && c.act != MOE_SWIGLU) ||
-        c.top_k > c.n_experts)
-        return MOE_ERR_INVALID_ARG;
-    if (c.priority != MOE_ORDER_TOKEN && c.priority != MOE_ORDER_PRIORITY && c.priority != MOE_ORDER_NTLB)
-        return MOE_ERR_INVALID_ARG;
-    if (c.n_experts > 128 || c.top_k > 2 || (c.dtype == MOE_BF16 && (c.d_model % 16 != 0 || c.d_ff % 16 != 0)))
-        return MOE_ERR_UNSUPPORTED;
     if (c.priority != MOE_ORDER_TOKEN) return MOE_ERR_UNSUPPORTED;   // its scratch has no room for the sort
     if (c.T > kNoAllocMaxTokens ||   // beyond the static scratch
         (size_t)scan_blocks(c.T) * c.top_k * c.n_experts > kNoAllocFlagWords)

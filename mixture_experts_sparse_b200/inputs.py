@@ -8,7 +8,8 @@ Limitations", section 2.2, and "From Switch Transformer to GLaM"):
     nearest even);
   * every weight matrix from a normal truncated at 2 sigma (out-of-range draws
     are redrawn), sigma = sqrt(0.1 / fan_in); fan_in is d_model for W_r, W1,
-    W3 and d_ff for W2; optional biases use the same law and fan-in;
+    W3 and d_ff for W2; optional biases use the same law and fan-in; each
+    expert's matrix comes from its own child seed stream;
   * the router W_r stays fp32; expert weights take the activation dtype;
   * skewed routing: router bias b_r[i] = 3 ln(pi_i), pi_i proportional to
     (i + 1)^-s over the experts;
@@ -17,9 +18,16 @@ Limitations", section 2.2, and "From Switch Transformer to GLaM"):
     discrete routing is unique.
 bf16 tensors are returned as uint16 bit patterns.
 """
+import concurrent.futures
+import os
+
 import numpy as np
 
 GAP = 1e-4
+
+
+def _threads():
+    return max(1, len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1))
 
 
 def _bf16_bits(a32):
@@ -85,15 +93,19 @@ def _small_gap(x_val, w_r, b_r, k):
 
 def make_layer(T, d_model, d_ff, n_experts, top_k=1, act="relu", dtype="bf16",
                norm="layernorm", biases=False, zipf_exponent=None, seed=0,
-               router_bias=None, gap_guard=True, **_ignored):
+               router_bias=None, gap_guard=True, x_seed=None, **_ignored):
     """Build one layer's inputs and weights.
 
     Returns a dict of numpy arrays: x [T, d] (uint16 bf16 bits or fp32), w_r
     [N, d] fp32, b_r [N] fp32 or None, w1 [N, d_ff, d], w3 (SwiGLU) or None,
-    w2 [N, d, d_ff], b1 [N, d_ff] / b3 / b2 [N, d] or None.
+    w2 [N, d, d_ff], b1 [N, d_ff] / b3 / b2 [N, d] or None.  x_seed (optional)
+    draws x from its own seed while the weights still come from `seed` (the
+    shards of one routing group share the weights).
     """
     ss = np.random.SeedSequence(seed)
     s_x, s_r, s_1, s_3, s_2, s_b = ss.spawn(6)
+    if x_seed is not None:
+        s_x = np.random.SeedSequence(x_seed).spawn(1)[0]
     N, d = n_experts, d_model
     rng_r = np.random.default_rng(s_r)
     w_r = _trunc_normal(rng_r, (N, d), np.sqrt(0.1 / d))
@@ -118,13 +130,23 @@ def make_layer(T, d_model, d_ff, n_experts, top_k=1, act="relu", dtype="bf16",
             raise RuntimeError("gap guard did not converge")
 
     def weight(seed_seq, shape, fan_in):
-        rng = np.random.default_rng(seed_seq)
-        if dtype == "bf16":
-            out = np.empty(shape, dtype=np.uint16)
-            for e in range(shape[0]):
-                out[e] = _bf16_bits(_trunc_normal(rng, shape[1:], np.sqrt(0.1 / fan_in)))
-            return out
-        return _trunc_normal(rng, shape, np.sqrt(0.1 / fan_in))
+        # one child stream per expert, so the experts can be drawn on several
+        # host threads (numpy's generators release the GIL while filling)
+        sigma = np.sqrt(0.1 / fan_in)
+        out = np.empty(shape, dtype=np.uint16 if dtype == "bf16" else np.float32)
+
+        def draw(e, ss):
+            w = _trunc_normal(np.random.default_rng(ss), shape[1:], sigma)
+            out[e] = _bf16_bits(w) if dtype == "bf16" else w
+
+        children = seed_seq.spawn(shape[0])
+        if out.nbytes < (64 << 20):
+            for e, ss in enumerate(children):
+                draw(e, ss)
+        else:
+            with concurrent.futures.ThreadPoolExecutor(max_workers=min(shape[0], _threads())) as ex:
+                list(ex.map(lambda a: draw(*a), enumerate(children)))
+        return out
 
     w1 = weight(s_1, (N, d_ff, d), d)
     w3 = weight(s_3, (N, d_ff, d), d) if act == "swiglu" else None
@@ -138,9 +160,9 @@ def make_layer(T, d_model, d_ff, n_experts, top_k=1, act="relu", dtype="bf16",
     return dict(x=x_store, w_r=w_r, b_r=b_r, w1=w1, w3=w3, w2=w2, b1=b1, b3=b3, b2=b2)
 
 
-def make_workload(w, **overrides):
+def make_workload(w, x_seed=None, **overrides):
     """Inputs for a configs.Workload (fields may be overridden, e.g. T=...)."""
     w = w.scaled(**overrides) if overrides else w
     return make_layer(T=w.T, d_model=w.d_model, d_ff=w.d_ff, n_experts=w.n_experts,
                       top_k=w.top_k, act=w.act, dtype=w.dtype, norm=w.norm, biases=w.biases,
-                      zipf_exponent=w.zipf_exponent, seed=w.seed)
+                      zipf_exponent=w.zipf_exponent, seed=w.seed, x_seed=x_seed)

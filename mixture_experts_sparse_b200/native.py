@@ -56,6 +56,12 @@ _SIGS = {
     "moe_claim_base": ([_P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _P, _P], ctypes.c_int32),
     "moe_aux_shards": ([ctypes.c_int32, ctypes.c_int32, _P, _P, _P, ctypes.c_float, _P, _P, _P, _P],
                        ctypes.c_int32),
+    "moe_ep_recv_rows": ([ctypes.POINTER(MoeConfig), ctypes.c_int32], ctypes.c_int64),
+    "moe_ep_workspace_bytes": ([ctypes.POINTER(MoeConfig), ctypes.c_int32], ctypes.c_size_t),
+    "moe_ep_layout": ([ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _P, _P, _P, _P], ctypes.c_int32),
+    "moe_ep_dispatch": ([ctypes.POINTER(MoeConfig), ctypes.c_int32, ctypes.c_int32] + [_P] * 12, ctypes.c_int32),
+    "moe_ep_expert_ffn": ([ctypes.POINTER(MoeConfig), ctypes.c_int32] + [_P] * 13 + [ctypes.c_size_t, _P],
+                          ctypes.c_int32),
     "moe_read_device_status": ([_P, _P], ctypes.c_int32),
     "moe_test_lookback_timeout": ([_P, ctypes.c_size_t, ctypes.c_int64, _P], ctypes.c_int32),
 }
@@ -246,3 +252,32 @@ def moe_read_device_status(ws, stream=None):
 
 def moe_test_lookback_timeout(ws, limit_ns, stream=None):
     return lib().moe_test_lookback_timeout(_p(ws), _nbytes(ws), int(limit_ns), _s(stream))
+
+
+# ---- expert parallelism (pointer tables are device int64 tensors of addresses)
+
+def moe_ep_recv_rows(cfg, n_ranks):
+    return int(lib().moe_ep_recv_rows(ctypes.byref(cfg), int(n_ranks)))
+
+
+def moe_ep_workspace_bytes(cfg, n_ranks):
+    return int(lib().moe_ep_workspace_bytes(ctypes.byref(cfg), int(n_ranks)))
+
+
+def moe_ep_layout(n_ranks, rank, n_experts, kept_all, dst_start, recv_offsets, stream=None):
+    return lib().moe_ep_layout(int(n_ranks), int(rank), int(n_experts), _p(kept_all), _p(dst_start),
+                               _p(recv_offsets), _s(stream))
+
+
+def moe_ep_dispatch(cfg, n_ranks, rank, x, offsets, row_token, row_gate, drop, dst_start, recv_x, recv_rank,
+                    recv_row, recv_gate, out, stream=None):
+    return lib().moe_ep_dispatch(ctypes.byref(cfg), int(n_ranks), int(rank), _p(x), _p(offsets), _p(row_token),
+                                 _p(row_gate), _p(drop), _p(dst_start), _p(recv_x), _p(recv_rank), _p(recv_row),
+                                 _p(recv_gate), _p(out), _s(stream))
+
+
+def moe_ep_expert_ffn(cfg, n_ranks, recv_x, recv_offsets, w1, b1, w3, b3, w2, b2, recv_rank, recv_row, recv_gate,
+                      out_ptrs, ws, stream=None):
+    return lib().moe_ep_expert_ffn(ctypes.byref(cfg), int(n_ranks), _p(recv_x), _p(recv_offsets), _p(w1), _p(b1),
+                                   _p(w3), _p(b3), _p(w2), _p(b2), _p(recv_rank), _p(recv_row), _p(recv_gate),
+                                   _p(out_ptrs), _p(ws), _nbytes(ws), _s(stream))

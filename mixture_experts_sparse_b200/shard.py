@@ -86,17 +86,23 @@ class Shard:
         nat.check(nat.moe_aux_shards(all_tokens.shape[0], self.N, all_tokens, all_f, all_P, self.alpha, f, P, aux))
 
 
-def sharded_forward(shards, xs, all_gather, first_index=0):
+def sharded_forward(shards, xs, all_gather, first_index=0, mark=None):
     """Run the forward of the given shards (shards[i] on input xs[i], group
     shard index first_index + i) with the exchanges done by all_gather.  In one
     process (emulation) pass every shard with local_stack; across GPUs each rank
-    passes its own shard, first_index = rank, and rank_all_gather.
+    passes its own shard, first_index = rank, and rank_all_gather.  mark
+    (optional) is called with "experts" and "experts_done" around the expert
+    FFN and combine calls (e.g. to record CUDA events there).
     Returns (outputs, group f, group P, group aux) of the shards given."""
     claims = [s.route_and_count(x) for s, x in zip(shards, xs)]
     all_claims = all_gather(claims)
     for i, (s, x) in enumerate(zip(shards, xs)):
         s.dispatch(x, all_claims, first_index + i)
+    if mark:
+        mark("experts")
     outs = [s.experts_and_combine() for s in shards]
+    if mark:
+        mark("experts_done")
     all_tokens = all_gather([s.tokens for s in shards]).reshape(-1)
     all_f = all_gather([s.f for s in shards])
     all_P = all_gather([s.P for s in shards])

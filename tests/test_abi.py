@@ -33,6 +33,28 @@ def test_library_exports_every_declared_symbol():
     assert set(nat._SIGS) >= set(names)
 
 
+def declared_arity():
+    """Number of parameters of every entry point declared in include/*.h."""
+    out = {}
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if not h.endswith(".h"):
+            continue
+        text = open(os.path.join(ROOT, "include", h)).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"\b(moe_\w+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S):
+            params = m.group(2).strip()
+            out[m.group(1)] = 0 if params in ("", "void") else params.count(",") + 1
+    return out
+
+
+def test_binding_signatures_match_the_header():
+    # every ctypes signature has as many arguments as the C declaration
+    arity = declared_arity()
+    assert arity["moe_forward"] == 24 and arity["moe_ep_dispatch"] == 15
+    for name, (args, _) in nat._SIGS.items():
+        assert len(args) == arity[name], (name, len(args), arity[name])
+
+
 def test_capacity_matches_oracle():
     rng = np.random.default_rng(0)
     cases = [(1024, 8, 2, 1.25), (65536, 64, 1, 1.25), (32768, 32, 2, 2.0), (16384, 8, 2, 1.25),
