@@ -459,6 +459,87 @@ def workload_summary(w, C, t, kept_rows, touched, pk):
     }
 
 
+def time_backward(w, L, layer, x, C, K, warmup, pk):
+    """The layer's backward on the same batch: the expert FFN backward
+    (moe_expert_backward: recompute of the first GEMM, dA, dx, dW1/dW3, dW2 and
+    the bias sums) and the router backward (moe_gate_grad + moe_router_backward).
+    Algorithmic FLOPs of the expert backward: dA, dx, dW1 (dW3), dW2 =
+    (4 ReLU | 6 SwiGLU) x 2 d d_ff per kept row; the recompute is not counted."""
+    import torch
+
+    from mixture_experts_sparse_b200 import native as nat
+    T, d, dff, N, k = w.T, w.d_model, w.d_ff, w.n_experts, w.top_k
+    dev = dict(device="cuda")
+    cfg = layer.cfg
+    R = max(1, min(k * T, N * C))
+    i32, f32 = torch.int32, torch.float32
+    idx = torch.empty(T, k, dtype=i32, **dev)
+    gate = torch.empty(T, k, dtype=f32, **dev)
+    probs = torch.empty(T, N, dtype=f32, **dev)
+    pos = torch.empty(T, k, dtype=i32, **dev)
+    drop = torch.empty(T, k, dtype=torch.uint8, **dev)
+    counts = torch.empty(k, N, dtype=i32, **dev)
+    kept = torch.empty(N, dtype=i32, **dev)
+    offsets = torch.empty(N + 1, dtype=i32, **dev)
+    row_token = torch.empty(R, dtype=i32, **dev)
+    row_gate = torch.empty(R, dtype=f32, **dev)
+    xe = torch.empty(R, d, dtype=torch.bfloat16, **dev)
+    ye = torch.empty(R, d, dtype=torch.bfloat16, **dev)
+    fv = torch.empty(N, dtype=torch.float64, **dev)
+    Wl = layer.w
+    nat.check(nat.moe_route(cfg, x, Wl["w_r"], Wl["b_r"], idx, gate, probs, fv, None, None, layer.ws))
+    nat.check(nat.moe_dispatch(cfg, x, idx, gate, pos, drop, counts, kept, offsets, row_token, row_gate, xe,
+                               layer.ws))
+    nat.check(nat.moe_expert_ffn(cfg, xe, offsets, Wl["w1"], Wl["b1"], Wl["w3"], Wl["b3"], Wl["w2"], Wl["b2"], ye,
+                                 layer.ws))
+    dout = (0.1 * torch.randn(T, d, **dev)).to(torch.bfloat16)
+    nb = nat.moe_expert_backward_workspace_bytes(cfg)
+    wsb = torch.empty(nb, dtype=torch.uint8, **dev)
+    nat.check(nat.moe_workspace_init(wsb))
+    sw = w.act == "swiglu"
+    dx = torch.empty(T, d, dtype=f32, **dev)
+    dw1 = torch.empty(N, dff, d, dtype=f32, **dev)
+    dw3 = torch.empty(N, dff, d, dtype=f32, **dev) if sw else None
+    dw2 = torch.empty(N, d, dff, dtype=f32, **dev)
+    dgate = torch.empty(T, k, dtype=f32, **dev)
+    dh = torch.empty(T, N, dtype=f32, **dev)
+    dwr = torch.empty(N, d, dtype=f32, **dev)
+    dxr = torch.empty(T, d, dtype=f32, **dev)
+    stream = torch.cuda.current_stream()
+
+    def expert():
+        nat.check(nat.moe_expert_backward(cfg, xe, offsets, row_token, row_gate, idx, pos, drop, dout, Wl["w1"],
+                                          Wl["b1"], Wl["w3"], Wl["b3"], Wl["w2"], dx, dw1, None, dw3, None, dw2,
+                                          None, wsb))
+
+    def router():
+        nat.check(nat.moe_gate_grad(cfg, dout, ye, idx, pos, drop, offsets, dgate))
+        nat.check(nat.moe_router_backward(cfg, x, Wl["w_r"], probs, idx, gate, fv, dgate, dh, dwr, None, dxr,
+                                          layer.ws))
+
+    out = {}
+    for name, fn in (("expert", expert), ("router", router)):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(K):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out[name] = e0.elapsed_time(e1) / K
+    nat.check(nat.moe_read_device_status(wsb))
+    nat.check(nat.moe_read_device_status(layer.ws))
+    kept_rows = int(offsets[-1].item())
+    flops = (6 if sw else 4) * 2 * d * dff * kept_rows
+    ach = flops / (out["expert"] * 1e-3) / 1e12
+    return {"expert_ms": out["expert"], "router_ms": out["router"], "expert_flops": flops,
+            "expert_achieved_tflops": ach, "expert_frac": ach / pk["bf16_tflops"],
+            "note": "expert backward: recompute of the first GEMM + dA, dx, dW1 (dW3), dW2 on the tensor cores; "
+                    "FLOPs count dA, dx and the weight gradients only; router backward on the FP32 pipe"}
+
+
 def build_layer(w, rank, local, x_seed=None):
     import torch
 
@@ -570,6 +651,8 @@ def run_single(args, local):
         kept_rows = int(layer.offsets[-1].item())
         touched = int((layer.kept > 0).sum().item())
         blocks[name] = workload_summary(w, C, t, kept_rows, touched, pk)
+        if w.dtype == "bf16" and not args.no_backward:
+            blocks[name]["backward"] = time_backward(w, L, layer, x, C, max(3, min(K, 10)), 2, pk)
         if name == args.workload:
             e2e_ms, h2d, d2h = e2e_single(layer, x, K, W)
             cpu = None if args.no_cpu_baseline else cpu_baselines(L, w, args.cpu_seconds)
@@ -804,6 +887,7 @@ def main():
                     help="N > 1: one independent routing group per GPU instead of one group split over the GPUs")
     ap.add_argument("--tokens", type=int, default=None, help="override the workload's T (profiling runs)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward timing of each workload")
     ap.add_argument("--no-graph", action="store_true", help="time direct moe_forward calls instead of graph replay")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--reference-budget-s", type=float, default=150.0)

@@ -31,8 +31,8 @@
  * z-loss (moe_route_z), one routing group split over several GPUs with one
  * small exchange (moe_expert_counts, moe_claim_base, moe_dispatch_shard,
  * moe_combine_shard, moe_aux_shards), the experts spread over several GPUs
- * with all-to-all dispatch and combine (moe_ep_*), the router backward
- * (moe_gate_grad, moe_router_backward), and a dispatch that needs no workspace
+ * with all-to-all dispatch and combine (moe_ep_*), the backward (moe_gate_grad,
+ * moe_router_backward, moe_expert_backward), and a dispatch that needs no workspace
  * (moe_dispatch_noalloc).
  *
  * Conventions shared by every entry point
@@ -190,6 +190,32 @@ int32_t moe_router_backward(const moe_config* cfg, const void* x, const float* w
                             const int32_t* idx, const float* gate, const double* f, const float* dgate,
                             float* dh, float* dw_r, float* db_r, float* dx,
                             void* ws, size_t ws_bytes, void* stream);
+
+/* Backward of the expert FFN (bf16, on the tensor cores): gradients of
+ * L = sum_t <dout_t, out_t> through the combine, the expert FFNs and their
+ * weights ("From Switch Transformer to GLaM", FFN(x) = W2 s(W1 x); CMU 10-423
+ * Lecture 16, section 2.3, SwiGLU expert), with the gates held fixed (their
+ * gradient is moe_gate_grad's).  For a kept row r of expert e (token t, gate
+ * g): dY = g dout_t; dA = dY W2[e]; dU = dA * relu'(u) (SwiGLU: dG = dA * up *
+ * silu'(gate pre-activation), dUp = dA * silu(gate pre-activation));
+ * dx_t += dU W1[e] (+ dUp W3[e]); dW1[e] = sum_r dU^T x, dW3[e] = sum_r dUp^T x,
+ * dW2[e] = sum_r dY^T a; db1, db3, db2 the column sums of dU, dUp, dY.  The
+ * first GEMM is recomputed from xe (its activations are not kept by the
+ * forward).  bf16 operands, fp32 accumulation; gradients are fp32.
+ * In:  xe [R, d], offsets [N + 1], row_token, row_gate [R] (moe_dispatch's),
+ *      idx, pos, drop [T, k], dout [T, d] bf16, w1, w3 [N, d_ff, d], w2
+ *      [N, d, d_ff], b1, b3 [N, d_ff] (nullable).
+ * Out: dx [T, d] fp32 (the expert part of dL/dx; 0 for a token with no kept
+ *      assignment), dw1, dw3 [N, d_ff, d], dw2 [N, d, d_ff], db1, db3 [N, d_ff],
+ *      db2 [N, d] fp32 (each nullable; experts without rows get zeros).
+ * ws: moe_expert_backward_workspace_bytes(cfg) bytes, moe_workspace_init'ed.
+ * MOE_ERR_UNSUPPORTED for MOE_F32, and for SwiGLU with d_ff not a multiple of 64. */
+size_t moe_expert_backward_workspace_bytes(const moe_config* cfg);
+int32_t moe_expert_backward(const moe_config* cfg, const void* xe, const int32_t* offsets, const int32_t* row_token,
+                            const float* row_gate, const int32_t* idx, const int32_t* pos, const uint8_t* drop,
+                            const void* dout, const void* w1, const void* b1, const void* w3, const void* b3,
+                            const void* w2, float* dx, float* dw1, float* db1, float* dw3, float* db3, float* dw2,
+                            float* db2, void* ws, size_t ws_bytes, void* stream);
 
 /* Capacity-limited dispatch (row A3 and the gather of A4).
  * In:  x [T, d] (dtype; nullable when xe is NULL), idx [T, k], gate [T, k].

@@ -693,6 +693,110 @@ int32_t moe_forward_events(const moe_config* cfg, const void* x, const float* w_
                         f, P, aux, ws, ws_bytes, (cudaStream_t)stream, events);
 }
 
+// ---- expert FFN backward ---------------------------------------------------
+
+struct BwdLayout {
+    size_t hdr, h, pre, dy, du, dxe, total;
+    int64_t rows;
+};
+
+static BwdLayout bwd_layout(const moe_config& c) {
+    BwdLayout L{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t o = off;
+        off += round_up(bytes > 0 ? bytes : 1, 256);
+        return o;
+    };
+    L.rows = compact_rows(c);
+    const size_t R = (size_t)(L.rows > 0 ? L.rows : 1), d = (size_t)c.d_model, dff = (size_t)c.d_ff;
+    const bool sw = c.act == MOE_SWIGLU;
+    L.hdr = take(sizeof(WsHeader));
+    L.h = take(2 * R * dff);
+    L.pre = take(sw ? 2 * R * 2 * dff : 0);
+    L.dy = take(2 * R * d);
+    L.du = take(2 * R * (sw ? 2 : 1) * dff);
+    L.dxe = take(c.top_k == 2 ? 4 * R * d : 0);
+    L.total = off;
+    return L;
+}
+
+size_t moe_expert_backward_workspace_bytes(const moe_config* cfg) {
+    if (validate(cfg) != MOE_OK || cfg->dtype != MOE_BF16) return 0;
+    return bwd_layout(*cfg).total;
+}
+
+int32_t moe_expert_backward(const moe_config* cfg, const void* xe, const int32_t* offsets, const int32_t* row_token,
+                            const float* row_gate, const int32_t* idx, const int32_t* pos, const uint8_t* drop,
+                            const void* dout, const void* w1, const void* b1, const void* w3, const void* b3,
+                            const void* w2, float* dx, float* dw1, float* db1, float* dw3, float* db3, float* dw2,
+                            float* db2, void* ws, size_t ws_bytes, void* stream) {
+    int32_t st = validate(cfg);
+    if (st != MOE_OK) return st;
+    if (cfg->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;   // the tensor-core backward is bf16
+    // SwiGLU: the dx GEMM reads W1 then W3 along K in 64-row blocks
+    if (cfg->act == MOE_SWIGLU && cfg->d_ff % 64 != 0) return MOE_ERR_UNSUPPORTED;
+    if (!req(offsets) || !req(w1) || !req(w2) || !opt(b1) || !opt(b3) || !opt(dw1) || !opt(db1) || !opt(dw3) ||
+        !opt(db3) || !opt(dw2) || !opt(db2) || !opt(dx))
+        return MOE_ERR_INVALID_ARG;
+    if (cfg->act == MOE_SWIGLU ? !req(w3) : !opt(w3)) return MOE_ERR_INVALID_ARG;
+    const BwdLayout L = bwd_layout(*cfg);
+    if (!ws || !aligned(ws) || ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+    if (cfg->T > 0 && (!req(xe) || !req(row_token) || !req(row_gate) || !req(idx) || !req(pos) || !req(drop) ||
+                       !req(dout) || !req(dx)))
+        return MOE_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    // an expert with no rows has zero weight gradients; the kernels write them too
+    if (L.rows <= 0 || cfg->T == 0) {
+        cudaError_t e = cudaSuccess;
+        const size_t N = (size_t)cfg->n_experts, d = (size_t)cfg->d_model, dff = (size_t)cfg->d_ff;
+        if (dw1) e = cudaMemsetAsync(dw1, 0, 4 * N * dff * d, s);
+        if (e == cudaSuccess && dw3) e = cudaMemsetAsync(dw3, 0, 4 * N * dff * d, s);
+        if (e == cudaSuccess && dw2) e = cudaMemsetAsync(dw2, 0, 4 * N * dff * d, s);
+        if (e == cudaSuccess && db1) e = cudaMemsetAsync(db1, 0, 4 * N * dff, s);
+        if (e == cudaSuccess && db3) e = cudaMemsetAsync(db3, 0, 4 * N * dff, s);
+        if (e == cudaSuccess && db2) e = cudaMemsetAsync(db2, 0, 4 * N * d, s);
+        if (e == cudaSuccess && dx && cfg->T > 0) e = cudaMemsetAsync(dx, 0, 4 * (size_t)cfg->T * d, s);
+        return cuda_status(e);
+    }
+    BwdArgs a{};
+    a.act = cfg->act;
+    a.N = cfg->n_experts;
+    a.d = cfg->d_model;
+    a.d_ff = cfg->d_ff;
+    a.k = cfg->top_k;
+    a.T = cfg->T;
+    a.R_cap = L.rows;
+    a.xe = xe;
+    a.offsets = offsets;
+    a.row_token = row_token;
+    a.row_gate = row_gate;
+    a.idx = idx;
+    a.pos = pos;
+    a.drop = drop;
+    a.dout = dout;
+    a.w1 = w1;
+    a.b1 = b1;
+    a.w3 = w3;
+    a.b3 = b3;
+    a.w2 = w2;
+    a.dx = dx;
+    a.dw1 = dw1;
+    a.db1 = db1;
+    a.dw3 = dw3;
+    a.db3 = db3;
+    a.dw2 = dw2;
+    a.db2 = db2;
+    a.top1_scatter = cfg->top_k == 1;
+    a.h = at<void>(ws, L.h);
+    a.pre = at<void>(ws, L.pre);
+    a.dy = at<void>(ws, L.dy);
+    a.du = at<void>(ws, L.du);
+    a.dxe = at<float>(ws, L.dxe);
+    a.hdr = at<WsHeader>(ws, L.hdr);
+    return cuda_status(launch_expert_backward_tc(a, s));
+}
+
 // ---- expert parallelism --------------------------------------------------
 
 // The receiving GPU's view of a layer split over n_ranks GPUs: its E = N / G

@@ -303,8 +303,25 @@ struct FfnArgs {
     void* const* scatter_ptrs; const int32_t* row_rank;
     WsHeader* hdr;
     void* mid_event;              // optional cudaEvent_t recorded between the two stages
+    void* pre_out;                // SwiGLU (optional): stage-1 pre-activations [R, 2 d_ff]
+    bool stage1_only;             // the first GEMM only (the backward's recompute)
 };
 cudaError_t launch_expert_ffn(const FfnArgs& a, cudaStream_t s);
+cudaError_t launch_expert_ffn_tc(const FfnArgs& a, cudaStream_t s);
+
+// Expert FFN backward on the tensor cores (gemm_bwd.cu), bf16.
+struct BwdArgs {
+    int act; int N; int d; int d_ff; int k; int64_t T; int64_t R_cap;
+    const void* xe; const int32_t* offsets; const int32_t* row_token; const float* row_gate;
+    const int32_t* idx; const int32_t* pos; const uint8_t* drop;
+    const void* dout;
+    const void* w1; const void* b1; const void* w3; const void* b3; const void* w2;
+    float* dx; float* dw1; float* db1; float* dw3; float* db3; float* dw2; float* db2;
+    bool top1_scatter;            // dx rows scattered by token (top-1), else combined from dxe
+    void* h; void* pre; void* dy; void* du; float* dxe;   // workspace
+    WsHeader* hdr;
+};
+cudaError_t launch_expert_backward_tc(const BwdArgs& a, cudaStream_t s);
 
 // Expert parallelism (ep.cu)
 struct EpDispatchArgs {

@@ -1,0 +1,590 @@
+// Backward of the expert FFN on the 5th-generation tensor cores.
+//
+// Forward, per kept assignment (row r of expert e, token t, gate g):
+//   u = W1[e] x + b1,  a = relu(u)   (SwiGLU: a = silu(W1 x + b1) * (W3 x + b3)),
+//   y = W2[e] a + b2,  out_t += g y
+// ("From Switch Transformer to GLaM", FFN(x) = W2 s(W1 x); CMU 10-423 Lecture
+// 16, section 2.3, the Mixtral SwiGLU expert).  With dY[r] = g dL/dout_t:
+//   dA  = dY W2[e]                       (row GEMM, B = W2 read MN-major)
+//   dU  = dA * relu'(u)                   (SwiGLU: dG = dA * up * silu'(gate_pre),
+//                                          dUp = dA * silu(gate_pre))
+//   dx_t += dU W1[e]  (+ dUp W3[e])       (row GEMM, B = W1 / W3 read MN-major)
+//   dW1[e] = dU^T X_e,  dW3[e] = dUp^T X_e,  dW2[e] = dY^T A_e
+//                                         (weight GEMMs: the reduction runs
+//                                          over the expert's rows, both operands
+//                                          read MN-major)
+//   db1 = column sums of dU, db3 of dUp, db2 of dY.
+//
+// One kernel template, single CTA per tile (M = 128, N = 256), persistent,
+// warp-specialised like the forward GEMM: warp 0 TMA producer, warp 1 MMA
+// issuer (and, in the weight GEMMs, the warp that zeroes the rows of a K block
+// past the expert's last row, since those rows belong to the next expert),
+// warps 2-5 epilogue.  Operands:
+//   K-major A (row GEMMs): box 64 K x 128 rows, as in the forward;
+//   MN-major A / B: boxes of 64 MN elements x 64 K rows (128-byte swizzle), two
+//   for A (M = 128), four for B (N = 256), 8 KB apart.
+// Every mbarrier wait is bounded (MOE_ERR_TIMEOUT on expiry, then a bounded
+// drain of the copies and MMAs in flight before TMEM is freed).
+#include "tc_common.cuh"
+
+namespace moe {
+using namespace tc;
+namespace {
+
+constexpr int BW_BM = 128, BW_BN = 256, BW_BK = 64;
+constexpr int BW_THREADS = 192;
+constexpr int BW_STAGES = 4;
+constexpr int BW_A_BYTES = BW_BM * BW_BK * 2;   // 16 KB
+constexpr int BW_B_BYTES = BW_BN * BW_BK * 2;   // 32 KB
+constexpr int BW_STAGE_BYTES = BW_A_BYTES + BW_B_BYTES;
+constexpr int BW_SMEM = BW_STAGES * BW_STAGE_BYTES + 1024;
+constexpr int BW_TMEM_COLS = 512;
+constexpr int MN_BOX = 64 * BW_BK * 2;          // one MN-major box: 64 MN x 64 K rows = 8 KB
+
+enum { BW_DU_RELU = 0, BW_DU_SWIGLU = 1, BW_DX = 2, BW_WGT = 3 };
+
+struct BwdParams {
+    const int32_t* offsets;   // [N + 1] compact rows of each expert
+    int N;
+    int m_dim, n_dim, k_dim;  // weight GEMMs: M, N per expert (K = its rows); row GEMMs: N, K
+    int k_split;              // row GEMM with two B tensors: K blocks below k_split read B, above B2
+    // epilogues
+    const __nv_bfloat16* h;   // BW_DU_RELU: H [R, n_dim] (relu'(u) = H > 0)
+    const __nv_bfloat16* pre; // BW_DU_SWIGLU: gate and up pre-activations [R, 2 n_dim]
+    __nv_bfloat16* du;        // BW_DU_*: dU [R, n_dim] or dG | dUp [R, 2 n_dim]
+    float* out;               // BW_DX: dx rows (scatter: [T, n_dim] by row_token; else [R, n_dim]);
+                              // BW_WGT: dW [N, m_dim, n_dim]
+    const int32_t* row_token; // BW_DX scatter (top-1)
+    int32_t* status;
+    long long limit_ns;
+};
+
+struct BwTile {
+    int e, row0, rows, m0, n0, k_rows, k_row0;
+};
+
+template <int MODE>
+__device__ __forceinline__ BwTile bw_decode(int tile, const int* prefix, const int* off, int N, int ntm, int ntn) {
+    BwTile t{};
+    if (MODE == BW_WGT) {   // (expert, m-tile, n-tile) over every expert, n fastest
+        const int per_e = ntm * ntn;
+        t.e = tile / per_e;
+        const int rem = tile - t.e * per_e;
+        t.m0 = (rem / ntn) * BW_BM;
+        t.n0 = (rem % ntn) * BW_BN;
+        t.k_row0 = off[t.e];
+        t.k_rows = off[t.e + 1] - off[t.e];
+        return t;
+    }
+    int lo = 0, hi = N;   // prefix[lo] <= tile < prefix[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (prefix[mid] <= tile) lo = mid;
+        else hi = mid;
+    }
+    t.e = lo;
+    const int local = tile - prefix[lo];
+    const int m_blk = local / ntn;
+    t.n0 = (local - m_blk * ntn) * BW_BN;
+    t.row0 = off[lo] + m_blk * BW_BM;
+    t.rows = min(BW_BM, off[lo + 1] - t.row0);
+    return t;
+}
+
+__device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + expf(-z)); }
+
+template <int MODE>
+__global__ void __launch_bounds__(BW_THREADS, 1)
+bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const __grid_constant__ CUtensorMap tmB2, const BwdParams p) {
+    constexpr bool A_MN = MODE == BW_WGT;
+    constexpr uint32_t IDESC = idesc_bf16_f32_major(BW_BM, BW_BN, A_MN, true);
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+    __shared__ __align__(8) uint64_t full_bar[BW_STAGES];
+    __shared__ __align__(8) uint64_t empty_bar[BW_STAGES];
+    __shared__ __align__(8) uint64_t tfull_bar[2];
+    __shared__ __align__(8) uint64_t tempty_bar[2];
+    __shared__ __align__(8) uint64_t done_bar;
+    __shared__ uint32_t s_tmem;
+    __shared__ int s_abort;
+    __shared__ int s_off[129];
+    __shared__ int s_prefix[129];
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int N = p.N;
+    if (tid == 0) {
+        for (int s = 0; s < BW_STAGES; ++s) {
+            mbar_init(smem_u32(&full_bar[s]), 1);
+            mbar_init(smem_u32(&empty_bar[s]), 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(smem_u32(&tfull_bar[a]), 1);
+            mbar_init(smem_u32(&tempty_bar[a]), 128);
+        }
+        mbar_init(smem_u32(&done_bar), 1);
+        s_abort = 0;
+        mbar_fence_init();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+    }
+    if (warp == 1) tmem_alloc(&s_tmem, BW_TMEM_COLS);
+    pdl_wait();
+    pdl_launch();
+    for (int i = tid; i <= N; i += BW_THREADS) s_off[i] = p.offsets[i];
+    __syncthreads();
+    const int ntn = (p.n_dim + BW_BN - 1) / BW_BN;
+    const int ntm = (p.m_dim + BW_BM - 1) / BW_BM;
+    if (warp == 2) {
+        if (MODE == BW_WGT) {
+            if (lane == 0) s_prefix[N] = N * ntm * ntn;
+        } else {   // tiles per expert (128-row m-tiles x n-tiles) and their exclusive prefix
+            int cnt[4], sum = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int e = lane * 4 + j;
+                cnt[j] = e < N ? ((s_off[e + 1] - s_off[e] + BW_BM - 1) / BW_BM) * ntn : 0;
+                sum += cnt[j];
+            }
+            int incl = sum;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            int run = incl - sum;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int e = lane * 4 + j;
+                if (e < N) s_prefix[e] = run;
+                run += cnt[j];
+            }
+            if (lane == 31) s_prefix[N] = incl;
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+
+    const uint32_t tmem_base = s_tmem;
+    const int total = s_prefix[N];
+    const Waiter w{&s_abort, p.status, p.limit_ns};
+    auto nkb_of = [&](const BwTile& ti) {
+        return MODE == BW_WGT ? (ti.k_rows + BW_BK - 1) / BW_BK : (p.k_dim + BW_BK - 1) / BW_BK;
+    };
+
+    if (warp == 0) {
+        // ---------------- TMA producer ----------------
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int last_par[BW_STAGES];
+#pragma unroll
+            for (int s = 0; s < BW_STAGES; ++s) last_par[s] = -1;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+                const BwTile ti = bw_decode<MODE>(tile, s_prefix, s_off, N, ntm, ntn);
+                const int nkb = nkb_of(ti);
+                for (int kb = 0; kb < nkb; ++kb) {
+                    if (!wait_bar(smem_u32(&empty_bar[stage]), phase ^ 1u, w)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&full_bar[stage]);
+                    const uint32_t a_dst = smem_u32(smem + stage * BW_STAGE_BYTES);
+                    const uint32_t b_dst = a_dst + BW_A_BYTES;
+                    mbar_expect_tx(fb, BW_STAGE_BYTES);
+                    if (MODE == BW_WGT) {
+                        const int kr = ti.k_row0 + kb * BW_BK;   // rows of the expert (K)
+#pragma unroll
+                        for (int j = 0; j < 2; ++j) tma_load_2d(a_dst + j * MN_BOX, &tmA, fb, ti.m0 + 64 * j, kr);
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) tma_load_2d(b_dst + j * MN_BOX, &tmB, fb, ti.n0 + 64 * j, kr);
+                    } else {
+                        tma_load_2d(a_dst, &tmA, fb, kb * BW_BK, ti.row0);
+                        // B = weights [N_exp * K rows][n cols]; two tensors split at k_split
+                        const bool second = p.k_split > 0 && kb * BW_BK >= p.k_split;
+                        const int kk = second ? kb * BW_BK - p.k_split : kb * BW_BK;
+                        const int kdim_b = p.k_split > 0 ? p.k_split : p.k_dim;
+                        const CUtensorMap* bm = second ? &tmB2 : &tmB;
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+                            tma_load_2d(b_dst + j * MN_BOX, bm, fb, ti.n0 + 64 * j, ti.e * kdim_b + kk);
+                    }
+                    last_par[stage] = (int)phase;
+                    if (++stage == BW_STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            for (int s = 0; s < BW_STAGES; ++s)
+                if (last_par[s] >= 0) drain_bar(smem_u32(&full_bar[s]), (uint32_t)last_par[s], p.limit_ns, p.status);
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer (lane 0); the warp zeroes K rows past an expert's end ----------------
+        int stage = 0;
+        uint32_t phase = 0;
+        int it = 0;
+        bool ok = true, issued = false;
+        for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+            const BwTile ti = bw_decode<MODE>(tile, s_prefix, s_off, N, ntm, ntn);
+            const int nkb = nkb_of(ti);
+            const int acc = it & 1;
+            const uint32_t acc_par = (uint32_t)((it >> 1) & 1);
+            bool got = wait_bar(smem_u32(&tempty_bar[acc]), acc_par ^ 1u, w);
+            if (!__all_sync(0xffffffffu, got)) break;
+            tc_fence_after();
+            const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BW_BN);
+            for (int kb = 0; kb < nkb; ++kb) {
+                got = wait_bar(smem_u32(&full_bar[stage]), phase, w);   // every lane: the copies have landed
+                if (!__all_sync(0xffffffffu, got)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t a_addr = smem_u32(smem + stage * BW_STAGE_BYTES);
+                const uint32_t b_addr = a_addr + BW_A_BYTES;
+                if (MODE == BW_WGT) {
+                    const int valid = ti.k_rows - kb * BW_BK;   // K rows of this block that are the expert's
+                    if (valid < BW_BK) {
+                        // rows [valid, 64) of each box: the next expert's rows (or out of bounds)
+                        uint8_t* st = smem + stage * BW_STAGE_BYTES;
+                        const int nz = (BW_BK - valid) * 128 / 16;   // 16-byte words per box
+                        for (int bx = 0; bx < 6; ++bx) {
+                            uint4* z = reinterpret_cast<uint4*>(st + bx * MN_BOX + valid * 128);
+                            for (int q = lane; q < nz; q += 32) z[q] = make_uint4(0, 0, 0, 0);
+                        }
+                        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                        __syncwarp();
+                    }
+                }
+                if (lane == 0) {
+                    issued = true;
+#pragma unroll
+                    for (int kk = 0; kk < BW_BK / 16; ++kk) {
+                        const uint64_t ad = A_MN ? umma_desc_mn(a_addr + kk * 2048, MN_BOX) : umma_desc(a_addr + kk * 32);
+                        const uint64_t bd = umma_desc_mn(b_addr + kk * 2048, MN_BOX);
+                        umma_f16(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    umma_commit(smem_u32(&empty_bar[stage]));
+                }
+                __syncwarp();
+                if (++stage == BW_STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
+            // no K block (an expert without rows): the accumulator is never written, and
+            // the epilogue writes zeros; the commit still orders the hand-over
+            if (ok && lane == 0) umma_commit(smem_u32(&tfull_bar[acc]));
+            __syncwarp();
+        }
+        if (lane == 0) {
+            umma_commit(smem_u32(&done_bar));
+            drain_bar(smem_u32(&done_bar), 0u, p.limit_ns, p.status);
+        }
+        (void)issued;
+        __syncwarp();
+    } else {
+        // ---------------- epilogue (warps 2..5): thread = accumulator row ----------------
+        const int q = warp & 3;
+        const int r_in = q * 32 + lane;
+        int it = 0;
+        for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+            const BwTile ti = bw_decode<MODE>(tile, s_prefix, s_off, N, ntm, ntn);
+            const int acc = it & 1;
+            const uint32_t acc_par = (uint32_t)((it >> 1) & 1);
+            const bool got = wait_bar(smem_u32(&tfull_bar[acc]), acc_par, w);
+            if (!__all_sync(0xffffffffu, got)) break;
+            tc_fence_after();
+            const uint32_t tbase = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BW_BN);
+            const bool empty_k = MODE == BW_WGT && ti.k_rows == 0;
+#pragma unroll 1
+            for (int c = 0; c < BW_BN / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld32(tbase + c * 32, v);
+                tmem_wait_ld();
+                const int col0 = ti.n0 + c * 32;
+                if (MODE == BW_WGT) {
+                    const int m = ti.m0 + r_in;
+                    if (m < p.m_dim) {
+                        float* dst = p.out + ((int64_t)ti.e * p.m_dim + m) * p.n_dim + col0;
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            if (col0 + j < p.n_dim) {
+                                float4 o = empty_k ? make_float4(0.f, 0.f, 0.f, 0.f)
+                                                   : make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
+                                                                 __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
+                                *reinterpret_cast<float4*>(dst + j) = o;
+                            }
+                        }
+                    }
+                    continue;
+                }
+                if (r_in >= ti.rows) continue;
+                const int64_t r = (int64_t)ti.row0 + r_in;
+                if constexpr (MODE == BW_DX) {
+                    const int64_t orow = p.row_token ? (int64_t)p.row_token[r] : r;
+                    float* dst = p.out + orow * p.n_dim + col0;
+#pragma unroll
+                    for (int j = 0; j < 32; j += 4)
+                        if (col0 + j < p.n_dim)
+                            *reinterpret_cast<float4*>(dst + j) =
+                                make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
+                                            __uint_as_float(v[j + 3]));
+                } else {
+                // dU from dA = the accumulator
+#pragma unroll
+                for (int j0 = 0; j0 < 32; j0 += 8) {
+                    const int col = col0 + j0;
+                    if (col >= p.n_dim) break;
+                    uint32_t pk[4], pk2[4];
+                    if (MODE == BW_DU_RELU) {
+                        const uint4 hv = *reinterpret_cast<const uint4*>(p.h + r * p.n_dim + col);
+                        const uint32_t* hw = reinterpret_cast<const uint32_t*>(&hv);
+#pragma unroll
+                        for (int h2 = 0; h2 < 4; ++h2) {
+                            const float a0 = bf16lo(hw[h2]) > 0.f ? __uint_as_float(v[j0 + 2 * h2]) : 0.f;
+                            const float a1 = bf16hi(hw[h2]) > 0.f ? __uint_as_float(v[j0 + 2 * h2 + 1]) : 0.f;
+                            pk[h2] = pack_bf16x2(a0, a1);
+                        }
+                        *reinterpret_cast<uint4*>(p.du + r * p.n_dim + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                    } else {
+                        const __nv_bfloat16* pre = p.pre + r * (int64_t)(2 * p.n_dim);
+                        const uint4 gv = *reinterpret_cast<const uint4*>(pre + col);
+                        const uint4 uv = *reinterpret_cast<const uint4*>(pre + p.n_dim + col);
+                        const uint32_t* gw = reinterpret_cast<const uint32_t*>(&gv);
+                        const uint32_t* uw = reinterpret_cast<const uint32_t*>(&uv);
+#pragma unroll
+                        for (int h2 = 0; h2 < 4; ++h2) {
+                            float dgo[2], duo[2];
+#pragma unroll
+                            for (int z = 0; z < 2; ++z) {
+                                const float g = z ? bf16hi(gw[h2]) : bf16lo(gw[h2]);
+                                const float up = z ? bf16hi(uw[h2]) : bf16lo(uw[h2]);
+                                const float da = __uint_as_float(v[j0 + 2 * h2 + z]);
+                                const float sg = sigmoidf_(g);
+                                dgo[z] = da * up * (sg * (1.f + g * (1.f - sg)));   // silu'(g) = s (1 + g (1 - s))
+                                duo[z] = da * (g * sg);                              // silu(g)
+                            }
+                            pk[h2] = pack_bf16x2(dgo[0], dgo[1]);
+                            pk2[h2] = pack_bf16x2(duo[0], duo[1]);
+                        }
+                        __nv_bfloat16* o = p.du + r * (int64_t)(2 * p.n_dim);
+                        *reinterpret_cast<uint4*>(o + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+                        *reinterpret_cast<uint4*>(o + p.n_dim + col) = make_uint4(pk2[0], pk2[1], pk2[2], pk2[3]);
+                    }
+                }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive_relaxed(smem_u32(&tempty_bar[acc]));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem_base, BW_TMEM_COLS);
+}
+
+// dY[r] = bf16(row_gate[r] * dout[row_token[r]]): one warp per compact row.
+__global__ void __launch_bounds__(256)
+dy_gather_kernel(const __nv_bfloat16* __restrict__ dout, const int32_t* __restrict__ offsets, int N,
+                 const int32_t* __restrict__ row_token, const float* __restrict__ row_gate, int d,
+                 __nv_bfloat16* __restrict__ dy) {
+    pdl_wait();
+    pdl_launch();
+    const int lane = threadIdx.x & 31;
+    const int64_t r = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (r >= offsets[N]) return;
+    const float g = row_gate[r];
+    const __nv_bfloat16* src = dout + (int64_t)row_token[r] * d;
+    __nv_bfloat16* dst = dy + r * d;
+    for (int c = lane * 8; c < d; c += 256) {
+        const uint4 v = *reinterpret_cast<const uint4*>(src + c);
+        const uint32_t* wv = reinterpret_cast<const uint32_t*>(&v);
+        uint32_t o[4];
+#pragma unroll
+        for (int h = 0; h < 4; ++h) o[h] = pack_bf16x2(g * bf16lo(wv[h]), g * bf16hi(wv[h]));
+        *reinterpret_cast<uint4*>(dst + c) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
+// out[e][c] = sum over expert e's rows of src[r][col_off + c] (fp32, rows in
+// order): the bias gradients.  One thread per (expert, column).
+__global__ void __launch_bounds__(256)
+col_sum_kernel(const __nv_bfloat16* __restrict__ src, int64_t ld, int col_off, int width,
+               const int32_t* __restrict__ offsets, int N, float* __restrict__ out) {
+    pdl_wait();
+    pdl_launch();
+    const int c = blockIdx.x * blockDim.x + threadIdx.x;
+    const int e = blockIdx.y;
+    if (c >= width || e >= N) return;
+    float acc = 0.f;
+    for (int64_t r = offsets[e]; r < offsets[e + 1]; ++r) acc += __bfloat162float(src[r * ld + col_off + c]);
+    out[(int64_t)e * width + c] = acc;
+}
+
+// top-2 (or fp32 row output): dx[t] = sum over kept r of dxe[offsets[idx] + pos]
+// (fp32, rank order); zero when every assignment of t was dropped.
+__global__ void __launch_bounds__(256)
+dx_combine_kernel(const float* __restrict__ dxe, const int32_t* __restrict__ idx, const int32_t* __restrict__ pos,
+                  const uint8_t* __restrict__ drop, const int32_t* __restrict__ offsets, int64_t T, int d, int k,
+                  float* __restrict__ dx) {
+    pdl_wait();
+    pdl_launch();
+    const int lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (t >= T) return;
+    int64_t row[2] = {-1, -1};
+    for (int r = 0; r < k; ++r)
+        if (!drop[t * k + r]) row[r] = (int64_t)offsets[idx[t * k + r]] + pos[t * k + r];
+    for (int c = lane; c < d; c += 32) {
+        float acc = 0.f;
+        for (int r = 0; r < k; ++r)
+            if (row[r] >= 0) acc += dxe[row[r] * d + c];
+        dx[t * d + c] = acc;
+    }
+}
+
+// rows of dropped tokens (top-1 scatter path): dx[t] = 0
+__global__ void __launch_bounds__(256)
+dx_zero_dropped_kernel(const uint8_t* __restrict__ drop, int64_t T, int d, float* __restrict__ dx) {
+    pdl_wait();
+    pdl_launch();
+    const int lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (t >= T || !drop[t]) return;
+    for (int c = lane; c < d; c += 32) dx[t * d + c] = 0.f;
+}
+
+template <int MODE>
+cudaError_t run_bwd(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const BwdParams& p,
+                    cudaStream_t s) {
+    int sms = 0;
+    cudaError_t err = device_sm_count(&sms);
+    if (err != cudaSuccess) return err;
+    err = once_per_device(reinterpret_cast<const void*>(bwd_gemm_kernel<MODE>), [](const void* k) {
+        return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, BW_SMEM);
+    });
+    if (err != cudaSuccess) return err;
+    return launch_k(bwd_gemm_kernel<MODE>, dim3((unsigned)sms), dim3(BW_THREADS), BW_SMEM, s, 1, a, b, b2, p);
+}
+
+}  // namespace
+
+cudaError_t launch_expert_backward_tc(const BwdArgs& a, cudaStream_t s) {
+    const int64_t R = a.R_cap > 0 ? a.R_cap : 1;
+    const bool sw = a.act == MOE_SWIGLU;
+    const int d = a.d, dff = a.d_ff, N = a.N;
+    cudaError_t err;
+    // 1. the forward's first GEMM again: H (and the SwiGLU pre-activations)
+    FfnArgs f{};
+    f.dtype = MOE_BF16;
+    f.act = a.act;
+    f.N = N;
+    f.d = d;
+    f.d_ff = dff;
+    f.R_cap = a.R_cap;
+    f.xe = a.xe;
+    f.offsets = a.offsets;
+    f.w1 = a.w1;
+    f.b1 = a.b1;
+    f.w3 = a.w3;
+    f.b3 = a.b3;
+    f.h = a.h;
+    f.pre_out = sw ? a.pre : nullptr;
+    f.stage1_only = true;
+    f.hdr = a.hdr;
+    if ((err = launch_expert_ffn_tc(f, s)) != cudaSuccess) return err;
+    // 2. dY = gate * dout[token]
+    const unsigned rows_grid = (unsigned)((R + 7) / 8);
+    if ((err = launch_k(dy_gather_kernel, dim3(rows_grid), dim3(256), 0, s, 1,
+                        reinterpret_cast<const __nv_bfloat16*>(a.dout), a.offsets, N, a.row_token, a.row_gate, d,
+                        reinterpret_cast<__nv_bfloat16*>(a.dy))) != cudaSuccess)
+        return err;
+    CUtensorMap m_dy, m_w2, m_du, m_w1, m_w3, m_xe, m_h, m_a2, m_b2;
+    // 3. dA = dY W2 -> dU (dG | dUp)
+    if (!make_map_bf16(&m_dy, a.dy, R, d, BW_BM) || !make_map_bf16_mn(&m_w2, a.w2, (int64_t)N * d, dff, BW_BK))
+        return cudaErrorInvalidValue;
+    BwdParams p{};
+    p.offsets = a.offsets;
+    p.N = N;
+    p.status = &a.hdr->status;
+    p.limit_ns = kWaitLimitNs;
+    p.n_dim = dff;
+    p.k_dim = d;
+    p.h = reinterpret_cast<const __nv_bfloat16*>(a.h);
+    p.pre = reinterpret_cast<const __nv_bfloat16*>(a.pre);
+    p.du = reinterpret_cast<__nv_bfloat16*>(a.du);
+    err = sw ? run_bwd<BW_DU_SWIGLU>(m_dy, m_w2, m_w2, p, s) : run_bwd<BW_DU_RELU>(m_dy, m_w2, m_w2, p, s);
+    if (err != cudaSuccess) return err;
+    // 4. dx rows = dU W1 (+ dUp W3): K = d_ff (2 d_ff for SwiGLU, W3 for the second half)
+    const int kdu = sw ? 2 * dff : dff;
+    if (!make_map_bf16(&m_du, a.du, R, kdu, BW_BM) || !make_map_bf16_mn(&m_w1, a.w1, (int64_t)N * dff, d, BW_BK))
+        return cudaErrorInvalidValue;
+    if (sw && !make_map_bf16_mn(&m_w3, a.w3, (int64_t)N * dff, d, BW_BK)) return cudaErrorInvalidValue;
+    BwdParams px = p;
+    px.n_dim = d;
+    px.k_dim = kdu;
+    px.k_split = sw ? dff : 0;
+    px.out = a.top1_scatter ? a.dx : a.dxe;
+    px.row_token = a.top1_scatter ? a.row_token : nullptr;
+    if ((err = run_bwd<BW_DX>(m_du, m_w1, sw ? m_w3 : m_w1, px, s)) != cudaSuccess) return err;
+    if (a.top1_scatter) {
+        if (a.T > 0 && (err = launch_k(dx_zero_dropped_kernel, dim3((unsigned)((a.T + 7) / 8)), dim3(256), 0, s, 1,
+                                       a.drop, a.T, d, a.dx)) != cudaSuccess)
+            return err;
+    } else if (a.T > 0) {
+        if ((err = launch_k(dx_combine_kernel, dim3((unsigned)((a.T + 7) / 8)), dim3(256), 0, s, 1,
+                            static_cast<const float*>(a.dxe), a.idx, a.pos, a.drop, a.offsets, a.T, d, a.k,
+                            a.dx)) != cudaSuccess)
+            return err;
+    }
+    // 5. weight gradients: dW1 = dU^T X (dW3 = dUp^T X), dW2 = dY^T A
+    if (!make_map_bf16_mn(&m_xe, a.xe, R, d, BW_BK) || !make_map_bf16_mn(&m_h, a.h, R, dff, BW_BK))
+        return cudaErrorInvalidValue;
+    BwdParams pw = p;
+    pw.m_dim = dff;
+    pw.n_dim = d;
+    // dU (dG): the first d_ff columns of each row of the du tensor (row stride kdu)
+    if (!make_map_bf16_strided(&m_a2, a.du, R, dff, kdu, BW_BK)) return cudaErrorInvalidValue;
+    pw.out = a.dw1;
+    if (a.dw1 && (err = run_bwd<BW_WGT>(m_a2, m_xe, m_xe, pw, s)) != cudaSuccess) return err;
+    if (sw && a.dw3) {   // dUp: columns [d_ff, 2 d_ff)
+        if (!make_map_bf16_strided(&m_b2, reinterpret_cast<const __nv_bfloat16*>(a.du) + dff, R, dff, kdu, BW_BK))
+            return cudaErrorInvalidValue;
+        pw.out = a.dw3;
+        if ((err = run_bwd<BW_WGT>(m_b2, m_xe, m_xe, pw, s)) != cudaSuccess) return err;
+    }
+    if (a.dw2) {
+        CUtensorMap m_dy_mn;
+        if (!make_map_bf16_mn(&m_dy_mn, a.dy, R, d, BW_BK)) return cudaErrorInvalidValue;
+        BwdParams p2 = p;
+        p2.m_dim = d;
+        p2.n_dim = dff;
+        p2.out = a.dw2;
+        if ((err = run_bwd<BW_WGT>(m_dy_mn, m_h, m_h, p2, s)) != cudaSuccess) return err;
+    }
+    // 6. bias gradients
+    const dim3 cs_block(256);
+    if (a.db1 && (err = launch_k(col_sum_kernel, dim3((unsigned)((dff + 255) / 256), (unsigned)N), cs_block, 0, s, 1,
+                                 static_cast<const __nv_bfloat16*>(a.du), (int64_t)kdu, 0, dff, a.offsets, N,
+                                 a.db1)) != cudaSuccess)
+        return err;
+    if (sw && a.db3 && (err = launch_k(col_sum_kernel, dim3((unsigned)((dff + 255) / 256), (unsigned)N), cs_block, 0, s,
+                                       1, static_cast<const __nv_bfloat16*>(a.du), (int64_t)kdu, dff, dff, a.offsets,
+                                       N, a.db3)) != cudaSuccess)
+        return err;
+    if (a.db2 && (err = launch_k(col_sum_kernel, dim3((unsigned)((d + 255) / 256), (unsigned)N), cs_block, 0, s, 1,
+                                 static_cast<const __nv_bfloat16*>(a.dy), (int64_t)d, 0, d, a.offsets, N, a.db2)) !=
+                     cudaSuccess)
+        return err;
+    return cudaSuccess;
+}
+
+}  // namespace moe

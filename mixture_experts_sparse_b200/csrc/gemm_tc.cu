@@ -87,6 +87,7 @@ struct GemmParams {
     const float* row_gate;        // scatter: nullable (no gate)
     void* const* out_ptrs;        // scatter to several GPUs: row r goes to out_ptrs[row_rank[r]]
     const int32_t* row_rank;
+    __nv_bfloat16* pre_out;       // SwiGLU (optional): the pre-activations W1 x + b1 | W3 x + b3, [R, 2 n_dim]
     int32_t* status;
     long long limit_ns;
 };
@@ -402,11 +403,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         }
                     }
                     uint32_t pk[4];
+                    uint32_t pre_g[4], pre_u[4];
 #pragma unroll
                     for (int h = 0; h < 4; ++h) {
                         const int j = 8 * gi + 2 * h;
                         float a0 = __uint_as_float(u[j]) + bu[2 * h];
                         float a1 = __uint_as_float(u[j + 1]) + bu[2 * h + 1];
+                        if (EPI == EPI_SWIGLU) {
+                            pre_g[h] = pack_bf16x2(a0, a1);
+                            pre_u[h] = pack_bf16x2(__uint_as_float(v[EPI == EPI_SWIGLU ? j : 0]) + bv[2 * h],
+                                                   __uint_as_float(v[EPI == EPI_SWIGLU ? j + 1 : 0]) + bv[2 * h + 1]);
+                        }
                         if (EPI == EPI_RELU) {
                             a0 = fmaxf(a0, 0.f);
                             a1 = fmaxf(a1, 0.f);
@@ -418,6 +425,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                             a1 *= g;
                         }
                         pk[h] = pack_bf16x2(a0, a1);
+                    }
+                    if (EPI == EPI_SWIGLU && p.pre_out != nullptr && valid && col < p.n_dim) {
+                        __nv_bfloat16* pr = p.pre_out + grow * (int64_t)(2 * p.n_dim) + col;
+                        *reinterpret_cast<uint4*>(pr) = make_uint4(pre_g[0], pre_g[1], pre_g[2], pre_g[3]);
+                        *reinterpret_cast<uint4*>(pr + p.n_dim) = make_uint4(pre_u[0], pre_u[1], pre_u[2], pre_u[3]);
                     }
                     const uint32_t dst = ebuf + lane * 128 + ((gi ^ (lane & 7)) << 4);
                     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pk[0]), "r"(pk[1]),
@@ -536,16 +548,29 @@ EncodeFn get_encode() {
 
 // 2-D bf16 tensor [rows, k] (k contiguous), box = box_rows x 64, 128-byte swizzle.
 bool tc::make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t k, int box_rows) {
+    return make_map_bf16_strided(map, base, rows, k, k, box_rows);
+}
+
+// The first `cols` columns of rows `row_stride` elements apart.
+bool tc::make_map_bf16_strided(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t row_stride,
+                               int box_rows) {
     EncodeFn enc = get_encode();
     if (!enc) return false;
+    const int64_t k = cols;
     cuuint64_t dims[2] = {(cuuint64_t)k, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)k * 2};
+    cuuint64_t strides[1] = {(cuuint64_t)row_stride * 2};
     cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
     cuuint32_t estr[2] = {1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+// 2-D bf16 tensor [rows, cols] (cols contiguous) as an MN-major operand:
+// box = 64 cols x box_rows rows, 128-byte swizzle.
+bool tc::make_map_bf16_mn(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows) {
+    return make_map_bf16(map, base, rows, cols, box_rows);   // the same box shape: 64 inner elements x rows
 }
 
 // Stage 1 + stage 2 of the bf16 expert FFN on the tensor cores, both
@@ -559,7 +584,8 @@ cudaError_t launch_expert_ffn_tc(const FfnArgs& a, cudaStream_t s) {
     const int b2_box = pair ? BN / 2 : BN;
     CUtensorMap mA1, mB1, mB3, mA2, mB2;
     if (!make_map_bf16(&mA1, a.xe, R, a.d, BM) || !make_map_bf16(&mB1, a.w1, (int64_t)a.N * a.d_ff, a.d, b1_box) ||
-        !make_map_bf16(&mA2, a.h, R, a.d_ff, BM) || !make_map_bf16(&mB2, a.w2, (int64_t)a.N * a.d, a.d_ff, b2_box))
+        !make_map_bf16(&mA2, a.h, R, a.d_ff, BM) ||
+        (!a.stage1_only && !make_map_bf16(&mB2, a.w2, (int64_t)a.N * a.d, a.d_ff, b2_box)))
         return cudaErrorInvalidValue;
     if (swiglu) {
         if (!make_map_bf16(&mB3, a.w3, (int64_t)a.N * a.d_ff, a.d, b1_box)) return cudaErrorInvalidValue;
@@ -577,9 +603,10 @@ cudaError_t launch_expert_ffn_tc(const FfnArgs& a, cudaStream_t s) {
     p1.out = reinterpret_cast<__nv_bfloat16*>(a.h);
     p1.status = &a.hdr->status;
     p1.limit_ns = kWaitLimitNs;
+    p1.pre_out = reinterpret_cast<__nv_bfloat16*>(a.pre_out);
     cudaError_t err = swiglu ? run_gemm_any<EPI_SWIGLU>(mA1, mB1, mB3, p1, s)
                              : run_gemm_any<EPI_RELU>(mA1, mB1, mB3, p1, s);
-    if (err != cudaSuccess) return err;
+    if (err != cudaSuccess || a.stage1_only) return err;
     if (a.mid_event && (err = cudaEventRecord((cudaEvent_t)a.mid_event, s)) != cudaSuccess) return err;
 
     GemmParams p2{};

@@ -32,9 +32,10 @@
 // issuer (the leader's), warps 2-5 epilogue with one thread per token of its
 // own CTA: the thread holds its token's NP logits (tcgen05.ld), computes max,
 // softmax, top-1/top-2 and the gate in registers, and writes idx/gate (and
-// probs).  Per-tile partial sums of p and top-1
-// counts are reduced in a fixed order (lanes in a warp through shared memory,
-// then the four warps in quadrant order), so the aux loss is deterministic.
+// probs).  Per-tile sums of p are reduced across each warp's lanes with a
+// fixed shuffle tree that leaves every lane the sums of NP/32 experts (kept in
+// registers over the CTA's tiles), then over the four warps in a fixed order,
+// so the aux loss is deterministic and no shared memory holds per-token sums.
 #include "tc_common.cuh"
 
 namespace moe {
@@ -50,12 +51,9 @@ struct RtShape {
     static constexpr int A_BYTES = RT_BM * RT_BK * 2;
     static constexpr int P_BYTES = (NP / 2) * RT_BK * 2;       // this CTA's half of one W part
     static constexpr int STAGE_BYTES = A_BYTES + 3 * P_BYTES;
-    static constexpr int STAGES = NP <= 64 ? 6 : 3;
-    // per epilogue thread, a row of running sums of p over its tokens (padded
-    // by one float so the rows of a warp fall in different banks)
-    static constexpr int ACC_STRIDE = NP + 1;
-    static constexpr int ACC_BYTES = 4 * 32 * ACC_STRIDE * 4;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + ACC_BYTES;
+    // as many stages as fit (the router is bound by the x bytes in flight)
+    static constexpr int STAGES = (200 * 1024) / STAGE_BYTES < 12 ? (200 * 1024) / STAGE_BYTES : 12;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
     // merged: one MMA of N = 3 NP covers the three W parts and leaves three
     // partial-logit blocks side by side in TMEM; the pair's leader holds W rows
     // [0, 3 NP / 2) of the stacked parts, the peer rows [3 NP / 2, 3 NP).
@@ -67,7 +65,36 @@ struct RtShape {
     static constexpr int MMA_PER_KB = MERGED ? RT_BK / 16 : 3 * (RT_BK / 16);
     static constexpr int KB_PER_GROUP = 64 / MMA_PER_KB;       // <= 64 MMAs per accumulator
     static_assert(STAGE_BYTES % 1024 == 0, "1024-byte aligned stages");
+    static constexpr int PER_LANE = NP / 32;   // experts whose warp sums of p a lane keeps
 };
+
+// Warp transpose-reduce: every lane holds NP values; after log2(32) halving
+// steps (partner = lane ^ 16, 8, 4, 2, 1; the lower-bit lane keeps the lower
+// half and adds the partner's copy of it) lane l holds the sums over the 32
+// lanes of experts [l NP / 32, (l + 1) NP / 32), in a fixed order.
+template <int NP>
+__device__ __forceinline__ void warp_transpose_sum(float (&v)[NP], int lane, float (&out)[NP / 32]) {
+    float a[NP / 2];
+#pragma unroll
+    for (int j = 0; j < NP / 2; ++j) {
+        const bool hi = lane & 16;
+        const float send = hi ? v[j] : v[j + NP / 2];
+        const float keep = hi ? v[j + NP / 2] : v[j];
+        a[j] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+#pragma unroll
+    for (int o = 8, w = NP / 4; o >= 1; o >>= 1, w >>= 1) {
+#pragma unroll
+        for (int j = 0; j < w; ++j) {
+            const bool hi = lane & o;
+            const float send = hi ? a[j] : a[j + w];
+            const float keep = hi ? a[j + w] : a[j];
+            a[j] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < NP / 32; ++j) out[j] = a[j];
+}
 
 struct RtParams {
     int64_t T;
@@ -141,7 +168,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     constexpr uint32_t IDESC = idesc_bf16_f32(2 * RT_BM, S::ACC_COLS);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-    float* pacc = reinterpret_cast<float*>(smem + S::STAGES * S::STAGE_BYTES);   // [4][32][NP + 1]
+    __shared__ float s_wsum[4][NP];    // per epilogue warp: sums of p over its tokens
     __shared__ __align__(8) uint64_t full_bar[S::STAGES];
     __shared__ __align__(8) uint64_t empty_bar[S::STAGES];
     __shared__ __align__(8) uint64_t tfull_bar[2];
@@ -173,7 +200,6 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         mbar_fence_init();
     }
     for (int e = tid; e < NP; e += RT_THREADS) s_hist[e] = 0;
-    for (int i = tid; i < 4 * 32 * S::ACC_STRIDE; i += RT_THREADS) pacc[i] = 0.f;
     if (warp == 0 && lane == 0) {
         prefetch_tmap(&tmX);
         prefetch_tmap(&tmW);
@@ -292,7 +318,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     } else {
         // ---------------- epilogue: one thread per token ----------------
         const int q = warp & 3;
-        float* prow = pacc + (q * 32 + lane) * S::ACC_STRIDE;   // this thread's running sums
+        float psum[S::PER_LANE];   // this warp's sums of p over its tokens, experts [lane NP/32, ...)
+#pragma unroll
+        for (int j = 0; j < S::PER_LANE; ++j) psum[j] = 0.f;
         const int N = p.N, k = p.k;
         const uint32_t tempty_leader0 = map_to_rank(smem_u32(&tempty_bar[0]), 0);
         const uint32_t tempty_leader1 = map_to_rank(smem_u32(&tempty_bar[1]), 0);
@@ -368,8 +396,14 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 atomicAdd(&s_hist[i1], 1);
             }
 #pragma unroll
-            for (int e = 0; e < NP; ++e) prow[e] += v[e] * inv;   // this thread's tokens, in tile order
+            for (int e = 0; e < NP; ++e) v[e] *= inv;   // p (0 for a token past T)
+            float ts[S::PER_LANE];
+            warp_transpose_sum<NP>(v, lane, ts);
+#pragma unroll
+            for (int j = 0; j < S::PER_LANE; ++j) psum[j] += ts[j];   // tiles in order
         }
+#pragma unroll
+        for (int j = 0; j < S::PER_LANE; ++j) s_wsum[q][lane * S::PER_LANE + j] = psum[j];
         // ---- this CTA's partials, expert-major: part[e][blockIdx.x] ----
         const int et = tid - 64;   // 0..127 across the four epilogue warps
         s_z[et] = zacc;
@@ -381,14 +415,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
         }
         const int Gp = ((int)gridDim.x + 3) & ~3;
         if (et < N) {
-            float ps = 0.f;   // fixed order: warp quadrant, then lane
-            for (int r = 0; r < 128; r += 8) {
-                float pv[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) pv[j] = pacc[(r + j) * S::ACC_STRIDE + et];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) ps += pv[j];
-            }
+            const float ps = (s_wsum[0][et] + s_wsum[1][et]) + (s_wsum[2][et] + s_wsum[3][et]);   // fixed order
             p.part_psum[(int64_t)et * Gp + blockIdx.x] = ps;
             p.part_cnt[(int64_t)et * Gp + blockIdx.x] = s_hist[et];
             __threadfence();

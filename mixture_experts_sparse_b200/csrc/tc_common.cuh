@@ -85,6 +85,16 @@ __device__ __forceinline__ uint64_t umma_desc(uint32_t addr) {
            ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
 }
 
+// Shared-memory matrix descriptor for an MN-major operand with 128-byte
+// swizzle: each K row holds 64 consecutive MN elements (128 B), 8 K rows form a
+// 1024-byte swizzle atom (SBO = 1024 between 8-row K groups), and the next 64
+// MN elements start `mn_stride` bytes later (LBO).  A TMA box of 64 MN x K rows
+// (inner dimension MN) lands in exactly this layout.
+__device__ __forceinline__ uint64_t umma_desc_mn(uint32_t addr, uint32_t mn_stride) {
+    return (uint64_t)((addr & 0x3FFFFu) >> 4) | ((uint64_t)((mn_stride >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)(1024 >> 4) << 32) | ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
 __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
@@ -151,6 +161,10 @@ __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+// ... with A (bit 15) and / or B (bit 16) read MN-major instead of K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16_f32_major(int M, int N, bool a_mn, bool b_mn) {
+    return idesc_bf16_f32(M, N) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16);
+}
 
 __device__ __forceinline__ void tmem_alloc(uint32_t* slot, uint32_t ncols) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(slot)),
@@ -175,6 +189,12 @@ __device__ __forceinline__ void named_bar(int id, int count) {
 
 // host: 2-D bf16 tensor [rows, k] (k contiguous), box = box_rows x 64, 128-byte swizzle
 bool make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t k, int box_rows);
+// host: 2-D bf16 tensor [rows, cols] (cols contiguous) read as an MN-major
+// operand: box = 64 cols x box_rows rows, 128-byte swizzle
+bool make_map_bf16_mn(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows);
+// host: the same over the first `cols` columns of rows `row_stride` elements apart
+bool make_map_bf16_strided(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t row_stride,
+                           int box_rows);
 
 }  // namespace tc
 }  // namespace moe

@@ -62,6 +62,8 @@ _SIGS = {
     "moe_ep_dispatch": ([ctypes.POINTER(MoeConfig), ctypes.c_int32, ctypes.c_int32] + [_P] * 12, ctypes.c_int32),
     "moe_ep_expert_ffn": ([ctypes.POINTER(MoeConfig), ctypes.c_int32] + [_P] * 13 + [ctypes.c_size_t, _P],
                           ctypes.c_int32),
+    "moe_expert_backward_workspace_bytes": ([ctypes.POINTER(MoeConfig)], ctypes.c_size_t),
+    "moe_expert_backward": ([ctypes.POINTER(MoeConfig)] + [_P] * 21 + [ctypes.c_size_t, _P], ctypes.c_int32),
     "moe_read_device_status": ([_P, _P], ctypes.c_int32),
     "moe_test_lookback_timeout": ([_P, ctypes.c_size_t, ctypes.c_int64, _P], ctypes.c_int32),
 }
@@ -281,3 +283,15 @@ def moe_ep_expert_ffn(cfg, n_ranks, recv_x, recv_offsets, w1, b1, w3, b3, w2, b2
     return lib().moe_ep_expert_ffn(ctypes.byref(cfg), int(n_ranks), _p(recv_x), _p(recv_offsets), _p(w1), _p(b1),
                                    _p(w3), _p(b3), _p(w2), _p(b2), _p(recv_rank), _p(recv_row), _p(recv_gate),
                                    _p(out_ptrs), _p(ws), _nbytes(ws), _s(stream))
+
+
+def moe_expert_backward_workspace_bytes(cfg):
+    return int(lib().moe_expert_backward_workspace_bytes(ctypes.byref(cfg)))
+
+
+def moe_expert_backward(cfg, xe, offsets, row_token, row_gate, idx, pos, drop, dout, w1, b1, w3, b3, w2, dx, dw1,
+                        db1, dw3, db3, dw2, db2, ws, stream=None):
+    return lib().moe_expert_backward(ctypes.byref(cfg), _p(xe), _p(offsets), _p(row_token), _p(row_gate), _p(idx),
+                                     _p(pos), _p(drop), _p(dout), _p(w1), _p(b1), _p(w3), _p(b3), _p(w2), _p(dx),
+                                     _p(dw1), _p(db1), _p(dw3), _p(db3), _p(dw2), _p(db2), _p(ws), _nbytes(ws),
+                                     _s(stream))
