@@ -12,7 +12,6 @@
 
 namespace moe {
 
-cudaError_t launch_expert_ffn_tc(const FfnArgs& a, cudaStream_t s);
 
 namespace {
 
@@ -45,16 +44,32 @@ simt_gemm_kernel(const float* __restrict__ A, const int32_t* __restrict__ offset
     const int tx = tid % 16, ty = tid / 16;
     float acc[4][4] = {};
     float acc3[4][4] = {};
+    // the next K chunk is loaded into registers while the current one is used
+    constexpr int PER = TS * KC / 256;
+    float pa[PER], pb[PER], pb3[PER];
+    auto fetch = [&](int k0) {
+#pragma unroll
+        for (int l = 0; l < PER; ++l) {
+            const int q = tid + 256 * l;
+            const int rr = q / KC, kk = q % KC;
+            const int m = m0 + rr, kx = k0 + kk, n = n0 + rr;
+            pa[l] = (m < rows && kx < K) ? A[(int64_t)(row0 + m) * K + kx] : 0.f;
+            pb[l] = (n < n_dim && kx < K) ? Be[(int64_t)n * K + kx] : 0.f;
+            if (MODE == SIMT_SWIGLU) pb3[l] = (n < n_dim && kx < K) ? B3e[(int64_t)n * K + kx] : 0.f;
+        }
+    };
+    fetch(0);
     for (int k0 = 0; k0 < K; k0 += KC) {
-        for (int q = tid; q < TS * KC; q += 256) {
-            int rr = q / KC, kk = q % KC;
-            int m = m0 + rr, kx = k0 + kk;
-            As[kk][rr] = (m < rows && kx < K) ? A[(int64_t)(row0 + m) * K + kx] : 0.f;
-            int n = n0 + rr;
-            Bs[kk][rr] = (n < n_dim && kx < K) ? Be[(int64_t)n * K + kx] : 0.f;
-            if (MODE == SIMT_SWIGLU) B3s[kk][rr] = (n < n_dim && kx < K) ? B3e[(int64_t)n * K + kx] : 0.f;
+#pragma unroll
+        for (int l = 0; l < PER; ++l) {
+            const int q = tid + 256 * l;
+            const int rr = q / KC, kk = q % KC;
+            As[kk][rr] = pa[l];
+            Bs[kk][rr] = pb[l];
+            if (MODE == SIMT_SWIGLU) B3s[kk][rr] = pb3[l];
         }
         __syncthreads();
+        if (k0 + KC < K) fetch(k0 + KC);
 #pragma unroll
         for (int kk = 0; kk < KC; ++kk) {
             float a[4], b[4], b3[4];

@@ -337,9 +337,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const TileInfo ti = decode_tile<S::TILE_M>(tile, s_prefix, s_off, N, ntn, BN_OUT);
             const int acc = it & 1;
             const uint32_t acc_par = (uint32_t)((it >> 1) & 1);
-            const bool got = wait_bar(smem_u32(&tfull_bar[acc]), acc_par, w);
-            if (!__all_sync(0xffffffffu, got)) break;   // warp-uniform exit on abort
-            tc_fence_after();
+            // the row's destination (and, scattering, its token and gate) are
+            // fetched before the accumulator is waited for
             const bool valid = r_in_tile < ti.rows;
             const int64_t grow = (int64_t)ti.row0 + r_in_tile;
             int64_t orow = grow;
@@ -363,26 +362,22 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 dst_row[k4] = reinterpret_cast<__nv_bfloat16*>(
                     __shfl_sync(0xffffffffu, reinterpret_cast<unsigned long long>(my_dst), r));
             }
-#pragma unroll 1
-            for (int c = 0; c < BN_OUT / CW; ++c) {
+            const bool got = wait_bar(smem_u32(&tfull_bar[acc]), acc_par, w);
+            if (!__all_sync(0xffffffffu, got)) break;   // warp-uniform exit on abort
+            tc_fence_after();
+
+            // one chunk of CW output columns from the accumulator values u (and v):
+            // bias / activation / gate, bf16 pack, staged rows, 128-byte row stores
+            auto emit = [&](int c, const uint32_t (&u)[CW], const uint32_t (&v)[EPI == EPI_SWIGLU ? CW : 1]) {
                 const int col0 = ti.n0 + c * CW;
-                uint32_t u[CW];
-                uint32_t v[EPI == EPI_SWIGLU ? CW : 1];
-                tmem_ld32(tbase + c * CW, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
-                tmem_ld32(tbase + c * CW + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
-                if (EPI == EPI_SWIGLU) {
-                    tmem_ld32(tbase + BN_OUT + c * CW, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
-                    tmem_ld32(tbase + BN_OUT + c * CW + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[EPI == EPI_SWIGLU ? 32 : 0]));
-                }
-                tmem_wait_ld();
 #pragma unroll
                 for (int gi = 0; gi < CW / 8; ++gi) {   // one 16-byte granule = 8 columns
                     const int col = col0 + 8 * gi;
                     float bu[8], bv[8];
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) {
-                        bu[j] = 0.f;
-                        bv[j] = 0.f;
+                    for (int jj = 0; jj < 8; ++jj) {
+                        bu[jj] = 0.f;
+                        bv[jj] = 0.f;
                     }
                     if (bias_e && col < p.n_dim) {
                         uint4 bw = __ldg(reinterpret_cast<const uint4*>(bias_e + col));
@@ -406,20 +401,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     uint32_t pre_g[4], pre_u[4];
 #pragma unroll
                     for (int h = 0; h < 4; ++h) {
-                        const int j = 8 * gi + 2 * h;
-                        float a0 = __uint_as_float(u[j]) + bu[2 * h];
-                        float a1 = __uint_as_float(u[j + 1]) + bu[2 * h + 1];
+                        const int jj = 8 * gi + 2 * h;
+                        float a0 = __uint_as_float(u[jj]) + bu[2 * h];
+                        float a1 = __uint_as_float(u[jj + 1]) + bu[2 * h + 1];
                         if (EPI == EPI_SWIGLU) {
                             pre_g[h] = pack_bf16x2(a0, a1);
-                            pre_u[h] = pack_bf16x2(__uint_as_float(v[EPI == EPI_SWIGLU ? j : 0]) + bv[2 * h],
-                                                   __uint_as_float(v[EPI == EPI_SWIGLU ? j + 1 : 0]) + bv[2 * h + 1]);
+                            pre_u[h] = pack_bf16x2(__uint_as_float(v[EPI == EPI_SWIGLU ? jj : 0]) + bv[2 * h],
+                                                   __uint_as_float(v[EPI == EPI_SWIGLU ? jj + 1 : 0]) + bv[2 * h + 1]);
                         }
                         if (EPI == EPI_RELU) {
                             a0 = fmaxf(a0, 0.f);
                             a1 = fmaxf(a1, 0.f);
                         } else if (EPI == EPI_SWIGLU) {
-                            a0 = silu(a0) * (__uint_as_float(v[EPI == EPI_SWIGLU ? j : 0]) + bv[2 * h]);
-                            a1 = silu(a1) * (__uint_as_float(v[EPI == EPI_SWIGLU ? j + 1 : 0]) + bv[2 * h + 1]);
+                            a0 = silu(a0) * (__uint_as_float(v[EPI == EPI_SWIGLU ? jj : 0]) + bv[2 * h]);
+                            a1 = silu(a1) * (__uint_as_float(v[EPI == EPI_SWIGLU ? jj + 1 : 0]) + bv[2 * h + 1]);
                         } else if (EPI == EPI_SCATTER) {
                             a0 *= g;
                             a1 *= g;
@@ -452,10 +447,46 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         *reinterpret_cast<uint4*>(dst_row[k4] + col0 + 8 * gi) = val;
                 }
                 __syncwarp();
+            };
+            auto release = [&]() {   // every TMEM read of this accumulator has completed
+                tc_fence_before();
+                if (PAIR) mbar_arrive_cluster_relaxed(acc ? tempty_leader1 : tempty_leader0);
+                else mbar_arrive_relaxed(smem_u32(&tempty_bar[acc]));
+            };
+            if constexpr (EPI == EPI_SWIGLU) {
+#pragma unroll 1
+                for (int c = 0; c < BN_OUT / CW; ++c) {
+                    uint32_t u[CW], v[CW];
+                    tmem_ld32(tbase + c * CW, *reinterpret_cast<uint32_t(*)[32]>(&u[0]));
+                    tmem_ld32(tbase + c * CW + 32, *reinterpret_cast<uint32_t(*)[32]>(&u[32]));
+                    tmem_ld32(tbase + BN_OUT + c * CW, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+                    tmem_ld32(tbase + BN_OUT + c * CW + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
+                    tmem_wait_ld();
+                    if (c == BN_OUT / CW - 1) release();
+                    emit(c, u, v);
+                }
+            } else {
+                // the next chunk's TMEM load is in flight while this chunk is
+                // processed; the accumulator is released right after its last load
+                constexpr int NC = BN_OUT / CW;
+                uint32_t ua[CW], ub[CW], none[1];
+                tmem_ld32(tbase, *reinterpret_cast<uint32_t(*)[32]>(&ua[0]));
+                tmem_ld32(tbase + 32, *reinterpret_cast<uint32_t(*)[32]>(&ua[32]));
+                tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < NC; ++c) {
+                    uint32_t(&cur)[CW] = (c & 1) ? ub : ua;
+                    uint32_t(&nxt)[CW] = (c & 1) ? ua : ub;
+                    if (c + 1 < NC) {
+                        tmem_ld32(tbase + (c + 1) * CW, *reinterpret_cast<uint32_t(*)[32]>(&nxt[0]));
+                        tmem_ld32(tbase + (c + 1) * CW + 32, *reinterpret_cast<uint32_t(*)[32]>(&nxt[32]));
+                    } else {
+                        release();
+                    }
+                    emit(c, cur, none);
+                    if (c + 1 < NC) tmem_wait_ld();
+                }
             }
-            tc_fence_before();
-            if (PAIR) mbar_arrive_cluster_relaxed(acc ? tempty_leader1 : tempty_leader0);
-            else mbar_arrive_relaxed(smem_u32(&tempty_bar[acc]));
         }
     }
 

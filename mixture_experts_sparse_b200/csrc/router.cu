@@ -160,12 +160,68 @@ router_kernel(const XT* __restrict__ x, const float* __restrict__ w_r, const flo
     }
     __syncthreads();
 
-    // ---- per token: softmax, top-k, gate (one warp per token) ------------------
+    // ---- per token: softmax, top-k, gate ----------------------------------------
     constexpr int MPL = (S::NP + 31) / 32;
     const int64_t rem_t = T - t0;
     const int tb_valid = rem_t < (int64_t)S::TB ? (int)rem_t : S::TB;
-    double zacc = 0.0;   // lane 0: sum over this warp's tokens of log-sum-exp^2
-    for (int tok = warp; tok < tb_valid; tok += kThreads / 32) {
+    double zacc = 0.0;   // sum over this warp's (thread's) tokens of log-sum-exp^2
+    if (S::NP <= 32) {
+        // few experts: one thread per token, its logits in registers (no
+        // shuffle chains; the same arithmetic and order per token as below)
+        for (int tok = tid; tok < tb_valid; tok += kThreads) {
+            float* row = lg + tok * (S::NP + 1);
+            float v[S::NP];
+            float m = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < S::NP; ++e) {
+                v[e] = e < N ? row[e] : -INFINITY;
+                m = fmaxf(m, v[e]);
+            }
+            float ex[S::NP];
+            float s = 0.f;
+#pragma unroll
+            for (int e = 0; e < S::NP; ++e) {
+                ex[e] = e < N ? expf(v[e] - m) : 0.f;
+                s += ex[e];
+            }
+            float bv = -INFINITY, cv = -INFINITY;
+            int bi = 0x7fffffff, ci = 0x7fffffff;
+#pragma unroll
+            for (int e = 0; e < S::NP; ++e)
+                if (e < N) argmax_merge(bv, bi, v[e], e);
+            if (k == 2) {
+#pragma unroll
+                for (int e = 0; e < S::NP; ++e)
+                    if (e < N && e != bi) argmax_merge(cv, ci, v[e], e);
+            }
+            const float inv = 1.f / s;
+            const int64_t t = t0 + tok;
+#pragma unroll
+            for (int e = 0; e < S::NP; ++e) {
+                if (e < N) {
+                    const float pe = ex[e] * inv;
+                    row[e] = pe;
+                    if (probs) probs[t * N + e] = pe;
+                }
+            }
+            const float lse = m + logf(s);
+            zacc += (double)lse * (double)lse;
+            atomicAdd(&s_cnt[bi], 1);
+            if (k == 1) {
+                idx[t] = bi;
+                gate[t] = inv;
+            } else {
+                const float r = expf(cv - bv);
+                idx[2 * t] = bi;
+                idx[2 * t + 1] = ci;
+                gate[2 * t] = 1.f / (1.f + r);
+                gate[2 * t + 1] = r / (1.f + r);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) zacc += __shfl_xor_sync(0xffffffffu, zacc, o);
+    }
+    for (int tok = warp; S::NP > 32 && tok < tb_valid; tok += kThreads / 32) {
         float* row = lg + tok * (S::NP + 1);
         float v[MPL];
         float m = -INFINITY;
