@@ -46,12 +46,12 @@ FP32_PEAK_NOTE = "148 SMs x 128 FP32 lanes x 2 flop x SM clock"
 # dram__bytes_write.sum) from one ncu capture, keyed by workload, valid only
 # for the kernel source it was measured on.
 NCU_TRAFFIC = {
-    # python bench.py --steps 3 --warmup 3 --no-cpu-baseline, then under
-    # ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none
-    #     -k regex:grouped_gemm -s 6 -c 2 (first timed step): stage 1 read
-    # 402836224 B (W1 + xe, the compulsory set) and wrote 362386432 B (H, part
-    # of it still in L2 when the kernel ends).
-    "switch_base": {"bytes_per_launch": 402836224 + 362386432, "src_sha": "7340ddffc88f93d6"},
+    # python bench.py --only --steps 3 --warmup 3 --no-cpu-baseline --no-backward --workload switch_base,
+    # then the same under ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none
+    #     -k regex:grouped_gemm -s 6 -c 2 (first timed forward): stage 1 read 402816512 B (W1 + xe, the
+    # compulsory set) and wrote 363179520 B (H, part of it still in L2 when the kernel ends).  Keyed to the
+    # GEMM's sources (gemm_tc.cu, tc_common.cuh) at the capture.
+    "switch_base": {"bytes_per_launch": 402816512 + 363179520, "src_sha": "aaba3448cdb8069c"},
 }
 
 
@@ -66,7 +66,7 @@ def peaks():
 
 def gemm_source_sha():
     h = hashlib.sha256()
-    for name in ("gemm_tc.cu", "common.cuh"):
+    for name in ("gemm_tc.cu", "tc_common.cuh"):
         with open(os.path.join(ROOT, "mixture_experts_sparse_b200", "csrc", name), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]

@@ -67,7 +67,7 @@ struct GemmShape {
     static constexpr int B_BYTES = B_ROWS * BK * 2;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
     static constexpr int STAGES = PAIR ? 6 : 4;
-    static constexpr int EPI_BYTES = 4 * 32 * 128;                // per epilogue warp: 32 rows x 128 B
+    static constexpr int EPI_BYTES = 2 * 4 * 32 * 128;            // per epilogue warp: 2 x (32 rows x 128 B)
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024;
     static constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, BN);
 };
@@ -130,7 +130,8 @@ __device__ __forceinline__ float silu(float z) { return z / (1.f + expf(-z)); }
 template <int EPI, bool PAIR>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const __grid_constant__ CUtensorMap tmB3, const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tmB3, const __grid_constant__ CUtensorMap tmOut,
+                    const GemmParams p) {
     using S = GemmShape<PAIR>;
     constexpr int BN_OUT = (EPI == EPI_SWIGLU) ? BN / 2 : BN;
     extern __shared__ uint8_t smem_raw[];
@@ -328,7 +329,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         // row), so every global store instruction writes whole 128-byte lines.
         const int q = warp & 3;                 // TMEM lane quadrant of this warp
         const int r_in_tile = (int)rank * BM + q * 32 + lane;
-        const uint32_t ebuf = smem_u32(smem + S::STAGES * S::STAGE_BYTES + q * 32 * 128);
+        // two staging buffers per warp (32 rows x 128 B each, 128-byte swizzled):
+        // compact outputs leave them through TMA stores issued by lane 0
+        const uint32_t ebuf0 = smem_u32(smem + S::STAGES * S::STAGE_BYTES + q * 2 * 32 * 128);
+        constexpr bool TMA_OUT = EPI != EPI_SCATTER;
+        uint32_t nchunk = 0;   // chunks staged so far (buffer = nchunk & 1; one bulk group each)
         const uint32_t tempty_leader0 = PAIR ? map_to_rank(smem_u32(&tempty_bar[0]), 0) : 0u;
         const uint32_t tempty_leader1 = PAIR ? map_to_rank(smem_u32(&tempty_bar[1]), 0) : 0u;
         constexpr int CW = 64;                  // output columns per chunk
@@ -370,6 +375,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             // bias / activation / gate, bf16 pack, staged rows, 128-byte row stores
             auto emit = [&](int c, const uint32_t (&u)[CW], const uint32_t (&v)[EPI == EPI_SWIGLU ? CW : 1]) {
                 const int col0 = ti.n0 + c * CW;
+                const uint32_t ebuf = ebuf0 + (nchunk & 1u) * (32 * 128);
+                if (TMA_OUT) {   // the store that last read this buffer (two chunks ago) is done with it
+                    if (lane == 0) bulk_wait_read<1>();
+                    __syncwarp();
+                }
 #pragma unroll
                 for (int gi = 0; gi < CW / 8; ++gi) {   // one 16-byte granule = 8 columns
                     const int col = col0 + 8 * gi;
@@ -431,22 +441,34 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                                  "r"(pk[2]), "r"(pk[3])
                                  : "memory");
                 }
-                __syncwarp();
-                const int gi = lane & 7;
-                const bool col_ok = col0 + 8 * gi < p.n_dim;
+                // all 32 rows of the warp's box belong to this tile: one TMA store
+                // (columns past n_dim are clipped by the tensor map); otherwise the
+                // rows are stored by the lanes, skipping the rows past the tile
+                const bool whole = TMA_OUT && (int)rank * BM + q * 32 + 32 <= ti.rows;
+                if (whole) {
+                    fence_proxy_async_smem();   // the staged rows are visible to the TMA unit
+                    __syncwarp();
+                    if (lane == 0) tma_store_2d(&tmOut, ebuf, col0, (int)(ti.row0 + (int)rank * BM + q * 32));
+                } else {
+                    __syncwarp();
+                    const int gi = lane & 7;
+                    const bool col_ok = col0 + 8 * gi < p.n_dim;
 #pragma unroll
-                for (int k4 = 0; k4 < 8; ++k4) {   // rows 4*k4 .. 4*k4+3 of the warp
-                    const int r = 4 * k4 + (lane >> 3);
-                    uint4 val;
-                    const uint32_t srcp = ebuf + r * 128 + ((gi ^ (r & 7)) << 4);
-                    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                                 : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
-                                 : "r"(srcp)
-                                 : "memory");
-                    if (dst_row[k4] != nullptr && col_ok)
-                        *reinterpret_cast<uint4*>(dst_row[k4] + col0 + 8 * gi) = val;
+                    for (int k4 = 0; k4 < 8; ++k4) {   // rows 4*k4 .. 4*k4+3 of the warp
+                        const int r = 4 * k4 + (lane >> 3);
+                        uint4 val;
+                        const uint32_t srcp = ebuf + r * 128 + ((gi ^ (r & 7)) << 4);
+                        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                     : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                                     : "r"(srcp)
+                                     : "memory");
+                        if (dst_row[k4] != nullptr && col_ok)
+                            *reinterpret_cast<uint4*>(dst_row[k4] + col0 + 8 * gi) = val;
+                    }
                 }
+                if (TMA_OUT && lane == 0) bulk_commit();   // one group per chunk, possibly empty
                 __syncwarp();
+                ++nchunk;
             };
             auto release = [&]() {   // every TMEM read of this accumulator has completed
                 tc_fence_before();
@@ -490,6 +512,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
     }
 
+    if (warp >= 2 && lane == 0 && EPI != EPI_SCATTER) bulk_wait_all();   // this warp's TMA stores have landed
     tc_fence_before();
     __syncthreads();
     if (PAIR) cluster_sync();   // no CTA leaves while its peer may still signal it
@@ -510,8 +533,8 @@ std::mutex g_mu;
 DeviceInfo g_dev[64];
 
 template <int EPI, bool PAIR>
-cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b3, const GemmParams& p,
-                     cudaStream_t s) {
+cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b3, const CUtensorMap& o,
+                     const GemmParams& p, cudaStream_t s) {
     using S = GemmShape<PAIR>;
     int dev = 0;
     cudaError_t err = cudaGetDevice(&dev);
@@ -534,10 +557,10 @@ cudaError_t run_gemm(const CUtensorMap& a, const CUtensorMap& b, const CUtensorM
     }
     if constexpr (!PAIR)
         return launch_k(grouped_gemm_kernel<EPI, false>, dim3((unsigned)sms), dim3(GEMM_THREADS), S::SMEM_BYTES, s,
-                        1, a, b, b3, p);
+                        1, a, b, b3, o, p);
     else
         return launch_k(grouped_gemm_kernel<EPI, true>, dim3((unsigned)(sms / 2) * 2), dim3(GEMM_THREADS),
-                        S::SMEM_BYTES, s, 2, a, b, b3, p);
+                        S::SMEM_BYTES, s, 2, a, b, b3, o, p);
 }
 
 // Variant choice: the CTA-pair kernel unless MOE_B200_GEMM=single (kept for
@@ -551,9 +574,9 @@ bool use_pair() {
 }
 
 template <int EPI>
-cudaError_t run_gemm_any(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b3, const GemmParams& p,
-                         cudaStream_t s) {
-    return use_pair() ? run_gemm<EPI, true>(a, b, b3, p, s) : run_gemm<EPI, false>(a, b, b3, p, s);
+cudaError_t run_gemm_any(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b3, const CUtensorMap& o,
+                         const GemmParams& p, cudaStream_t s) {
+    return use_pair() ? run_gemm<EPI, true>(a, b, b3, o, p, s) : run_gemm<EPI, false>(a, b, b3, o, p, s);
 }
 
 }  // namespace
@@ -635,8 +658,10 @@ cudaError_t launch_expert_ffn_tc(const FfnArgs& a, cudaStream_t s) {
     p1.status = &a.hdr->status;
     p1.limit_ns = kWaitLimitNs;
     p1.pre_out = reinterpret_cast<__nv_bfloat16*>(a.pre_out);
-    cudaError_t err = swiglu ? run_gemm_any<EPI_SWIGLU>(mA1, mB1, mB3, p1, s)
-                             : run_gemm_any<EPI_RELU>(mA1, mB1, mB3, p1, s);
+    CUtensorMap mO1, mO2;   // the compact outputs H [R, d_ff] and ye [R, d], 32-row boxes (TMA stores)
+    if (!make_map_bf16(&mO1, a.h, R, a.d_ff, 32)) return cudaErrorInvalidValue;
+    cudaError_t err = swiglu ? run_gemm_any<EPI_SWIGLU>(mA1, mB1, mB3, mO1, p1, s)
+                             : run_gemm_any<EPI_RELU>(mA1, mB1, mB3, mO1, p1, s);
     if (err != cudaSuccess || a.stage1_only) return err;
     if (a.mid_event && (err = cudaEventRecord((cudaEvent_t)a.mid_event, s)) != cudaSuccess) return err;
 
@@ -655,10 +680,11 @@ cudaError_t launch_expert_ffn_tc(const FfnArgs& a, cudaStream_t s) {
         p2.row_gate = a.row_gate;
         p2.out_ptrs = a.scatter_ptrs;
         p2.row_rank = a.row_rank;
-        return run_gemm_any<EPI_SCATTER>(mA2, mB2, mB2, p2, s);
+        return run_gemm_any<EPI_SCATTER>(mA2, mB2, mB2, mA2, p2, s);
     }
     p2.out = reinterpret_cast<__nv_bfloat16*>(a.ye);
-    return run_gemm_any<EPI_BIAS>(mA2, mB2, mB2, p2, s);
+    if (!make_map_bf16(&mO2, a.ye, R, a.d, 32)) return cudaErrorInvalidValue;
+    return run_gemm_any<EPI_BIAS>(mA2, mB2, mB2, mO2, p2, s);
 }
 
 }  // namespace moe
