@@ -63,6 +63,7 @@ struct Layout {
     size_t ntlb_probs, ntlb_ch, ntlb_last, ntlb_first, ntlb_placed, ntlb_lp;               // re-routing only
     size_t ntlb_agg, ntlb_unplaced, ntlb_bar;
     size_t bwd_part_dw, bwd_part_db;   // router backward partials
+    size_t rb_adx, rb_adw, rb_bdx, rb_offs, rb_part;   // router backward on the tensor cores (bf16)
     size_t total;
     int64_t rows;   // min(k T, N C): compact rows the buffers hold
 };
@@ -111,6 +112,14 @@ Layout layout_of(const moe_config& c) {
     const size_t nch = (size_t)router_bwd_chunks(c.T);
     L.bwd_part_dw = take(4 * nch * N * (size_t)c.d_model);
     L.bwd_part_db = take(4 * nch * N);
+    if (c.dtype == MOE_BF16) {
+        const size_t np16 = (size_t)router_bwd_np16(c.n_experts), nct = (size_t)router_bwd_tc_chunks(c.T);
+        L.rb_adx = take(2 * T * 6 * np16);
+        L.rb_adw = take(2 * T * 3 * np16);
+        L.rb_bdx = take(2 * 6 * np16 * (size_t)c.d_model);
+        L.rb_offs = take(4 * (nct + 3));
+        L.rb_part = take(4 * nct * 3 * np16 * (size_t)c.d_model);
+    }
     if (c.priority == MOE_ORDER_PRIORITY) {   // batch-priority claim order scratch
         L.prio_hist = take(4 * (size_t)(kPrioBuckets + 1));
         L.prio_cursor = take(4 * (size_t)kPrioBuckets);
@@ -442,6 +451,14 @@ int32_t moe_router_backward(const moe_config* cfg, const void* x, const float* w
     a.dx = dx;
     a.part_dw = at<float>(ws, L.bwd_part_dw);
     a.part_db = at<float>(ws, L.bwd_part_db);
+    if (cfg->dtype == MOE_BF16) {
+        a.tc_adx = at<void>(ws, L.rb_adx);
+        a.tc_adw = at<void>(ws, L.rb_adw);
+        a.tc_bdx = at<void>(ws, L.rb_bdx);
+        a.tc_offs = at<int32_t>(ws, L.rb_offs);
+        a.tc_part = at<float>(ws, L.rb_part);
+    }
+    a.status = &at<WsHeader>(ws, L.hdr)->status;
     return cuda_status(launch_router_backward(a, (cudaStream_t)stream));
 }
 

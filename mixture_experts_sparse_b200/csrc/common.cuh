@@ -222,8 +222,16 @@ struct RouterBwdArgs {
     float* dh;                        // [T, N]
     float* dw; float* db; float* dx;  // [N, d], [N], [T, d] (each nullable)
     float* part_dw; float* part_db;   // [router_bwd_chunks(T), N, d], [.., N]
+    // tensor-core path (bf16 x): workspace regions, see router_bwd_tc_bytes
+    void* tc_adx; void* tc_adw; void* tc_bdx; int32_t* tc_offs; float* tc_part;
+    int32_t* status;
 };
 int router_bwd_chunks(int64_t T);
+// tensor-core router backward: padded experts (a multiple of 16), tokens per
+// dW_r chunk (at most 128 chunks), and the chunk count
+int router_bwd_np16(int N);
+int64_t router_bwd_tc_chunk(int64_t T);
+int router_bwd_tc_chunks(int64_t T);
 cudaError_t launch_router_backward(const RouterBwdArgs& a, cudaStream_t s);
 int router_blocks(int64_t T, int N);               // partial rows the FP32-pipe router writes
 int router_partial_rows(int64_t T, int N);         // partial rows any router path writes
@@ -322,6 +330,10 @@ struct BwdArgs {
     WsHeader* hdr;
 };
 cudaError_t launch_expert_backward_tc(const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_tc_rows_f32(const void* A, int64_t rows, int K, const void* B, int n, const int32_t* offsets,
+                               float* out, int32_t* status, cudaStream_t s);
+cudaError_t launch_tc_weights_f32(const void* A, int64_t rows, int m, const void* B, int n, const int32_t* offsets,
+                                  int groups, float* out, int32_t* status, cudaStream_t s);
 
 // Expert parallelism (ep.cu)
 struct EpDispatchArgs {

@@ -477,6 +477,44 @@ cudaError_t run_bwd(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMa
 
 }  // namespace
 
+// Plain tensor-core products of the router backward (router_bwd.cu), over
+// groups of rows given by `offsets` [groups + 1] (device):
+//   rows: out[r, :] = A[r, :] B with A [rows, K] K-major, B [K, n] read MN-major;
+//   weights: out[g] = A_g^T B_g over each group's rows, A [rows, m] and B
+//   [rows, n] both read MN-major (out [groups, m, n]).
+// Outputs fp32.
+cudaError_t launch_tc_rows_f32(const void* A, int64_t rows, int K, const void* B, int n, const int32_t* offsets,
+                               float* out, int32_t* status, cudaStream_t s) {
+    CUtensorMap ma, mb;
+    if (!make_map_bf16(&ma, A, rows, K, BW_BM) || !make_map_bf16_mn(&mb, B, K, n, BW_BK))
+        return cudaErrorInvalidValue;
+    BwdParams p{};
+    p.offsets = offsets;
+    p.N = 1;
+    p.n_dim = n;
+    p.k_dim = K;
+    p.out = out;
+    p.status = status;
+    p.limit_ns = kWaitLimitNs;
+    return run_bwd<BW_DX>(ma, mb, mb, p, s);
+}
+
+cudaError_t launch_tc_weights_f32(const void* A, int64_t rows, int m, const void* B, int n, const int32_t* offsets,
+                                  int groups, float* out, int32_t* status, cudaStream_t s) {
+    CUtensorMap ma, mb;
+    if (!make_map_bf16_mn(&ma, A, rows, m, BW_BK) || !make_map_bf16_mn(&mb, B, rows, n, BW_BK))
+        return cudaErrorInvalidValue;
+    BwdParams p{};
+    p.offsets = offsets;
+    p.N = groups;
+    p.m_dim = m;
+    p.n_dim = n;
+    p.out = out;
+    p.status = status;
+    p.limit_ns = kWaitLimitNs;
+    return run_bwd<BW_WGT>(ma, mb, mb, p, s);
+}
+
 cudaError_t launch_expert_backward_tc(const BwdArgs& a, cudaStream_t s) {
     const int64_t R = a.R_cap > 0 ? a.R_cap : 1;
     const bool sw = a.act == MOE_SWIGLU;

@@ -12,10 +12,13 @@
 //  - dW_r = dh^T x, db_r = sum_t dh_t (a contraction over tokens: per
 //    512-token chunk partials, then a fixed-order fp64 sum over chunks), and
 //    dx_t = dh_t W_r.
-// Kernels: router_bwd_dh_kernel (one warp per token), router_bwd_dw_kernel
-// (32 experts x 128 columns per block over one token chunk),
-// router_bwd_reduce_kernel, router_bwd_dx_kernel (64 tokens x 128 columns).
-// All sums run in a fixed order: results are bit-identical run to run.
+// Kernels: router_bwd_dh_kernel (one warp per token); for bf16 x the two
+// contractions run on the tensor cores through exact three-way bf16 splits
+// (rbwd_* kernels, the grouped GEMMs of gemm_bwd.cu); for fp32 x on the FP32
+// pipe: router_bwd_dw_kernel (32 experts x 128 columns per block over one
+// token chunk), router_bwd_reduce_kernel, router_bwd_dx_kernel (64 tokens x
+// 128 columns).  All sums run in a fixed order: results are bit-identical run
+// to run.
 #include "common.cuh"
 
 namespace moe {
@@ -210,9 +213,122 @@ router_bwd_dx_kernel(const float* __restrict__ dh, const float* __restrict__ w_r
     }
 }
 
+// ---- tensor-core contractions (bf16 x) ---------------------------------------
+// x is exact in bf16; dh and W_r (fp32) split exactly into three bf16 parts
+// each (v = v0 + v1 + v2).  dW_r = sum_j dh_j^T x (three exact products, fp32
+// accumulation per token chunk, fp64 over chunks and parts); dx = dh W_r from
+// the six part products dh_i w_j with i + j <= 2 (the dropped ones are below
+// 2^-24 of the result), one GEMM with K = 6 NP16 over
+// [dh0 dh0 dh1 dh0 dh1 dh2] x [w0; w1; w0; w2; w1; w0].
+__device__ __forceinline__ void split3(float v, __nv_bfloat16& a, __nv_bfloat16& b, __nv_bfloat16& c) {
+    a = __float2bfloat16_rn(v);
+    const float r1 = v - __bfloat162float(a);
+    b = __float2bfloat16_rn(r1);
+    c = __float2bfloat16_rn(r1 - __bfloat162float(b));
+}
+
+__global__ void __launch_bounds__(256)
+rbwd_split_kernel(const float* __restrict__ dh, int64_t T, int N, int NP16, __nv_bfloat16* __restrict__ adx,
+                  __nv_bfloat16* __restrict__ adw, int32_t* __restrict__ offs, int64_t chunk, int nchunk) {
+    pdl_wait();
+    pdl_launch();
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        offs[0] = 0;
+        offs[1] = (int32_t)T;
+        for (int i = 0; i <= nchunk; ++i) offs[2 + i] = (int32_t)min((int64_t)i * chunk, T);
+    }
+    const int64_t n_el = T * NP16;
+    for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < n_el; q += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = q / NP16;
+        const int e = (int)(q - t * NP16);
+        const float v = e < N ? dh[t * N + e] : 0.f;
+        __nv_bfloat16 h0, h1, h2;
+        split3(v, h0, h1, h2);
+        __nv_bfloat16* rx = adx + t * (6 * NP16) + e;
+        rx[0] = h0;
+        rx[NP16] = h0;
+        rx[2 * NP16] = h1;
+        rx[3 * NP16] = h0;
+        rx[4 * NP16] = h1;
+        rx[5 * NP16] = h2;
+        __nv_bfloat16* rw = adw + t * (3 * NP16) + e;
+        rw[0] = h0;
+        rw[NP16] = h1;
+        rw[2 * NP16] = h2;
+    }
+}
+
+__global__ void __launch_bounds__(256)
+rbwd_wsplit_kernel(const float* __restrict__ w_r, int N, int NP16, int d, __nv_bfloat16* __restrict__ bdx) {
+    pdl_wait();
+    pdl_launch();
+    const int64_t n_el = (int64_t)NP16 * d;
+    for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < n_el; q += (int64_t)gridDim.x * blockDim.x) {
+        const int e = (int)(q / d);
+        const int c = (int)(q - (int64_t)e * d);
+        __nv_bfloat16 w[3];
+        split3(e < N ? w_r[(int64_t)e * d + c] : 0.f, w[0], w[1], w[2]);
+        const int part[6] = {0, 1, 0, 2, 1, 0};   // the W_r part each K segment multiplies
+#pragma unroll
+        for (int sg = 0; sg < 6; ++sg) bdx[((int64_t)sg * NP16 + e) * d + c] = w[part[sg]];
+    }
+}
+
+// part_db[chunk][e] = sum over the chunk's tokens of dh[t][e] (fp32, in order)
+__global__ void __launch_bounds__(128)
+rbwd_db_kernel(const float* __restrict__ dh, int64_t T, int N, int64_t chunk, float* __restrict__ part_db) {
+    pdl_wait();
+    pdl_launch();
+    const int e = threadIdx.x;
+    if (e >= N) return;
+    const int64_t t0 = (int64_t)blockIdx.x * chunk, t1 = min(T, t0 + chunk);
+    float acc = 0.f;
+    for (int64_t t = t0; t < t1; ++t) acc += dh[t * N + e];
+    part_db[(int64_t)blockIdx.x * N + e] = acc;
+}
+
+// dw[e][c] = sum over chunks (in order) of the three parts' partial products,
+// db[e] = sum over chunks of part_db; fp64
+__global__ void __launch_bounds__(256)
+rbwd_reduce_tc_kernel(const float* __restrict__ part, const float* __restrict__ part_db, int nchunk, int N, int NP16,
+                      int d, float* __restrict__ dw, float* __restrict__ db) {
+    pdl_wait();
+    pdl_launch();
+    const int64_t n = (int64_t)N * d;
+    for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < n + N; q += (int64_t)gridDim.x * blockDim.x) {
+        if (q < n) {
+            if (!dw) continue;
+            const int e = (int)(q / d);
+            const int c = (int)(q - (int64_t)e * d);
+            double acc = 0.0;
+            for (int ch = 0; ch < nchunk; ++ch) {
+                const float* pc = part + (int64_t)ch * 3 * NP16 * d;
+#pragma unroll
+                for (int j = 0; j < 3; ++j) acc += (double)pc[((int64_t)j * NP16 + e) * d + c];
+            }
+            dw[q] = (float)acc;
+        } else if (db) {
+            const int e = (int)(q - n);
+            double acc = 0.0;
+            for (int ch = 0; ch < nchunk; ++ch) acc += (double)part_db[(int64_t)ch * N + e];
+            db[e] = (float)acc;
+        }
+    }
+}
+
 }  // namespace
 
 int router_bwd_chunks(int64_t T) { return (int)((T + kBwdChunk - 1) / kBwdChunk); }
+int router_bwd_np16(int N) { return (N + 15) / 16 * 16; }
+int64_t router_bwd_tc_chunk(int64_t T) {
+    int64_t c = (T + 127) / 128;   // at most 128 chunks (the weight GEMM's group limit)
+    c = (c + 63) / 64 * 64;
+    return c < kBwdChunk ? kBwdChunk : c;
+}
+int router_bwd_tc_chunks(int64_t T) {
+    const int64_t c = router_bwd_tc_chunk(T);
+    return (int)((T + c - 1) / c);
+}
 
 cudaError_t launch_router_backward(const RouterBwdArgs& a, cudaStream_t s) {
     if (a.T <= 0) {   // no tokens: every gradient is zero
@@ -224,6 +340,43 @@ cudaError_t launch_router_backward(const RouterBwdArgs& a, cudaStream_t s) {
     cudaError_t err = launch_k(router_bwd_dh_kernel, dim3((unsigned)((a.T + 7) / 8)), dim3(256), 0, s, 1, a.probs,
                                a.idx, a.gate, a.dgate, a.f, a.alpha, a.T, a.N, a.k, a.dh);
     if (err != cudaSuccess) return err;
+    if (a.dtype == MOE_BF16 && a.tc_adx && (a.dw || a.db || a.dx)) {
+        // the contractions on the tensor cores
+        const int NP16 = router_bwd_np16(a.N);
+        const int64_t chunk = router_bwd_tc_chunk(a.T);
+        const int nchunk = router_bwd_tc_chunks(a.T);
+        const int64_t n_el = a.T * NP16;
+        const unsigned sg = (unsigned)((n_el + 255) / 256 < 8192 ? (n_el + 255) / 256 : 8192);
+        if ((err = launch_k(rbwd_split_kernel, dim3(sg), dim3(256), 0, s, 1, static_cast<const float*>(a.dh), a.T,
+                            a.N, NP16, reinterpret_cast<__nv_bfloat16*>(a.tc_adx),
+                            reinterpret_cast<__nv_bfloat16*>(a.tc_adw), a.tc_offs, chunk, nchunk)) != cudaSuccess)
+            return err;
+        if (a.dx) {
+            const int64_t w_el = (int64_t)NP16 * a.d;
+            const unsigned wg = (unsigned)((w_el + 255) / 256 < 4096 ? (w_el + 255) / 256 : 4096);
+            if ((err = launch_k(rbwd_wsplit_kernel, dim3(wg), dim3(256), 0, s, 1, a.w_r, a.N, NP16, a.d,
+                                reinterpret_cast<__nv_bfloat16*>(a.tc_bdx))) != cudaSuccess)
+                return err;
+            if ((err = launch_tc_rows_f32(a.tc_adx, a.T, 6 * NP16, a.tc_bdx, a.d, a.tc_offs, a.dx, a.status, s)) !=
+                cudaSuccess)
+                return err;
+        }
+        if (a.dw || a.db) {
+            if (a.dw && (err = launch_tc_weights_f32(a.tc_adw, a.T, 3 * NP16, a.x, a.d, a.tc_offs + 2, nchunk,
+                                                     a.tc_part, a.status, s)) != cudaSuccess)
+                return err;
+            if ((err = launch_k(rbwd_db_kernel, dim3((unsigned)nchunk), dim3(128), 0, s, 1,
+                                static_cast<const float*>(a.dh), a.T, a.N, chunk, a.part_db)) != cudaSuccess)
+                return err;
+            const int64_t n = (int64_t)a.N * a.d + a.N;
+            const unsigned rg = (unsigned)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+            if ((err = launch_k(rbwd_reduce_tc_kernel, dim3(rg), dim3(256), 0, s, 1,
+                                static_cast<const float*>(a.tc_part), static_cast<const float*>(a.part_db), nchunk,
+                                a.N, NP16, a.d, a.dw, a.db)) != cudaSuccess)
+                return err;
+        }
+        return cudaSuccess;
+    }
     if (a.dw || a.db) {
         const int nchunk = router_bwd_chunks(a.T);
         const dim3 g((unsigned)nchunk, (unsigned)((a.N + 31) / 32), (unsigned)((a.d + 127) / 128));

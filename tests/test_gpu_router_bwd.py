@@ -3,9 +3,10 @@ dL/dh, dW_r, db_r and the router's part of dL/dx for L = sum dgate * gate +
 L_aux (gate path of "From Switch Transformer to GLaM"; load-balancing
 gradient through P with coefficient f, CMU 10-423 Lecture 16, section 4.2).
 Inputs are the oracle's forward values (probs, idx, gate, f), so both sides
-differentiate the same point.  The GPU computes in fp32 (per-chunk fp32 sums
-over tokens, fp64 over chunks): tolerances are relative to each output's
-largest magnitude.  Needs a B200."""
+differentiate the same point.  bf16 layers take the tensor-core path (exact
+three-way bf16 splits of dh and W_r, fp32 accumulation over token chunks,
+fp64 over chunks), fp32 layers the FP32 pipe: tolerances are relative to each
+output's largest magnitude.  Needs a B200."""
 import numpy as np
 import pytest
 
@@ -65,6 +66,22 @@ def test_router_backward_matches_oracle(T, d, N, k, dtype):
     again = _run(L, r, f, dgate, T, d, N, k, dtype, alpha)
     for key in got:
         np.testing.assert_array_equal(got[key], again[key], err_msg=f"{key} not deterministic")
+
+
+def test_router_backward_full_size_matches_oracle():
+    # the Switch-Base router at full size: T = 65536 tokens, d = 768, N = 64,
+    # top-1, bf16 tokens: every output element against the oracle
+    T, d, N, k, alpha = 65536, 768, 64, 1, 0.01
+    L = inputs.make_layer(T=T, d_model=d, d_ff=64, n_experts=N, top_k=k, dtype="bf16", seed=65)
+    r = oracle.route(L["x"], L["w_r"], L["b_r"], k)
+    f, _, _ = oracle.aux_loss(r["idx"], r["probs"], alpha)
+    dgate = np.random.default_rng(65).standard_normal((T, k)).astype(np.float32)
+    ref = oracle.router_backward(L["x"], L["w_r"], r["probs"], r["idx"], r["gate"], f, dgate, alpha)
+    got = _run(L, r, f, dgate, T, d, N, k, "bf16", alpha)
+    _close(got["dh"], ref["dh"], TOL_DH, "dh")
+    _close(got["dw"], ref["dw"], TOL_SUM, "dW_r")
+    _close(got["db"], ref["db"], TOL_SUM, "db_r")
+    _close(got["dx"], ref["dx"], TOL_SUM, "dx")
 
 
 def test_router_backward_empty_batch():
