@@ -246,6 +246,50 @@ scatter_kernel(const XT* __restrict__ x, const int32_t* __restrict__ idx, const 
     }
 }
 
+// The same slot bookkeeping without the compact copy and without output rows
+// to zero (moe_dispatch called with no xe): one thread per assignment writes
+// pos, drop, row_token and row_gate -- 32x fewer warps than scatter_kernel,
+// whose warp per assignment exists for the row copy.
+__global__ void __launch_bounds__(256)
+rowmap_kernel(const int32_t* __restrict__ idx, const float* __restrict__ gate, int64_t T, int N, int k, int C,
+              const int32_t* __restrict__ claim_base, int32_t* __restrict__ pos, uint8_t* __restrict__ drop,
+              const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
+              int32_t* __restrict__ row_token, float* __restrict__ row_gate, const AuxArgs aux,
+              const int32_t* __restrict__ perm, const int32_t* __restrict__ pos_in) {
+    pdl_wait();
+    pdl_launch();
+    if (aux.G > 0 && blockIdx.x == 0) {   // the load-balancing loss, as in scatter_kernel
+        __shared__ double s_aux[kAuxScratch];
+        aux_reduce_block(aux, s_aux);
+        return;
+    }
+    const int64_t a = (int64_t)(blockIdx.x - (aux.G > 0 ? 1 : 0)) * 256 + threadIdx.x;
+    if (a >= T * k) return;
+    const int64_t q = a / k;
+    const int r = (int)(a - q * k);
+    const int64_t t = perm ? (int64_t)perm[q] : q;
+    const int64_t ao = t * k + r;
+    const int e = idx[ao];
+    const int lp = pos_in ? pos_in[a] : pos[a];
+    int p, row_off;
+    if (r == 0) {
+        p = (claim_base ? claim_base[e] : 0) + lp;
+        row_off = lp;
+    } else {
+        const int base0 = claim_base ? claim_base[e] : 0;
+        p = (claim_base ? claim_base[N + e] : counts[e]) + lp;
+        row_off = kept_after(base0, counts[e], C) + lp;
+    }
+    const bool keep = p < C;
+    pos[ao] = p;
+    drop[ao] = keep ? 0 : 1;
+    if (keep) {
+        const int row = offsets[e] + row_off;
+        row_token[row] = (int32_t)t;
+        row_gate[row] = gate[ao];
+    }
+}
+
 // ---- batch priority: the claim order --------------------------------------
 // CS25 Lecture 05 notes, section on Vision MoE: with capacity short, priority
 // routing lets the tokens with the highest priority score take the expert
@@ -709,6 +753,12 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
     err = launch_k(scan_kernel, dim3((unsigned)nblk), dim3(kScanThreads), 0, s, 1, scan_idx, a.T, a.N, a.k, a.C, nblk,
                    a.claim_base, scan_pos, a.counts, a.kept, a.offsets, a.scan_state, a.hdr, kWaitLimitNs);
     if (err != cudaSuccess) return err;
+    if (a.xe == nullptr && a.zero_out == nullptr) {   // row map only: thread per assignment
+        const unsigned grid = (unsigned)((a.T * a.k + 255) / 256) + (a.aux.G > 0 ? 1u : 0u);
+        return launch_k(rowmap_kernel, dim3(grid), dim3(256), 0, s, 1, a.idx, a.gate, a.T, a.N, a.k, a.C,
+                        a.claim_base, a.pos, a.drop, a.counts, a.offsets, a.row_token, a.row_gate, a.aux, perm,
+                        pos_in);
+    }
     const int64_t warps = a.T * a.k;
     const unsigned grid = (unsigned)((warps + 7) / 8) + (a.aux.G > 0 ? 1u : 0u);
     if (a.dtype == MOE_BF16)
@@ -772,9 +822,16 @@ cudaError_t launch_dispatch_ntlb(const NtlbArgs& a, cudaStream_t s) {
     cfg.numAttrs = 1;
     if ((err = cudaLaunchKernelEx(&cfg, ntlb_grid_kernel, g)) != cudaSuccess) return err;
     // the gather, from the final experts and claim numbers (rank 0, no claim base)
-    const unsigned grid = (unsigned)((a.T + 7) / 8) + (a.aux.G > 0 ? 1u : 0u);
     const int32_t* none = nullptr;
     const int N = a.N;
+    if (a.xe == nullptr && a.zero_out == nullptr) {   // row map only
+        const unsigned g2 = (unsigned)((a.T + 255) / 256) + (a.aux.G > 0 ? 1u : 0u);
+        return launch_k(rowmap_kernel, dim3(g2), dim3(256), 0, s, 1, static_cast<const int32_t*>(a.expert),
+                        static_cast<const float*>(a.gate), a.T, N, 1, a.C, none, a.pos, a.drop,
+                        static_cast<const int32_t*>(a.counts), static_cast<const int32_t*>(a.offsets), a.row_token,
+                        a.row_gate, a.aux, none, none);
+    }
+    const unsigned grid = (unsigned)((a.T + 7) / 8) + (a.aux.G > 0 ? 1u : 0u);
     if (a.dtype == MOE_BF16)
         return launch_k(scatter_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, 1,
                         reinterpret_cast<const __nv_bfloat16*>(a.x), static_cast<const int32_t*>(a.expert),

@@ -26,7 +26,7 @@ if not torch.cuda.is_available():
     pytest.skip("needs a CUDA device", allow_module_level=True)
 
 
-def _gpu_ntlb(L, probs, T, d, N, C):
+def _gpu_ntlb(L, probs, T, d, N, C, copy=True):
     cfg = nat.config(T, d, 64, N, 1, C, priority=nat.MOE_ORDER_NTLB)
     ws = nat.new_workspace(cfg)
     R = max(1, min(T, N * C))
@@ -43,7 +43,7 @@ def _gpu_ntlb(L, probs, T, d, N, C):
                xe=torch.zeros(R, d, dtype=torch.bfloat16, **dev))
     nat.check(nat.moe_dispatch_ntlb(cfg, to_device(L["x"]), to_device(probs), out["expert"], out["gate"], out["pos"],
                                     out["drop"], out["counts"], out["kept"], out["offsets"], out["row_token"],
-                                    out["row_gate"], out["xe"], ws))
+                                    out["row_gate"], out["xe"] if copy else None, ws))
     torch.cuda.synchronize()
     nat.check(nat.moe_read_device_status(ws))
     return {key: (to_host_bits(v) if key == "xe" else v.cpu().numpy()) for key, v in out.items()}
@@ -52,7 +52,8 @@ def _gpu_ntlb(L, probs, T, d, N, C):
 @pytest.mark.parametrize("T,N,cf,bias,ties", [(4099, 7, 1.0, 0.8, False), (3000, 16, 1.25, 1.5, False),
                                               (2000, 8, 0.5, 0.0, False), (1000, 1, 0.5, 0.0, False),
                                               (1500, 6, 1.0, 1.0, True), (700, 5, 0.0, 0.5, False)])
-def test_ntlb_dispatch_exact(T, N, cf, bias, ties):
+@pytest.mark.parametrize("copy", [True, False], ids=["copy", "rowmap"])
+def test_ntlb_dispatch_exact(T, N, cf, bias, ties, copy):
     d = 128
     rb = np.linspace(bias, 0.0, N).astype(np.float32) if bias else None
     L = inputs.make_layer(T=T, d_model=d, d_ff=64, n_experts=N, top_k=1, dtype="bf16", seed=T + N, router_bias=rb)
@@ -63,7 +64,7 @@ def test_ntlb_dispatch_exact(T, N, cf, bias, ties):
     C = nat.moe_capacity(T, N, 1, cf)
     first = np.array([min(range(N), key=lambda e: (-float(probs[t, e]), e)) for t in range(T)])
     want = oracle.dispatch_ntlb(probs, probs[np.arange(T), first], C)
-    got = _gpu_ntlb(L, probs, T, d, N, C)
+    got = _gpu_ntlb(L, probs, T, d, N, C, copy)
     for key in ("expert", "gate", "pos", "drop", "counts", "kept", "offsets"):
         np.testing.assert_array_equal(got[key], want[key], err_msg=key)
     nrows = int(want["offsets"][-1])
@@ -73,7 +74,8 @@ def test_ntlb_dispatch_exact(T, N, cf, bias, ties):
     want_t[rows] = kept_t
     np.testing.assert_array_equal(got["row_token"][:nrows], want_t)
     np.testing.assert_array_equal(got["row_gate"][:nrows], want["gate"][want_t])
-    np.testing.assert_array_equal(got["xe"][:nrows], L["x"][want_t])
+    if copy:
+        np.testing.assert_array_equal(got["xe"][:nrows], L["x"][want_t])
 
 
 @pytest.mark.parametrize("case", [(3000, 128, 256, 8, 1.0, "relu", "bf16", 1.0), (900, 64, 128, 5, 1.25, "relu", "f32", 0.8)],
