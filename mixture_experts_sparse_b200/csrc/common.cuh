@@ -37,6 +37,17 @@ __device__ __forceinline__ long long global_ns() {
     return (long long)t;
 }
 
+// 2^x in one MUFU instruction (PTX ex2.approx.ftz.f32: relative error about
+// 2^-22; results below 2^-126 flush to zero, 2^-inf = 0).  e^z is taken as
+// 2^(z log2 e).  CUDA's exp2f/expf add range handling that costs about 50
+// cycles a call -- the bulk of a per-token softmax over 64 experts.
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+constexpr float kLog2e = 1.4426950408889634f;
+
 __device__ __forceinline__ void latch_status(int32_t* status, int32_t code) {
     atomicCAS(status, 0, code);
 }

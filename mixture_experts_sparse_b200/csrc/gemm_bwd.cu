@@ -91,7 +91,7 @@ __device__ __forceinline__ BwTile bw_decode(int tile, const int* prefix, const i
     return t;
 }
 
-__device__ __forceinline__ float sigmoidf_(float z) { return 1.f / (1.f + expf(-z)); }
+__device__ __forceinline__ float sigmoidf_(float z) { return __fdividef(1.f, 1.f + fast_exp2(-z * kLog2e)); }
 
 template <int MODE>
 __global__ void __launch_bounds__(BW_THREADS, 1)

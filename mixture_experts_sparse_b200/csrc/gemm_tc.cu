@@ -125,7 +125,9 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const int* prefix, con
     return ti;
 }
 
-__device__ __forceinline__ float silu(float z) { return z / (1.f + expf(-z)); }
+// z sigmoid(z) = z / (1 + e^-z); e^-z = 2^(-z log2 e) -> inf for very negative
+// z, where the fast division gives the limit 0
+__device__ __forceinline__ float silu(float z) { return __fdividef(z, 1.f + fast_exp2(-z * kLog2e)); }
 
 template <int EPI, bool PAIR>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)

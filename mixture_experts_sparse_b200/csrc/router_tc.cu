@@ -369,10 +369,10 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 m2 = tree_max(v, i1);
                 i2 = tree_first(v, m2, i1);
             }
-            // v now holds exp(h - max) = 2^((h - max) log2 e)
-            constexpr float kLog2e = 1.4426950408889634f;
+            // v now holds exp(h - max) = 2^((h - max) log2 e); padding experts
+            // hold -inf (their bias), so their terms are 0
 #pragma unroll
-            for (int e = 0; e < NP; ++e) v[e] = (e < N) ? exp2f((v[e] - m) * kLog2e) : 0.f;
+            for (int e = 0; e < NP; ++e) v[e] = fast_exp2((v[e] - m) * kLog2e);
             const float s = tree_sum(v);
             const float inv = valid ? 1.f / s : 0.f;
             if (valid) {
@@ -382,7 +382,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     p.idx[t] = i1;
                     p.gate[t] = inv;   // p_{i*} = exp(0) / s
                 } else {
-                    const float r = exp2f((m2 - m) * kLog2e);
+                    const float r = fast_exp2((m2 - m) * kLog2e);
                     p.idx[2 * t] = i1;
                     p.idx[2 * t + 1] = i2;
                     p.gate[2 * t] = 1.f / (1.f + r);
