@@ -48,10 +48,10 @@ FP32_PEAK_NOTE = "148 SMs x 128 FP32 lanes x 2 flop x SM clock"
 NCU_TRAFFIC = {
     # python bench.py --only --steps 3 --warmup 3 --no-cpu-baseline --no-backward --workload switch_base,
     # then the same under ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none
-    #     -k regex:grouped_gemm -s 6 -c 2 (first timed forward): stage 1 read 402816512 B (W1 + xe, the
-    # compulsory set) and wrote 363179520 B (H, part of it still in L2 when the kernel ends).  Keyed to the
+    #     -k regex:grouped_gemm -s 6 -c 2 (first timed forward): stage 1 read 402795008 B (W1 + xe, the
+    # compulsory set) and wrote 362309376 B (H, part of it still in L2 when the kernel ends).  Keyed to the
     # GEMM's sources (gemm_tc.cu, tc_common.cuh) at the capture.
-    "switch_base": {"bytes_per_launch": 402816512 + 363179520, "src_sha": "aaba3448cdb8069c"},
+    "switch_base": {"bytes_per_launch": 402795008 + 362309376, "src_sha": "10155ce446bde52c"},
 }
 
 
@@ -537,7 +537,8 @@ def time_backward(w, L, layer, x, C, K, warmup, pk):
     return {"expert_ms": out["expert"], "router_ms": out["router"], "expert_flops": flops,
             "expert_achieved_tflops": ach, "expert_frac": ach / pk["bf16_tflops"],
             "note": "expert backward: recompute of the first GEMM + dA, dx, dW1 (dW3), dW2 on the tensor cores; "
-                    "FLOPs count dA, dx and the weight gradients only; router backward on the FP32 pipe"}
+                    "FLOPs count dA, dx and the weight gradients only; router backward on the tensor cores (bf16 x: "
+                    "exact three-way bf16 splits of dh and W_r)"}
 
 
 def build_layer(w, rank, local, x_seed=None):
