@@ -36,9 +36,9 @@
 // one N=256 MMA produces the gate and up halves side by side in TMEM.
 // Tiles: an expert's rows are cut into m-tiles; the tile list is expert-major
 // with m-tiles grouped by 8 inside an expert (concurrent CTAs share B columns and
-// A rows in L2).  Rows past an expert's end inside its last m-tile belong to the
-// next expert (or are zero-filled out of bounds); the MMA computes them and the
-// epilogue masks them.
+// A rows in L2), n-tiles fastest when there are at most 4 of them.  Rows past
+// an expert's end inside its last m-tile belong to the next expert (or are
+// zero-filled out of bounds); the MMA computes them and the epilogue masks them.
 // Every wait on an mbarrier is bounded: on expiry the kernel latches
 // MOE_ERR_TIMEOUT, stops issuing work, waits (bounded) for its own copies and
 // MMAs in flight, frees TMEM and returns.
@@ -115,8 +115,12 @@ __device__ __forceinline__ TileInfo decode_tile(int tile, const int* prefix, con
     const int first_m = g * GROUP_M;
     const int gsz = min(mt - first_m, GROUP_M);
     const int rem = local - g * per_group;
-    const int m_blk = first_m + rem % gsz;
-    const int n_blk = rem / gsz;
+    // few n-tiles (a second GEMM with d <= 1024): n fastest, so the tiles that
+    // share one block of A rows run at the same time and it is read from DRAM
+    // once (Switch-Base stage 2: 764 -> 750 MB read, top-2: 956 -> 879 MB);
+    // otherwise m fastest in groups of GROUP_M (tiles sharing B columns)
+    const int m_blk = ntn <= 4 ? first_m + rem / ntn : first_m + rem % gsz;
+    const int n_blk = ntn <= 4 ? rem % ntn : rem / gsz;
     TileInfo ti;
     ti.e = e;
     ti.row0 = off[e] + m_blk * TILE_M;
