@@ -45,6 +45,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "tc_common.cuh"
 
@@ -378,8 +379,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             tc_fence_after();
 
             // one chunk of CW output columns from the accumulator values u (and v):
-            // bias / activation / gate, bf16 pack, staged rows, 128-byte row stores
-            auto emit = [&](int c, const uint32_t (&u)[CW], const uint32_t (&v)[EPI == EPI_SWIGLU ? CW : 1]) {
+            // bias / activation / gate, bf16 pack, staged rows, 128-byte row stores.
+            // hb: whether a bias is added -- a compile-time switch, since the
+            // epilogue's instruction count slows the MMA issue on the SM
+            // sub-partition it shares with the MMA warp (an always-zero bias add
+            // cost 5% of the K = 768 GEMM)
+            const bool has_bias = bias_e != nullptr || (EPI == EPI_SWIGLU && bias3_e != nullptr);
+            auto emit = [&](auto hb, int c, const uint32_t (&u)[CW],
+                            const uint32_t (&v)[EPI == EPI_SWIGLU ? CW : 1]) {
+                constexpr bool HB = decltype(hb)::value;
                 const int col0 = ti.n0 + c * CW;
                 const uint32_t ebuf = ebuf0 + (nchunk & 1u) * (32 * 128);
                 if (TMA_OUT) {   // the store that last read this buffer (two chunks ago) is done with it
@@ -395,7 +403,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         bu[jj] = 0.f;
                         bv[jj] = 0.f;
                     }
-                    if (bias_e && col < p.n_dim) {
+                    if (HB && bias_e && col < p.n_dim) {
                         uint4 bw = __ldg(reinterpret_cast<const uint4*>(bias_e + col));
                         const uint32_t* bp = reinterpret_cast<const uint32_t*>(&bw);
 #pragma unroll
@@ -404,7 +412,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                             bu[2 * h + 1] = bf16hi(bp[h]);
                         }
                     }
-                    if (EPI == EPI_SWIGLU && bias3_e && col < p.n_dim) {
+                    if (HB && EPI == EPI_SWIGLU && bias3_e && col < p.n_dim) {
                         uint4 bw = __ldg(reinterpret_cast<const uint4*>(bias3_e + col));
                         const uint32_t* bp = reinterpret_cast<const uint32_t*>(&bw);
 #pragma unroll
@@ -418,19 +426,26 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 #pragma unroll
                     for (int h = 0; h < 4; ++h) {
                         const int jj = 8 * gi + 2 * h;
-                        float a0 = __uint_as_float(u[jj]) + bu[2 * h];
-                        float a1 = __uint_as_float(u[jj + 1]) + bu[2 * h + 1];
+                        float a0 = __uint_as_float(u[jj]);
+                        float a1 = __uint_as_float(u[jj + 1]);
+                        float v0 = EPI == EPI_SWIGLU ? __uint_as_float(v[EPI == EPI_SWIGLU ? jj : 0]) : 0.f;
+                        float v1 = EPI == EPI_SWIGLU ? __uint_as_float(v[EPI == EPI_SWIGLU ? jj + 1 : 0]) : 0.f;
+                        if (HB) {
+                            a0 += bu[2 * h];
+                            a1 += bu[2 * h + 1];
+                            v0 += bv[2 * h];
+                            v1 += bv[2 * h + 1];
+                        }
                         if (EPI == EPI_SWIGLU) {
                             pre_g[h] = pack_bf16x2(a0, a1);
-                            pre_u[h] = pack_bf16x2(__uint_as_float(v[EPI == EPI_SWIGLU ? jj : 0]) + bv[2 * h],
-                                                   __uint_as_float(v[EPI == EPI_SWIGLU ? jj + 1 : 0]) + bv[2 * h + 1]);
+                            pre_u[h] = pack_bf16x2(v0, v1);
                         }
                         if (EPI == EPI_RELU) {
-                            a0 = fmaxf(a0, 0.f);
-                            a1 = fmaxf(a1, 0.f);
+                            pk[h] = pack_relu_bf16x2(a0, a1);
+                            continue;
                         } else if (EPI == EPI_SWIGLU) {
-                            a0 = silu(a0) * (__uint_as_float(v[EPI == EPI_SWIGLU ? jj : 0]) + bv[2 * h]);
-                            a1 = silu(a1) * (__uint_as_float(v[EPI == EPI_SWIGLU ? jj + 1 : 0]) + bv[2 * h + 1]);
+                            a0 = silu(a0) * v0;
+                            a1 = silu(a1) * v1;
                         } else if (EPI == EPI_SCATTER) {
                             a0 *= g;
                             a1 *= g;
@@ -491,7 +506,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     tmem_ld32(tbase + BN_OUT + c * CW + 32, *reinterpret_cast<uint32_t(*)[32]>(&v[32]));
                     tmem_wait_ld();
                     if (c == BN_OUT / CW - 1) release();
-                    emit(c, u, v);
+                    if (has_bias) emit(std::true_type{}, c, u, v);
+                    else emit(std::false_type{}, c, u, v);
                 }
             } else {
                 // the next chunk's TMEM load is in flight while this chunk is
@@ -511,7 +527,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     } else {
                         release();
                     }
-                    emit(c, cur, none);
+                    if (has_bias) emit(std::true_type{}, c, cur, none);
+                    else emit(std::false_type{}, c, cur, none);
                     if (c + 1 < NC) tmem_wait_ld();
                 }
             }
