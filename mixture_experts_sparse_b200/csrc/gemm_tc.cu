@@ -70,6 +70,7 @@ struct GemmShape {
     static constexpr int STAGES = PAIR ? 6 : 4;
     static constexpr int EPI_BYTES = 2 * 4 * 32 * 128;            // per epilogue warp: 2 x (32 rows x 128 B)
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024;
+    static_assert((STAGES * STAGE_BYTES) % 1024 == 0, "epilogue staging buffers start 1024-byte aligned");
     static constexpr uint32_t IDESC = idesc_bf16_f32(TILE_M, BN);
 };
 
@@ -390,6 +391,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 constexpr bool HB = decltype(hb)::value;
                 const int col0 = ti.n0 + c * CW;
                 const uint32_t ebuf = ebuf0 + (nchunk & 1u) * (32 * 128);
+                // this lane's staged row with its swizzle key in bits 4-6 (ebuf is
+                // 1024-byte aligned): granule gi lands at row_sw ^ (gi << 4)
+                const uint32_t row_sw = ebuf + lane * 128 + ((lane & 7) << 4);
                 if (TMA_OUT) {   // the store that last read this buffer (two chunks ago) is done with it
                     if (lane == 0) bulk_wait_read<1>();
                     __syncwarp();
@@ -457,7 +461,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                         *reinterpret_cast<uint4*>(pr) = make_uint4(pre_g[0], pre_g[1], pre_g[2], pre_g[3]);
                         *reinterpret_cast<uint4*>(pr + p.n_dim) = make_uint4(pre_u[0], pre_u[1], pre_u[2], pre_u[3]);
                     }
-                    const uint32_t dst = ebuf + lane * 128 + ((gi ^ (lane & 7)) << 4);
+                    const uint32_t dst = row_sw ^ (uint32_t)(gi << 4);
                     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(pk[0]), "r"(pk[1]),
                                  "r"(pk[2]), "r"(pk[3])
                                  : "memory");
