@@ -295,10 +295,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     tc_fence_after();
                     issued = true;
                     const uint32_t a_addr = smem_u32(smem + stage * S::STAGE_BYTES);
-                    const uint32_t b_addr = a_addr + A_BYTES;
+                    // the descriptors' address field counts 16-byte units: the next
+                    // 16-wide K slice (32 bytes) of the swizzled rows is +2
+                    const uint64_t a_desc = umma_desc(a_addr), b_desc = umma_desc(a_addr + A_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t ad = umma_desc(a_addr + kk * 32), bd = umma_desc(b_addr + kk * 32);
+                        const uint64_t ad = a_desc + 2 * kk, bd = b_desc + 2 * kk;
                         const uint32_t accf = (kb | kk) != 0 ? 1u : 0u;
                         if (PAIR) umma_f16_pair(d_tmem, ad, bd, S::IDESC, accf);
                         else umma_f16(d_tmem, ad, bd, S::IDESC, accf);

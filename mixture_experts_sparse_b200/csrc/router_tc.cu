@@ -272,9 +272,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                 const uint32_t acc_par = (uint32_t)(p.nbuf == 2 ? ((it >> 1) & 1) : (it & 1));
                 if (!wait_bar(smem_u32(&tempty_bar[acc]), acc_par ^ 1u, w)) break;
                 tc_fence_after();
+                int g = 0, kin = 0;   // K group and k-block inside it (no division on the issue path)
                 for (int kb = 0; kb < nkb; ++kb) {
-                    const int g = kb / p.kb_per_group;
-                    const bool first = kb == g * p.kb_per_group;
+                    const bool first = kin == 0;
                     const uint32_t d_tmem = tmem_base + (uint32_t)((acc * p.groups + g) * S::ACC_COLS);
                     if (!wait_bar(smem_u32(&full_bar[stage]), phase, w)) {
                         ok = false;
@@ -302,6 +302,10 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     if (++stage == S::STAGES) {
                         stage = 0;
                         phase ^= 1u;
+                    }
+                    if (++kin == p.kb_per_group) {
+                        kin = 0;
+                        ++g;
                     }
                 }
                 if (ok) umma_commit_pair(smem_u32(&tfull_bar[acc]), 0x3);
