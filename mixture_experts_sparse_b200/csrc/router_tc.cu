@@ -177,7 +177,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
     __shared__ uint32_t s_tmem;
     __shared__ int s_abort;
     __shared__ int s_hist[NP];
-    __shared__ float s_bias[NP];   // b_r, 0 without a bias, -inf for padding experts
+    __shared__ __align__(16) float s_bias[NP];   // b_r, 0 without a bias, -inf for padding experts
     __shared__ double s_z[128];    // per epilogue thread: sum of lse^2 over its tokens
     __shared__ int s_last;
 
@@ -340,7 +340,13 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             const bool valid = t < p.T;
             float v[NP];   // logits: the bias, then the partial products in a fixed order
 #pragma unroll
-            for (int e = 0; e < NP; ++e) v[e] = s_bias[e];
+            for (int e = 0; e < NP; e += 4) {   // 16-byte broadcast reads
+                const float4 b4 = *reinterpret_cast<const float4*>(&s_bias[e]);
+                v[e] = b4.x;
+                v[e + 1] = b4.y;
+                v[e + 2] = b4.z;
+                v[e + 3] = b4.w;
+            }
             const uint32_t tbase =
                 tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * p.groups * S::ACC_COLS);
             for (int g = 0; g < p.groups; ++g) {   // partial logits of the K groups (and W parts), in order
@@ -375,8 +381,9 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             }
             // v now holds exp(h - max) = 2^((h - max) log2 e); padding experts
             // hold -inf (their bias), so their terms are 0
+            const float m_l2 = m * kLog2e;   // exp(h - max) = 2^(h log2 e - max log2 e), one FMA per expert
 #pragma unroll
-            for (int e = 0; e < NP; ++e) v[e] = fast_exp2((v[e] - m) * kLog2e);
+            for (int e = 0; e < NP; ++e) v[e] = fast_exp2(fmaf(v[e], kLog2e, -m_l2));
             const float s = tree_sum(v);
             const float inv = valid ? 1.f / s : 0.f;
             if (valid) {
