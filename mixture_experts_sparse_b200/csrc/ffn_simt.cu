@@ -6,7 +6,7 @@
 // H = act(A W1[e]^T + b1[e]) (or the SwiGLU product), then Y = H W2[e]^T + b2[e]
 // ("From Switch Transformer to GLaM", FFN(x) = W2 s(W1 x); CMU 10-423 Lecture
 // 16, section 2.3, SwiGLU expert).  A 64x64 output tile per block, 4x4 per
-// thread, K staged through shared memory in chunks of 16.  Grid = (m-tiles up to
+// thread, K staged through shared memory in chunks of 32.  Grid = (m-tiles up to
 // the capacity C, n-tiles, experts); blocks past an expert's kept rows return.
 #include "common.cuh"
 
@@ -16,7 +16,7 @@ namespace moe {
 namespace {
 
 constexpr int TS = 64;
-constexpr int KC = 16;
+constexpr int KC = 32;
 
 enum { SIMT_RELU = 0, SIMT_SWIGLU = 1, SIMT_BIAS = 2 };
 

@@ -22,9 +22,8 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kDK = 16;   // reduction chunk staged in shared memory
-constexpr int kTT = 4;    // tokens per thread
 
-template <int TE, int EG>
+template <int TE, int EG, int kTT>   // kTT: tokens per thread
 struct RouterShape {
     static constexpr int TG = 8 / EG;            // token groups (warps per expert group)
     static constexpr int TB = TG * 32 * kTT;     // tokens per block
@@ -43,13 +42,13 @@ __device__ __forceinline__ void argmax_merge(float& v, int& i, float ov, int oi)
     }
 }
 
-template <typename XT, int TE, int EG>
+template <typename XT, int TE, int EG, int kTT>
 __global__ void __launch_bounds__(kThreads)
 router_kernel(const XT* __restrict__ x, const float* __restrict__ w_r, const float* __restrict__ b_r,
               int64_t T, int d, int N, int k,
               int32_t* __restrict__ idx, float* __restrict__ gate, float* __restrict__ probs,
               int32_t* __restrict__ part_cnt, float* __restrict__ part_psum, double* __restrict__ part_z) {
-    using S = RouterShape<TE, EG>;
+    using S = RouterShape<TE, EG, kTT>;
     constexpr int VEC = 16 / sizeof(XT);          // elements per 16-byte load
     constexpr int PARTS = kDK / VEC;              // 16-byte loads per row chunk
     constexpr int NL = S::TB * PARTS / kThreads;  // 16-byte loads per thread per chunk
@@ -392,15 +391,15 @@ aux_finalize_kernel(const double* __restrict__ part_z, double* __restrict__ z,
     if (z && tid < 32) z_reduce_warp(part_z, nblk, T, z);
 }
 
-template <typename XT, int TE, int EG>
+template <typename XT, int TE, int EG, int kTT>
 cudaError_t launch_router_t(const RouterArgs& a, cudaStream_t s) {
-    using S = RouterShape<TE, EG>;
+    using S = RouterShape<TE, EG, kTT>;
     const int nblk = (int)((a.T + S::TB - 1) / S::TB);
     const size_t smem = sizeof(float) * S::SMEM_FLOATS;
-    auto kern = router_kernel<XT, TE, EG>;
+    auto kern = router_kernel<XT, TE, EG, kTT>;
     cudaError_t err = once_per_device(reinterpret_cast<const void*>(kern), [](const void* k) {
         return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    (int)(sizeof(float) * RouterShape<TE, EG>::SMEM_FLOATS));
+                                    (int)(sizeof(float) * RouterShape<TE, EG, kTT>::SMEM_FLOATS));
     });
     if (err != cudaSuccess) return err;
     if (nblk > 0) {
@@ -412,23 +411,38 @@ cudaError_t launch_router_t(const RouterArgs& a, cudaStream_t s) {
     return launch_aux_finalize(a.part_z, a.z, a.part_cnt, a.part_psum, nblk, a.N, a.T, a.alpha, a.f, a.P, a.aux, s);
 }
 
+// Few tokens (fewer than 64 blocks of the four-tokens-per-thread shape): one
+// token per thread and 64- or 128-token blocks, so the work spreads over more
+// SMs (the 512-token fp32 layer: 4 blocks instead of 1).
+bool small_batch(int64_t T, int N) {
+    const int64_t tb = N <= 8 ? RouterShape<8, 1, 4>::TB : RouterShape<16, 1, 4>::TB;
+    return (T + tb - 1) / tb < 64;
+}
+
 template <typename XT>
 cudaError_t launch_router_x(const RouterArgs& a, cudaStream_t s) {
-    if (a.N <= 8) return launch_router_t<XT, 8, 1>(a, s);
-    if (a.N <= 16) return launch_router_t<XT, 16, 1>(a, s);
-    if (a.N <= 32) return launch_router_t<XT, 16, 2>(a, s);
-    if (a.N <= 64) return launch_router_t<XT, 16, 4>(a, s);
-    return launch_router_t<XT, 16, 8>(a, s);
+    if (small_batch(a.T, a.N)) {
+        if (a.N <= 8) return launch_router_t<XT, 4, 2, 1>(a, s);
+        if (a.N <= 16) return launch_router_t<XT, 4, 4, 1>(a, s);
+        if (a.N <= 32) return launch_router_t<XT, 8, 4, 1>(a, s);
+    }
+    if (a.N <= 8) return launch_router_t<XT, 8, 1, 4>(a, s);
+    if (a.N <= 16) return launch_router_t<XT, 16, 1, 4>(a, s);
+    if (a.N <= 32) return launch_router_t<XT, 16, 2, 4>(a, s);
+    if (a.N <= 64) return launch_router_t<XT, 16, 4, 4>(a, s);
+    return launch_router_t<XT, 16, 8, 4>(a, s);
 }
 
 }  // namespace
 
 int router_blocks(int64_t T, int N) {
     int tb;
-    if (N <= 16) tb = RouterShape<16, 1>::TB;
-    else if (N <= 32) tb = RouterShape<16, 2>::TB;
-    else if (N <= 64) tb = RouterShape<16, 4>::TB;
-    else tb = RouterShape<16, 8>::TB;
+    if (small_batch(T, N) && N <= 32) tb = N <= 8 ? RouterShape<4, 2, 1>::TB : (N <= 16 ? RouterShape<4, 4, 1>::TB : RouterShape<8, 4, 1>::TB);
+    else if (N <= 8) tb = RouterShape<8, 1, 4>::TB;
+    else if (N <= 16) tb = RouterShape<16, 1, 4>::TB;
+    else if (N <= 32) tb = RouterShape<16, 2, 4>::TB;
+    else if (N <= 64) tb = RouterShape<16, 4, 4>::TB;
+    else tb = RouterShape<16, 8, 4>::TB;
     return (int)((T + tb - 1) / tb);
 }
 
