@@ -297,6 +297,41 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             const BwTile ti = bw_decode<MODE>(tile, s_prefix, s_off, N, ntm, ntn);
             const int acc = it & 1;
             const uint32_t acc_par = (uint32_t)((it >> 1) & 1);
+            // dU epilogues read this row's forward values (H, or the SwiGLU
+            // pre-activations) for each 32-column chunk: they are loaded one chunk
+            // ahead (the first before the accumulator wait), so the global-load
+            // latency overlaps the previous chunk instead of stalling every chunk
+            constexpr bool DU = MODE == BW_DU_RELU || MODE == BW_DU_SWIGLU;
+            constexpr int NPF = MODE == BW_DU_SWIGLU ? 8 : (MODE == BW_DU_RELU ? 4 : 1);   // 16-byte loads per chunk
+            const bool row_ok = DU && r_in < ti.rows;
+            const int64_t r_du = (int64_t)ti.row0 + r_in;
+            uint4 fv[NPF], fnext[NPF];
+            auto fetch_fwd = [&](int c, uint4 (&dst)[NPF]) {
+#pragma unroll
+                for (int i = 0; i < NPF; ++i) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+                if constexpr (DU) {
+                    if (!row_ok) return;
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int col = ti.n0 + c * 32 + 8 * i;
+                        if (col >= p.n_dim) break;
+                        if (MODE == BW_DU_RELU) {
+                            dst[i] = __ldg(reinterpret_cast<const uint4*>(p.h + r_du * p.n_dim + col));
+                        } else {
+                            const __nv_bfloat16* pre = p.pre + r_du * (int64_t)(2 * p.n_dim);
+                            dst[i] = __ldg(reinterpret_cast<const uint4*>(pre + col));
+                            dst[(4 + i) % NPF] = __ldg(reinterpret_cast<const uint4*>(pre + p.n_dim + col));
+                        }
+                    }
+                }
+            };
+            if (DU) fetch_fwd(0, fnext);
+            // dx rows: the destination row (the token, when scattering) before the wait
+            int64_t dx_row = 0;
+            if (MODE == BW_DX && r_in < ti.rows) {
+                const int64_t r = (int64_t)ti.row0 + r_in;
+                dx_row = p.row_token ? (int64_t)p.row_token[r] : r;
+            }
             const bool got = wait_bar(smem_u32(&tfull_bar[acc]), acc_par, w);
             if (!__all_sync(0xffffffffu, got)) break;
             tc_fence_after();
@@ -306,6 +341,11 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             for (int c = 0; c < BW_BN / 32; ++c) {
                 uint32_t v[32];
                 tmem_ld32(tbase + c * 32, v);
+                if (DU) {
+#pragma unroll
+                    for (int i = 0; i < NPF; ++i) fv[i] = fnext[i];
+                    if (c + 1 < BW_BN / 32) fetch_fwd(c + 1, fnext);
+                }
                 tmem_wait_ld();
                 const int col0 = ti.n0 + c * 32;
                 if (MODE == BW_WGT) {
@@ -327,8 +367,7 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 if (r_in >= ti.rows) continue;
                 const int64_t r = (int64_t)ti.row0 + r_in;
                 if constexpr (MODE == BW_DX) {
-                    const int64_t orow = p.row_token ? (int64_t)p.row_token[r] : r;
-                    float* dst = p.out + orow * p.n_dim + col0;
+                    float* dst = p.out + dx_row * p.n_dim + col0;
 #pragma unroll
                     for (int j = 0; j < 32; j += 4)
                         if (col0 + j < p.n_dim)
@@ -343,8 +382,7 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     if (col >= p.n_dim) break;
                     uint32_t pk[4], pk2[4];
                     if (MODE == BW_DU_RELU) {
-                        const uint4 hv = *reinterpret_cast<const uint4*>(p.h + r * p.n_dim + col);
-                        const uint32_t* hw = reinterpret_cast<const uint32_t*>(&hv);
+                        const uint32_t* hw = reinterpret_cast<const uint32_t*>(&fv[(j0 / 8) % NPF]);
 #pragma unroll
                         for (int h2 = 0; h2 < 4; ++h2) {
                             const float a0 = bf16lo(hw[h2]) > 0.f ? __uint_as_float(v[j0 + 2 * h2]) : 0.f;
@@ -353,11 +391,8 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         }
                         *reinterpret_cast<uint4*>(p.du + r * p.n_dim + col) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
                     } else {
-                        const __nv_bfloat16* pre = p.pre + r * (int64_t)(2 * p.n_dim);
-                        const uint4 gv = *reinterpret_cast<const uint4*>(pre + col);
-                        const uint4 uv = *reinterpret_cast<const uint4*>(pre + p.n_dim + col);
-                        const uint32_t* gw = reinterpret_cast<const uint32_t*>(&gv);
-                        const uint32_t* uw = reinterpret_cast<const uint32_t*>(&uv);
+                        const uint32_t* gw = reinterpret_cast<const uint32_t*>(&fv[(j0 / 8) % NPF]);
+                        const uint32_t* uw = reinterpret_cast<const uint32_t*>(&fv[(4 + j0 / 8) % NPF]);
 #pragma unroll
                         for (int h2 = 0; h2 < 4; ++h2) {
                             float dgo[2], duo[2];
