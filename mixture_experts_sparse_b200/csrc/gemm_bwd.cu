@@ -37,7 +37,11 @@ constexpr int BW_STAGES = 4;
 constexpr int BW_A_BYTES = BW_BM * BW_BK * 2;   // 16 KB
 constexpr int BW_B_BYTES = BW_BN * BW_BK * 2;   // 32 KB
 constexpr int BW_STAGE_BYTES = BW_A_BYTES + BW_B_BYTES;
-constexpr int BW_SMEM = BW_STAGES * BW_STAGE_BYTES + 1024;
+// weight-gradient epilogue: per epilogue warp two staging buffers of 32 rows x
+// 128 bytes (32 fp32 columns), written to dW with TMA tensor stores
+constexpr int BW_EPI_BYTES = 4 * 2 * 32 * 128;
+constexpr int BW_SMEM = BW_STAGES * BW_STAGE_BYTES + BW_EPI_BYTES + 1024;
+static_assert((BW_STAGES * BW_STAGE_BYTES) % 1024 == 0, "staging buffers 1024-byte aligned");
 constexpr int BW_TMEM_COLS = 512;
 constexpr int MN_BOX = 64 * BW_BK * 2;          // one MN-major box: 64 MN x 64 K rows = 8 KB
 
@@ -55,6 +59,8 @@ struct BwdParams {
     float* out;               // BW_DX: dx rows (scatter: [T, n_dim] by row_token; else [R, n_dim]);
                               // BW_WGT: dW [N, m_dim, n_dim]
     const int32_t* row_token; // BW_DX scatter (top-1)
+    int mn3;                  // bit 0: tmA is a blocked 3-D MN map (2 blocks per load),
+                              // bit 1: tmB and tmB2 are (4 blocks per load)
     int32_t* status;
     long long limit_ns;
 };
@@ -96,7 +102,8 @@ __device__ __forceinline__ float sigmoidf_(float z) { return __fdividef(1.f, 1.f
 template <int MODE>
 __global__ void __launch_bounds__(BW_THREADS, 1)
 bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const __grid_constant__ CUtensorMap tmB2, const BwdParams p) {
+                const __grid_constant__ CUtensorMap tmB2, const __grid_constant__ CUtensorMap tmOut,
+                const BwdParams p) {
     constexpr bool A_MN = MODE == BW_WGT;
     constexpr uint32_t IDESC = idesc_bf16_f32_major(BW_BM, BW_BN, A_MN, true);
     extern __shared__ uint8_t smem_raw[];
@@ -198,10 +205,18 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     mbar_expect_tx(fb, BW_STAGE_BYTES);
                     if (MODE == BW_WGT) {
                         const int kr = ti.k_row0 + kb * BW_BK;   // rows of the expert (K)
+                        if (p.mn3 & 1) {
+                            tma_load_3d(a_dst, &tmA, fb, 0, kr, ti.m0 / 64);
+                        } else {
 #pragma unroll
-                        for (int j = 0; j < 2; ++j) tma_load_2d(a_dst + j * MN_BOX, &tmA, fb, ti.m0 + 64 * j, kr);
+                            for (int j = 0; j < 2; ++j) tma_load_2d(a_dst + j * MN_BOX, &tmA, fb, ti.m0 + 64 * j, kr);
+                        }
+                        if (p.mn3 & 2) {
+                            tma_load_3d(b_dst, &tmB, fb, 0, kr, ti.n0 / 64);
+                        } else {
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) tma_load_2d(b_dst + j * MN_BOX, &tmB, fb, ti.n0 + 64 * j, kr);
+                            for (int j = 0; j < 4; ++j) tma_load_2d(b_dst + j * MN_BOX, &tmB, fb, ti.n0 + 64 * j, kr);
+                        }
                     } else {
                         tma_load_2d(a_dst, &tmA, fb, kb * BW_BK, ti.row0);
                         // B = weights [N_exp * K rows][n cols]; two tensors split at k_split
@@ -209,9 +224,13 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                         const int kk = second ? kb * BW_BK - p.k_split : kb * BW_BK;
                         const int kdim_b = p.k_split > 0 ? p.k_split : p.k_dim;
                         const CUtensorMap* bm = second ? &tmB2 : &tmB;
+                        if (p.mn3 & 2) {
+                            tma_load_3d(b_dst, bm, fb, 0, ti.e * kdim_b + kk, ti.n0 / 64);
+                        } else {
 #pragma unroll
-                        for (int j = 0; j < 4; ++j)
-                            tma_load_2d(b_dst + j * MN_BOX, bm, fb, ti.n0 + 64 * j, ti.e * kdim_b + kk);
+                            for (int j = 0; j < 4; ++j)
+                                tma_load_2d(b_dst + j * MN_BOX, bm, fb, ti.n0 + 64 * j, ti.e * kdim_b + kk);
+                        }
                     }
                     last_par[stage] = (int)phase;
                     if (++stage == BW_STAGES) {
@@ -292,6 +311,8 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
         // ---------------- epilogue (warps 2..5): thread = accumulator row ----------------
         const int q = warp & 3;
         const int r_in = q * 32 + lane;
+        const uint32_t ebuf0 = smem_u32(smem + BW_STAGES * BW_STAGE_BYTES + q * 2 * 32 * 128);
+        uint32_t nchunk = 0;   // chunks staged so far (buffer = nchunk & 1; one bulk group each)
         int it = 0;
         for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
             const BwTile ti = bw_decode<MODE>(tile, s_prefix, s_off, N, ntm, ntn);
@@ -349,19 +370,47 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 tmem_wait_ld();
                 const int col0 = ti.n0 + c * 32;
                 if (MODE == BW_WGT) {
-                    const int m = ti.m0 + r_in;
-                    if (m < p.m_dim) {
-                        float* dst = p.out + ((int64_t)ti.e * p.m_dim + m) * p.n_dim + col0;
+                    // the warp's 32 rows x 32 fp32 columns go through a swizzled
+                    // staging buffer: one TMA store when all 32 rows are the
+                    // expert's, else 128-byte row pieces (8 lanes per row)
+                    const uint32_t ebuf = ebuf0 + (nchunk & 1u) * (32 * 128);
+                    const uint32_t row_sw = ebuf + lane * 128 + ((lane & 7) << 4);
+                    if (lane == 0) bulk_wait_read<1>();   // the store that last read this buffer is done
+                    __syncwarp();
 #pragma unroll
-                        for (int j = 0; j < 32; j += 4) {
-                            if (col0 + j < p.n_dim) {
-                                float4 o = empty_k ? make_float4(0.f, 0.f, 0.f, 0.f)
-                                                   : make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]),
-                                                                 __uint_as_float(v[j + 2]), __uint_as_float(v[j + 3]));
-                                *reinterpret_cast<float4*>(dst + j) = o;
-                            }
+                    for (int g = 0; g < 8; ++g) {
+                        const uint32_t x0 = empty_k ? 0u : v[4 * g], x1 = empty_k ? 0u : v[4 * g + 1];
+                        const uint32_t x2 = empty_k ? 0u : v[4 * g + 2], x3 = empty_k ? 0u : v[4 * g + 3];
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_sw ^ (uint32_t)(g << 4)),
+                                     "r"(x0), "r"(x1), "r"(x2), "r"(x3)
+                                     : "memory");
+                    }
+                    const int wrow0 = ti.m0 + q * 32;   // the warp's first row
+                    if (wrow0 + 32 <= p.m_dim) {
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) tma_store_2d(&tmOut, ebuf, col0, ti.e * p.m_dim + wrow0);
+                    } else {
+                        __syncwarp();
+                        const int gi = lane & 7;
+                        const bool col_ok = col0 + 4 * gi < p.n_dim;
+#pragma unroll
+                        for (int k4 = 0; k4 < 8; ++k4) {
+                            const int r = 4 * k4 + (lane >> 3);
+                            uint4 val;
+                            const uint32_t srcp = ebuf + r * 128 + ((gi ^ (r & 7)) << 4);
+                            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                         : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                                         : "r"(srcp)
+                                         : "memory");
+                            if (wrow0 + r < p.m_dim && col_ok)
+                                *reinterpret_cast<uint4*>(p.out + ((int64_t)ti.e * p.m_dim + wrow0 + r) * p.n_dim +
+                                                          col0 + 4 * gi) = val;
                         }
                     }
+                    if (lane == 0) bulk_commit();
+                    __syncwarp();
+                    ++nchunk;
                     continue;
                 }
                 if (r_in >= ti.rows) continue;
@@ -418,6 +467,7 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             tc_fence_before();
             mbar_arrive_relaxed(smem_u32(&tempty_bar[acc]));
         }
+        if (MODE == BW_WGT && lane == 0) bulk_wait_all();   // this warp's TMA stores have landed
     }
 
     tc_fence_before();
@@ -498,8 +548,8 @@ dx_zero_dropped_kernel(const uint8_t* __restrict__ drop, int64_t T, int d, float
 }
 
 template <int MODE>
-cudaError_t run_bwd(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const BwdParams& p,
-                    cudaStream_t s) {
+cudaError_t run_bwd(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& b2, const CUtensorMap& o,
+                    const BwdParams& p, cudaStream_t s) {
     int sms = 0;
     cudaError_t err = device_sm_count(&sms);
     if (err != cudaSuccess) return err;
@@ -507,7 +557,40 @@ cudaError_t run_bwd(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMa
         return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, BW_SMEM);
     });
     if (err != cudaSuccess) return err;
-    return launch_k(bwd_gemm_kernel<MODE>, dim3((unsigned)sms), dim3(BW_THREADS), BW_SMEM, s, 1, a, b, b2, p);
+    return launch_k(bwd_gemm_kernel<MODE>, dim3((unsigned)sms), dim3(BW_THREADS), BW_SMEM, s, 1, a, b, b2, o, p);
+}
+
+// dW [groups * m, n] fp32 as the weight-gradient epilogue's TMA store target:
+// boxes of 32 rows x 32 columns (128 bytes), 128-byte swizzle
+bool wgt_out_map(CUtensorMap* m, const float* out, int64_t rows, int n) {
+    using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+    static EncodeFn enc = [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return (EncodeFn) nullptr;
+        return reinterpret_cast<EncodeFn>(ptr);
+    }();
+    if (!enc || out == nullptr || n % 4 != 0 || rows < 1) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)n, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)n * 4};
+    cuuint32_t box[2] = {32u, 32u};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(out), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// An MN-major operand: the blocked 3-D map (one TMA load of `blocks` 64-column
+// blocks per stage) when its shape allows, else the 2-D map (one load per
+// block); *blocked says which.
+bool mn_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, int64_t row_stride, int blocks,
+            bool* blocked) {
+    *blocked = make_map_bf16_mn_blocks(m, base, rows, cols, row_stride, BW_BK, blocks);
+    return *blocked || make_map_bf16_strided(m, base, rows, cols, row_stride, BW_BK);
 }
 
 }  // namespace
@@ -521,9 +604,10 @@ cudaError_t run_bwd(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMa
 cudaError_t launch_tc_rows_f32(const void* A, int64_t rows, int K, const void* B, int n, const int32_t* offsets,
                                float* out, int32_t* status, cudaStream_t s) {
     CUtensorMap ma, mb;
-    if (!make_map_bf16(&ma, A, rows, K, BW_BM) || !make_map_bf16_mn(&mb, B, K, n, BW_BK))
-        return cudaErrorInvalidValue;
+    bool bb = false;
+    if (!make_map_bf16(&ma, A, rows, K, BW_BM) || !mn_map(&mb, B, K, n, n, 4, &bb)) return cudaErrorInvalidValue;
     BwdParams p{};
+    p.mn3 = bb ? 2 : 0;
     p.offsets = offsets;
     p.N = 1;
     p.n_dim = n;
@@ -531,15 +615,16 @@ cudaError_t launch_tc_rows_f32(const void* A, int64_t rows, int K, const void* B
     p.out = out;
     p.status = status;
     p.limit_ns = kWaitLimitNs;
-    return run_bwd<BW_DX>(ma, mb, mb, p, s);
+    return run_bwd<BW_DX>(ma, mb, mb, ma, p, s);
 }
 
 cudaError_t launch_tc_weights_f32(const void* A, int64_t rows, int m, const void* B, int n, const int32_t* offsets,
                                   int groups, float* out, int32_t* status, cudaStream_t s) {
     CUtensorMap ma, mb;
-    if (!make_map_bf16_mn(&ma, A, rows, m, BW_BK) || !make_map_bf16_mn(&mb, B, rows, n, BW_BK))
-        return cudaErrorInvalidValue;
+    bool ba = false, bb = false;
+    if (!mn_map(&ma, A, rows, m, m, 2, &ba) || !mn_map(&mb, B, rows, n, n, 4, &bb)) return cudaErrorInvalidValue;
     BwdParams p{};
+    p.mn3 = (ba ? 1 : 0) | (bb ? 2 : 0);
     p.offsets = offsets;
     p.N = groups;
     p.m_dim = m;
@@ -547,7 +632,9 @@ cudaError_t launch_tc_weights_f32(const void* A, int64_t rows, int m, const void
     p.out = out;
     p.status = status;
     p.limit_ns = kWaitLimitNs;
-    return run_bwd<BW_WGT>(ma, mb, mb, p, s);
+    CUtensorMap mo;
+    if (!wgt_out_map(&mo, out, (int64_t)groups * m, n)) return cudaErrorInvalidValue;
+    return run_bwd<BW_WGT>(ma, mb, mb, mo, p, s);
 }
 
 cudaError_t launch_expert_backward_tc(const BwdArgs& a, cudaStream_t s) {
@@ -582,9 +669,11 @@ cudaError_t launch_expert_backward_tc(const BwdArgs& a, cudaStream_t s) {
         return err;
     CUtensorMap m_dy, m_w2, m_du, m_w1, m_w3, m_xe, m_h, m_a2, m_b2;
     // 3. dA = dY W2 -> dU (dG | dUp)
-    if (!make_map_bf16(&m_dy, a.dy, R, d, BW_BM) || !make_map_bf16_mn(&m_w2, a.w2, (int64_t)N * d, dff, BW_BK))
+    bool bw2 = false;
+    if (!make_map_bf16(&m_dy, a.dy, R, d, BW_BM) || !mn_map(&m_w2, a.w2, (int64_t)N * d, dff, dff, 4, &bw2))
         return cudaErrorInvalidValue;
     BwdParams p{};
+    p.mn3 = bw2 ? 2 : 0;
     p.offsets = a.offsets;
     p.N = N;
     p.status = &a.hdr->status;
@@ -594,20 +683,28 @@ cudaError_t launch_expert_backward_tc(const BwdArgs& a, cudaStream_t s) {
     p.h = reinterpret_cast<const __nv_bfloat16*>(a.h);
     p.pre = reinterpret_cast<const __nv_bfloat16*>(a.pre);
     p.du = reinterpret_cast<__nv_bfloat16*>(a.du);
-    err = sw ? run_bwd<BW_DU_SWIGLU>(m_dy, m_w2, m_w2, p, s) : run_bwd<BW_DU_RELU>(m_dy, m_w2, m_w2, p, s);
+    err = sw ? run_bwd<BW_DU_SWIGLU>(m_dy, m_w2, m_w2, m_dy, p, s) : run_bwd<BW_DU_RELU>(m_dy, m_w2, m_w2, m_dy, p, s);
     if (err != cudaSuccess) return err;
     // 4. dx rows = dU W1 (+ dUp W3): K = d_ff (2 d_ff for SwiGLU, W3 for the second half)
     const int kdu = sw ? 2 * dff : dff;
-    if (!make_map_bf16(&m_du, a.du, R, kdu, BW_BM) || !make_map_bf16_mn(&m_w1, a.w1, (int64_t)N * dff, d, BW_BK))
+    bool bw1 = false, bw3 = false;
+    if (!make_map_bf16(&m_du, a.du, R, kdu, BW_BM) || !mn_map(&m_w1, a.w1, (int64_t)N * dff, d, d, 4, &bw1))
         return cudaErrorInvalidValue;
-    if (sw && !make_map_bf16_mn(&m_w3, a.w3, (int64_t)N * dff, d, BW_BK)) return cudaErrorInvalidValue;
+    if (sw && !mn_map(&m_w3, a.w3, (int64_t)N * dff, d, d, 4, &bw3)) return cudaErrorInvalidValue;
+    if (sw && bw1 != bw3) {   // both B tensors of one launch in the same form
+        bw1 = bw3 = false;
+        if (!make_map_bf16_mn(&m_w1, a.w1, (int64_t)N * dff, d, BW_BK) ||
+            !make_map_bf16_mn(&m_w3, a.w3, (int64_t)N * dff, d, BW_BK))
+            return cudaErrorInvalidValue;
+    }
     BwdParams px = p;
+    px.mn3 = bw1 ? 2 : 0;
     px.n_dim = d;
     px.k_dim = kdu;
     px.k_split = sw ? dff : 0;
     px.out = a.top1_scatter ? a.dx : a.dxe;
     px.row_token = a.top1_scatter ? a.row_token : nullptr;
-    if ((err = run_bwd<BW_DX>(m_du, m_w1, sw ? m_w3 : m_w1, px, s)) != cudaSuccess) return err;
+    if ((err = run_bwd<BW_DX>(m_du, m_w1, sw ? m_w3 : m_w1, m_du, px, s)) != cudaSuccess) return err;
     if (a.top1_scatter) {
         if (a.T > 0 && (err = launch_k(dx_zero_dropped_kernel, dim3((unsigned)((a.T + 7) / 8)), dim3(256), 0, s, 1,
                                        a.drop, a.T, d, a.dx)) != cudaSuccess)
@@ -619,29 +716,41 @@ cudaError_t launch_expert_backward_tc(const BwdArgs& a, cudaStream_t s) {
             return err;
     }
     // 5. weight gradients: dW1 = dU^T X (dW3 = dUp^T X), dW2 = dY^T A
-    if (!make_map_bf16_mn(&m_xe, a.xe, R, d, BW_BK) || !make_map_bf16_mn(&m_h, a.h, R, dff, BW_BK))
+    bool bxe = false, bh = false, ba2 = false;
+    if (!mn_map(&m_xe, a.xe, R, d, d, 4, &bxe) || !mn_map(&m_h, a.h, R, dff, dff, 4, &bh))
         return cudaErrorInvalidValue;
     BwdParams pw = p;
     pw.m_dim = dff;
     pw.n_dim = d;
     // dU (dG): the first d_ff columns of each row of the du tensor (row stride kdu)
-    if (!make_map_bf16_strided(&m_a2, a.du, R, dff, kdu, BW_BK)) return cudaErrorInvalidValue;
+    if (!mn_map(&m_a2, a.du, R, dff, kdu, 2, &ba2)) return cudaErrorInvalidValue;
     pw.out = a.dw1;
-    if (a.dw1 && (err = run_bwd<BW_WGT>(m_a2, m_xe, m_xe, pw, s)) != cudaSuccess) return err;
+    pw.mn3 = (ba2 ? 1 : 0) | (bxe ? 2 : 0);
+    CUtensorMap m_o;
+    if (a.dw1) {
+        if (!wgt_out_map(&m_o, a.dw1, (int64_t)N * dff, d)) return cudaErrorInvalidValue;
+        if ((err = run_bwd<BW_WGT>(m_a2, m_xe, m_xe, m_o, pw, s)) != cudaSuccess) return err;
+    }
     if (sw && a.dw3) {   // dUp: columns [d_ff, 2 d_ff)
-        if (!make_map_bf16_strided(&m_b2, reinterpret_cast<const __nv_bfloat16*>(a.du) + dff, R, dff, kdu, BW_BK))
+        bool bb2 = false;
+        if (!mn_map(&m_b2, reinterpret_cast<const __nv_bfloat16*>(a.du) + dff, R, dff, kdu, 2, &bb2))
             return cudaErrorInvalidValue;
         pw.out = a.dw3;
-        if ((err = run_bwd<BW_WGT>(m_b2, m_xe, m_xe, pw, s)) != cudaSuccess) return err;
+        pw.mn3 = (bb2 ? 1 : 0) | (bxe ? 2 : 0);
+        if (!wgt_out_map(&m_o, a.dw3, (int64_t)N * dff, d)) return cudaErrorInvalidValue;
+        if ((err = run_bwd<BW_WGT>(m_b2, m_xe, m_xe, m_o, pw, s)) != cudaSuccess) return err;
     }
     if (a.dw2) {
         CUtensorMap m_dy_mn;
-        if (!make_map_bf16_mn(&m_dy_mn, a.dy, R, d, BW_BK)) return cudaErrorInvalidValue;
+        bool bdy = false;
+        if (!mn_map(&m_dy_mn, a.dy, R, d, d, 2, &bdy)) return cudaErrorInvalidValue;
         BwdParams p2 = p;
         p2.m_dim = d;
         p2.n_dim = dff;
         p2.out = a.dw2;
-        if ((err = run_bwd<BW_WGT>(m_dy_mn, m_h, m_h, p2, s)) != cudaSuccess) return err;
+        p2.mn3 = (bdy ? 1 : 0) | (bh ? 2 : 0);
+        if (!wgt_out_map(&m_o, a.dw2, (int64_t)N * d, dff)) return cudaErrorInvalidValue;
+        if ((err = run_bwd<BW_WGT>(m_dy_mn, m_h, m_h, m_o, p2, s)) != cudaSuccess) return err;
     }
     // 6. bias gradients
     const dim3 cs_block(256);

@@ -656,6 +656,21 @@ bool tc::make_map_bf16_mn(CUtensorMap* map, const void* base, int64_t rows, int6
     return make_map_bf16(map, base, rows, cols, box_rows);   // the same box shape: 64 inner elements x rows
 }
 
+bool tc::make_map_bf16_mn_blocks(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t row_stride,
+                                 int box_rows, int blocks) {
+    if (cols % 64 != 0 || row_stride < cols || blocks < 1 || blocks > 8) return false;
+    EncodeFn enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {64u, (cuuint64_t)rows, (cuuint64_t)(cols / 64)};
+    cuuint64_t strides[2] = {(cuuint64_t)row_stride * 2, 128u};
+    cuuint32_t box[3] = {64u, (cuuint32_t)box_rows, (cuuint32_t)blocks};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 // Stage 1 + stage 2 of the bf16 expert FFN on the tensor cores, both
 // on CTA pairs unless MOE_B200_GEMM=single.
 cudaError_t launch_expert_ffn_tc(const FfnArgs& a, cudaStream_t s) {

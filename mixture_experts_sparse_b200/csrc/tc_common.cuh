@@ -78,6 +78,15 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
         : "memory");
 }
 
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, uint32_t bar, int c0, int c1,
+                                            int c2) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+        "[%2];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+
 // TMA store of a 2-D box from shared memory (bulk-group completion), and the
 // bulk-group bookkeeping of the issuing thread.
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int c0, int c1) {
@@ -212,6 +221,14 @@ bool make_map_bf16(CUtensorMap* map, const void* base, int64_t rows, int64_t k, 
 // host: 2-D bf16 tensor [rows, cols] (cols contiguous) read as an MN-major
 // operand: box = 64 cols x box_rows rows, 128-byte swizzle
 bool make_map_bf16_mn(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int box_rows);
+// host: the same operand as a 3-D view [cols / 64 blocks][rows][64]: one box is
+// `blocks` adjacent 64-column blocks x box_rows rows, each block landing as its
+// own swizzled 64 x box_rows tile, box_rows x 128 bytes after the previous one
+// -- one TMA load where the 2-D map needs `blocks`.  Rows are row_stride
+// elements apart.  Only for cols a multiple of 64 (else false, as when the
+// driver rejects the view)
+bool make_map_bf16_mn_blocks(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t row_stride,
+                             int box_rows, int blocks);
 // host: the same over the first `cols` columns of rows `row_stride` elements apart
 bool make_map_bf16_strided(CUtensorMap* map, const void* base, int64_t rows, int64_t cols, int64_t row_stride,
                            int box_rows);
