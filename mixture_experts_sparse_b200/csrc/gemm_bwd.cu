@@ -37,8 +37,8 @@ constexpr int BW_STAGES = 4;
 constexpr int BW_A_BYTES = BW_BM * BW_BK * 2;   // 16 KB
 constexpr int BW_B_BYTES = BW_BN * BW_BK * 2;   // 32 KB
 constexpr int BW_STAGE_BYTES = BW_A_BYTES + BW_B_BYTES;
-// weight-gradient epilogue: per epilogue warp two staging buffers of 32 rows x
-// 128 bytes (32 fp32 columns), written to dW with TMA tensor stores
+// fp32 epilogues (weight gradients, dx): per epilogue warp two staging buffers
+// of 32 rows x 128 bytes (32 fp32 columns), written out with TMA tensor stores
 constexpr int BW_EPI_BYTES = 4 * 2 * 32 * 128;
 constexpr int BW_SMEM = BW_STAGES * BW_STAGE_BYTES + BW_EPI_BYTES + 1024;
 static_assert((BW_STAGES * BW_STAGE_BYTES) % 1024 == 0, "staging buffers 1024-byte aligned");
@@ -347,12 +347,18 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 }
             };
             if (DU) fetch_fwd(0, fnext);
-            // dx rows: the destination row (the token, when scattering) before the wait
-            int64_t dx_row = 0;
+            // dx rows: the destination row (the token, when scattering) before the
+            // wait; -1 for rows past the tile.  dx_dst[k4]: the row this lane
+            // stores in step k4 of the row-piece path (rows 4 k4 + lane / 8)
+            long long dx_row = -1;
             if (MODE == BW_DX && r_in < ti.rows) {
                 const int64_t r = (int64_t)ti.row0 + r_in;
-                dx_row = p.row_token ? (int64_t)p.row_token[r] : r;
+                dx_row = p.row_token ? (long long)p.row_token[r] : (long long)r;
             }
+            long long dx_dst[8];
+#pragma unroll
+            for (int k4 = 0; k4 < 8; ++k4)
+                dx_dst[k4] = MODE == BW_DX ? __shfl_sync(0xffffffffu, dx_row, 4 * k4 + (lane >> 3)) : -1;
             const bool got = wait_bar(smem_u32(&tfull_bar[acc]), acc_par, w);
             if (!__all_sync(0xffffffffu, got)) break;
             tc_fence_after();
@@ -413,17 +419,48 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     ++nchunk;
                     continue;
                 }
+                if constexpr (MODE == BW_DX) {
+                    // fp32 rows through the staging buffer: one TMA store when the
+                    // warp's 32 rows are compact rows of this tile, else 128-byte
+                    // row pieces (8 lanes per row) to their token rows
+                    const uint32_t ebuf = ebuf0 + (nchunk & 1u) * (32 * 128);
+                    const uint32_t row_sw = ebuf + lane * 128 + ((lane & 7) << 4);
+                    if (lane == 0) bulk_wait_read<1>();
+                    __syncwarp();
+#pragma unroll
+                    for (int g = 0; g < 8; ++g)
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_sw ^ (uint32_t)(g << 4)),
+                                     "r"(v[4 * g]), "r"(v[4 * g + 1]), "r"(v[4 * g + 2]), "r"(v[4 * g + 3])
+                                     : "memory");
+                    if (p.row_token == nullptr && q * 32 + 32 <= ti.rows) {
+                        fence_proxy_async_smem();
+                        __syncwarp();
+                        if (lane == 0) tma_store_2d(&tmOut, ebuf, col0, ti.row0 + q * 32);
+                    } else {
+                        __syncwarp();
+                        const int gi = lane & 7;
+                        const bool col_ok = col0 + 4 * gi < p.n_dim;
+#pragma unroll
+                        for (int k4 = 0; k4 < 8; ++k4) {
+                            const int r = 4 * k4 + (lane >> 3);
+                            uint4 val;
+                            const uint32_t srcp = ebuf + r * 128 + ((gi ^ (r & 7)) << 4);
+                            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                         : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                                         : "r"(srcp)
+                                         : "memory");
+                            if (dx_dst[k4] >= 0 && col_ok)
+                                *reinterpret_cast<uint4*>(p.out + (int64_t)dx_dst[k4] * p.n_dim + col0 + 4 * gi) = val;
+                        }
+                    }
+                    if (lane == 0) bulk_commit();
+                    __syncwarp();
+                    ++nchunk;
+                    continue;
+                }
                 if (r_in >= ti.rows) continue;
                 const int64_t r = (int64_t)ti.row0 + r_in;
-                if constexpr (MODE == BW_DX) {
-                    float* dst = p.out + dx_row * p.n_dim + col0;
-#pragma unroll
-                    for (int j = 0; j < 32; j += 4)
-                        if (col0 + j < p.n_dim)
-                            *reinterpret_cast<float4*>(dst + j) =
-                                make_float4(__uint_as_float(v[j]), __uint_as_float(v[j + 1]), __uint_as_float(v[j + 2]),
-                                            __uint_as_float(v[j + 3]));
-                } else {
+                {
                 // dU from dA = the accumulator
 #pragma unroll
                 for (int j0 = 0; j0 < 32; j0 += 8) {
@@ -467,7 +504,7 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             tc_fence_before();
             mbar_arrive_relaxed(smem_u32(&tempty_bar[acc]));
         }
-        if (MODE == BW_WGT && lane == 0) bulk_wait_all();   // this warp's TMA stores have landed
+        if ((MODE == BW_WGT || MODE == BW_DX) && lane == 0) bulk_wait_all();   // this warp's TMA stores have landed
     }
 
     tc_fence_before();
@@ -560,9 +597,10 @@ cudaError_t run_bwd(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMa
     return launch_k(bwd_gemm_kernel<MODE>, dim3((unsigned)sms), dim3(BW_THREADS), BW_SMEM, s, 1, a, b, b2, o, p);
 }
 
-// dW [groups * m, n] fp32 as the weight-gradient epilogue's TMA store target:
+// [rows, n] fp32 (dW as [groups * m, n], or compact dx rows) as an fp32
+// epilogue's TMA store target:
 // boxes of 32 rows x 32 columns (128 bytes), 128-byte swizzle
-bool wgt_out_map(CUtensorMap* m, const float* out, int64_t rows, int n) {
+bool f32_out_map(CUtensorMap* m, const float* out, int64_t rows, int n) {
     using EncodeFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -615,7 +653,9 @@ cudaError_t launch_tc_rows_f32(const void* A, int64_t rows, int K, const void* B
     p.out = out;
     p.status = status;
     p.limit_ns = kWaitLimitNs;
-    return run_bwd<BW_DX>(ma, mb, mb, ma, p, s);
+    CUtensorMap mo;
+    if (!f32_out_map(&mo, out, rows, n)) return cudaErrorInvalidValue;
+    return run_bwd<BW_DX>(ma, mb, mb, mo, p, s);
 }
 
 cudaError_t launch_tc_weights_f32(const void* A, int64_t rows, int m, const void* B, int n, const int32_t* offsets,
@@ -633,7 +673,7 @@ cudaError_t launch_tc_weights_f32(const void* A, int64_t rows, int m, const void
     p.status = status;
     p.limit_ns = kWaitLimitNs;
     CUtensorMap mo;
-    if (!wgt_out_map(&mo, out, (int64_t)groups * m, n)) return cudaErrorInvalidValue;
+    if (!f32_out_map(&mo, out, (int64_t)groups * m, n)) return cudaErrorInvalidValue;
     return run_bwd<BW_WGT>(ma, mb, mb, mo, p, s);
 }
 
@@ -704,7 +744,9 @@ cudaError_t launch_expert_backward_tc(const BwdArgs& a, cudaStream_t s) {
     px.k_split = sw ? dff : 0;
     px.out = a.top1_scatter ? a.dx : a.dxe;
     px.row_token = a.top1_scatter ? a.row_token : nullptr;
-    if ((err = run_bwd<BW_DX>(m_du, m_w1, sw ? m_w3 : m_w1, m_du, px, s)) != cudaSuccess) return err;
+    CUtensorMap m_dxo = m_du;   // compact dx rows (top-2): the TMA store target
+    if (!a.top1_scatter && !f32_out_map(&m_dxo, a.dxe, R, d)) return cudaErrorInvalidValue;
+    if ((err = run_bwd<BW_DX>(m_du, m_w1, sw ? m_w3 : m_w1, m_dxo, px, s)) != cudaSuccess) return err;
     if (a.top1_scatter) {
         if (a.T > 0 && (err = launch_k(dx_zero_dropped_kernel, dim3((unsigned)((a.T + 7) / 8)), dim3(256), 0, s, 1,
                                        a.drop, a.T, d, a.dx)) != cudaSuccess)
@@ -728,7 +770,7 @@ cudaError_t launch_expert_backward_tc(const BwdArgs& a, cudaStream_t s) {
     pw.mn3 = (ba2 ? 1 : 0) | (bxe ? 2 : 0);
     CUtensorMap m_o;
     if (a.dw1) {
-        if (!wgt_out_map(&m_o, a.dw1, (int64_t)N * dff, d)) return cudaErrorInvalidValue;
+        if (!f32_out_map(&m_o, a.dw1, (int64_t)N * dff, d)) return cudaErrorInvalidValue;
         if ((err = run_bwd<BW_WGT>(m_a2, m_xe, m_xe, m_o, pw, s)) != cudaSuccess) return err;
     }
     if (sw && a.dw3) {   // dUp: columns [d_ff, 2 d_ff)
@@ -737,7 +779,7 @@ cudaError_t launch_expert_backward_tc(const BwdArgs& a, cudaStream_t s) {
             return cudaErrorInvalidValue;
         pw.out = a.dw3;
         pw.mn3 = (bb2 ? 1 : 0) | (bxe ? 2 : 0);
-        if (!wgt_out_map(&m_o, a.dw3, (int64_t)N * dff, d)) return cudaErrorInvalidValue;
+        if (!f32_out_map(&m_o, a.dw3, (int64_t)N * dff, d)) return cudaErrorInvalidValue;
         if ((err = run_bwd<BW_WGT>(m_b2, m_xe, m_xe, m_o, pw, s)) != cudaSuccess) return err;
     }
     if (a.dw2) {
@@ -749,7 +791,7 @@ cudaError_t launch_expert_backward_tc(const BwdArgs& a, cudaStream_t s) {
         p2.n_dim = dff;
         p2.out = a.dw2;
         p2.mn3 = (bdy ? 1 : 0) | (bh ? 2 : 0);
-        if (!wgt_out_map(&m_o, a.dw2, (int64_t)N * d, dff)) return cudaErrorInvalidValue;
+        if (!f32_out_map(&m_o, a.dw2, (int64_t)N * d, dff)) return cudaErrorInvalidValue;
         if ((err = run_bwd<BW_WGT>(m_dy_mn, m_h, m_h, m_o, p2, s)) != cudaSuccess) return err;
     }
     // 6. bias gradients
