@@ -458,6 +458,61 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                     ++nchunk;
                     continue;
                 }
+                if constexpr (MODE == BW_DU_RELU) {
+                    // dU = dA where H > 0: bf16, two 32-column chunks per 128-byte
+                    // staging row, then one TMA store per 64 columns (row pieces
+                    // when some of the warp's rows are past the tile)
+                    const uint32_t half = (uint32_t)(c & 1);
+                    const uint32_t ebuf = ebuf0 + (nchunk & 1u) * (32 * 128);
+                    const uint32_t row_sw = ebuf + lane * 128 + ((lane & 7) << 4);
+                    if (half == 0) {
+                        if (lane == 0) bulk_wait_read<1>();
+                        __syncwarp();
+                    }
+#pragma unroll
+                    for (int h = 0; h < 4; ++h) {
+                        const uint32_t* hw = reinterpret_cast<const uint32_t*>(&fv[h % NPF]);
+                        uint32_t pk[4];
+#pragma unroll
+                        for (int h2 = 0; h2 < 4; ++h2) {
+                            const float a0 = bf16lo(hw[h2]) > 0.f ? __uint_as_float(v[8 * h + 2 * h2]) : 0.f;
+                            const float a1 = bf16hi(hw[h2]) > 0.f ? __uint_as_float(v[8 * h + 2 * h2 + 1]) : 0.f;
+                            pk[h2] = pack_bf16x2(a0, a1);
+                        }
+                        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(row_sw ^ ((half * 4 + h) << 4)),
+                                     "r"(pk[0]), "r"(pk[1]), "r"(pk[2]), "r"(pk[3])
+                                     : "memory");
+                    }
+                    if (half == 1) {
+                        const int pcol0 = col0 - 32;   // first column of the 64-column pair
+                        if (q * 32 + 32 <= ti.rows) {
+                            fence_proxy_async_smem();
+                            __syncwarp();
+                            if (lane == 0) tma_store_2d(&tmOut, ebuf, pcol0, ti.row0 + q * 32);
+                        } else {
+                            __syncwarp();
+                            const int gi = lane & 7;
+                            const bool col_ok = pcol0 + 8 * gi < p.n_dim;
+#pragma unroll
+                            for (int k4 = 0; k4 < 8; ++k4) {
+                                const int rr = 4 * k4 + (lane >> 3);
+                                uint4 val;
+                                const uint32_t srcp = ebuf + rr * 128 + ((gi ^ (rr & 7)) << 4);
+                                asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                                             : "=r"(val.x), "=r"(val.y), "=r"(val.z), "=r"(val.w)
+                                             : "r"(srcp)
+                                             : "memory");
+                                if (q * 32 + rr < ti.rows && col_ok)
+                                    *reinterpret_cast<uint4*>(p.du + ((int64_t)ti.row0 + q * 32 + rr) * p.n_dim + pcol0 +
+                                                              8 * gi) = val;
+                            }
+                        }
+                        if (lane == 0) bulk_commit();
+                        __syncwarp();
+                        ++nchunk;
+                    }
+                    continue;
+                }
                 if (r_in >= ti.rows) continue;
                 const int64_t r = (int64_t)ti.row0 + r_in;
                 {
@@ -504,7 +559,7 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
             tc_fence_before();
             mbar_arrive_relaxed(smem_u32(&tempty_bar[acc]));
         }
-        if ((MODE == BW_WGT || MODE == BW_DX) && lane == 0) bulk_wait_all();   // this warp's TMA stores have landed
+        if ((MODE == BW_WGT || MODE == BW_DX || MODE == BW_DU_RELU) && lane == 0) bulk_wait_all();   // TMA stores landed
     }
 
     tc_fence_before();
@@ -723,7 +778,10 @@ cudaError_t launch_expert_backward_tc(const BwdArgs& a, cudaStream_t s) {
     p.h = reinterpret_cast<const __nv_bfloat16*>(a.h);
     p.pre = reinterpret_cast<const __nv_bfloat16*>(a.pre);
     p.du = reinterpret_cast<__nv_bfloat16*>(a.du);
-    err = sw ? run_bwd<BW_DU_SWIGLU>(m_dy, m_w2, m_w2, m_dy, p, s) : run_bwd<BW_DU_RELU>(m_dy, m_w2, m_w2, m_dy, p, s);
+    CUtensorMap m_duo;   // ReLU dU [R, d_ff]: the TMA store target, 64 columns x 32 rows
+    if (!sw && !make_map_bf16(&m_duo, a.du, R, dff, 32)) return cudaErrorInvalidValue;
+    err = sw ? run_bwd<BW_DU_SWIGLU>(m_dy, m_w2, m_w2, m_dy, p, s)
+             : run_bwd<BW_DU_RELU>(m_dy, m_w2, m_w2, m_duo, p, s);
     if (err != cudaSuccess) return err;
     // 4. dx rows = dU W1 (+ dUp W3): K = d_ff (2 d_ff for SwiGLU, W3 for the second half)
     const int kdu = sw ? 2 * dff : dff;
