@@ -282,10 +282,14 @@ bwd_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__
                 }
                 if (lane == 0) {
                     issued = true;
+                    // the next 16-deep K slice: +32 bytes in a K-major tile, +16 rows of
+                    // 128 bytes in an MN-major one (the address field counts 16 bytes)
+                    const uint64_t ad0 = A_MN ? umma_desc_mn(a_addr, MN_BOX) : umma_desc(a_addr);
+                    const uint64_t bd0 = umma_desc_mn(b_addr, MN_BOX);
 #pragma unroll
                     for (int kk = 0; kk < BW_BK / 16; ++kk) {
-                        const uint64_t ad = A_MN ? umma_desc_mn(a_addr + kk * 2048, MN_BOX) : umma_desc(a_addr + kk * 32);
-                        const uint64_t bd = umma_desc_mn(b_addr + kk * 2048, MN_BOX);
+                        const uint64_t ad = ad0 + (uint64_t)(kk * (A_MN ? 2048 / 16 : 32 / 16));
+                        const uint64_t bd = bd0 + (uint64_t)(kk * (2048 / 16));
                         umma_f16(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
                     }
                     umma_commit(smem_u32(&empty_bar[stage]));
