@@ -13,21 +13,21 @@
 // and the gate-scaled top-1 combine y = p_{i*} E_{i*}(x) of the GLaM page.
 //
 // Kernel design (persistent, one CTA per SM, 192 threads, warp-specialised):
-//   warp 0   TMA producer: per stage a 128x64 A tile and a 64-wide B tile
-//            (128-byte swizzle) into an mbarrier ring.
+//   warp 0   TMA producer: per stage two 64-deep K boxes (128-byte swizzle) of
+//            A (128 rows) and of B into an mbarrier ring.
 //   warp 1   TMEM allocator + MMA issuer: tcgen05.mma kind::f16, bf16 x bf16 ->
 //            fp32 in TMEM, N = 256; two 256-column accumulators (all 512
 //            columns) so the epilogue of tile i overlaps the main loop of i+1.
 //   warps 2-5 epilogue: tcgen05.ld 32x32b (thread = row), bias, activation,
 //            gate, bf16 pack, 16-byte stores (optionally scattered to token rows).
 // Two variants share this code:
-//   single   one CTA owns a 128 x 256 tile (M=128 MMA); a stage is 16 KB of A
-//            plus 32 KB of B, 4 stages.
+//   single   one CTA owns a 128 x 256 tile (M=128 MMA); a stage is 32 KB of A
+//            plus 64 KB of B (128 deep in K), 2 stages.
 //   pair     a cluster of two CTAs owns a 256 x 256 tile with cta_group::2
 //            MMAs (M=256) issued by the pair's leader: each CTA loads its own
-//            128 rows of A and its own 128 rows of B, so a stage is 32 KB per CTA
-//            and 6 stages fit -- half the shared-memory traffic per MMA and more
-//            loads in flight.  Both CTAs' loads complete on the leader's full
+//            128 rows of A and its own 128 rows of B, so a stage is 64 KB per CTA
+//            (128 deep in K) and 3 stages fit -- half the shared-memory traffic
+//            per MMA.  Both CTAs' loads complete on the leader's full
 //            barrier (only the leader expects the bytes), the leader's MMA
 //            commits release both CTAs' stages and accumulators, and both CTAs'
 //            epilogues release the leader's accumulator.
@@ -55,8 +55,11 @@ namespace {
 
 constexpr int BM = 128;          // rows per CTA
 constexpr int BN = 256;          // MMA N (and TMEM columns per accumulator)
-constexpr int BK = 64;           // 64 bf16 = one 128-byte swizzle row
-constexpr int A_BYTES = BM * BK * 2;
+constexpr int BK = 64;           // 64 bf16 = one 128-byte swizzle row (one TMA box wide)
+constexpr int KSUB = 2;          // K boxes per pipeline stage: 128-deep stages, 8 MMAs per barrier round trip
+constexpr int BKS = BK * KSUB;   // K per stage
+constexpr int A_SUB = BM * BK * 2;   // one A box (16 KB)
+constexpr int A_BYTES = A_SUB * KSUB;
 constexpr int TMEM_COLS = 512;
 constexpr int GEMM_THREADS = 192;
 constexpr int GROUP_M = 8;
@@ -65,9 +68,12 @@ template <bool PAIR>
 struct GemmShape {
     static constexpr int TILE_M = PAIR ? 2 * BM : BM;             // rows per tile
     static constexpr int B_ROWS = PAIR ? BN / 2 : BN;             // B rows loaded per CTA
-    static constexpr int B_BYTES = B_ROWS * BK * 2;
+    static constexpr int B_SUB = B_ROWS * BK * 2;                 // one K box of B rows
+    static constexpr int B_BYTES = B_SUB * KSUB;
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-    static constexpr int STAGES = PAIR ? 6 : 4;
+    // 128-deep stages measured faster than 64-deep ones at the same bytes in
+    // flight (Switch-Base 599 -> 586 us, top-2 940 -> 900 us, Mixtral 9.8 -> 9.0 ms)
+    static constexpr int STAGES = PAIR ? 3 : 2;
     static constexpr int EPI_BYTES = 2 * 4 * 32 * 128;            // per epilogue warp: 2 x (32 rows x 128 B)
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + EPI_BYTES + 1024;
     static_assert((STAGES * STAGE_BYTES) % 1024 == 0, "epilogue staging buffers start 1024-byte aligned");
@@ -218,7 +224,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
     const uint32_t tmem_base = s_tmem;
     const int total = s_prefix[N];
-    const int nkb = (p.k_dim + BK - 1) / BK;
+    const int nkb = (p.k_dim + BKS - 1) / BKS;   // stages per tile (the last box of the last one may be K padding)
     const Waiter w{&s_abort, p.status, p.limit_ns};
 
     if (warp == 0) {
@@ -246,16 +252,23 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     if (PAIR) {
                         const uint32_t fb_leader = map_to_rank(fb, 0);
                         if (leader) mbar_expect_tx(fb, 2 * S::STAGE_BYTES);   // both CTAs' bytes
-                        tma_load_2d_pair(a_dst, &tmA, fb_leader, kb * BK, arow);
-                        tma_load_2d_pair(b_dst, bmap, fb_leader, kb * BK, brow);
+#pragma unroll
+                        for (int j = 0; j < KSUB; ++j) {
+                            tma_load_2d_pair(a_dst + j * A_SUB, &tmA, fb_leader, kb * BKS + j * BK, arow);
+                            tma_load_2d_pair(b_dst + j * S::B_SUB, bmap, fb_leader, kb * BKS + j * BK, brow);
+                        }
                     } else {
                         mbar_expect_tx(fb, S::STAGE_BYTES);
-                        tma_load_2d(a_dst, &tmA, fb, kb * BK, arow);
-                        if (EPI == EPI_SWIGLU) {
-                            tma_load_2d(b_dst, &tmB, fb, kb * BK, brow);
-                            tma_load_2d(b_dst + S::B_BYTES / 2, &tmB3, fb, kb * BK, brow);
-                        } else {
-                            tma_load_2d(b_dst, &tmB, fb, kb * BK, brow);
+#pragma unroll
+                        for (int j = 0; j < KSUB; ++j) {
+                            const int k0 = kb * BKS + j * BK;
+                            tma_load_2d(a_dst + j * A_SUB, &tmA, fb, k0, arow);
+                            if (EPI == EPI_SWIGLU) {   // W1 rows, then the same W3 rows
+                                tma_load_2d(b_dst + j * S::B_SUB, &tmB, fb, k0, brow);
+                                tma_load_2d(b_dst + j * S::B_SUB + S::B_SUB / 2, &tmB3, fb, k0, brow);
+                            } else {
+                                tma_load_2d(b_dst + j * S::B_SUB, &tmB, fb, k0, brow);
+                            }
                         }
                     }
                     last_par[stage] = (int)phase;
@@ -296,14 +309,19 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     issued = true;
                     const uint32_t a_addr = smem_u32(smem + stage * S::STAGE_BYTES);
                     // the descriptors' address field counts 16-byte units: the next
-                    // 16-wide K slice (32 bytes) of the swizzled rows is +2
+                    // 16-wide K slice (32 bytes) of the swizzled rows is +2, the
+                    // stage's second K box A_SUB (B_SUB) bytes on
                     const uint64_t a_desc = umma_desc(a_addr), b_desc = umma_desc(a_addr + A_BYTES);
 #pragma unroll
-                    for (int kk = 0; kk < BK / 16; ++kk) {
-                        const uint64_t ad = a_desc + 2 * kk, bd = b_desc + 2 * kk;
-                        const uint32_t accf = (kb | kk) != 0 ? 1u : 0u;
-                        if (PAIR) umma_f16_pair(d_tmem, ad, bd, S::IDESC, accf);
-                        else umma_f16(d_tmem, ad, bd, S::IDESC, accf);
+                    for (int j = 0; j < KSUB; ++j) {
+#pragma unroll
+                        for (int kk = 0; kk < BK / 16; ++kk) {
+                            const uint64_t ad = a_desc + (uint64_t)((j * A_SUB) >> 4) + 2 * kk;
+                            const uint64_t bd = b_desc + (uint64_t)((j * S::B_SUB) >> 4) + 2 * kk;
+                            const uint32_t accf = (kb | j | kk) != 0 ? 1u : 0u;
+                            if (PAIR) umma_f16_pair(d_tmem, ad, bd, S::IDESC, accf);
+                            else umma_f16(d_tmem, ad, bd, S::IDESC, accf);
+                        }
                     }
                     // frees the stage (in both CTAs of a pair) when these MMAs finish
                     if (PAIR) umma_commit_pair(smem_u32(&empty_bar[stage]), 0x3);
