@@ -48,23 +48,29 @@ constexpr int RT_BK = 64;
 
 template <int NP>
 struct RtShape {
-    static constexpr int A_BYTES = RT_BM * RT_BK * 2;
-    static constexpr int P_BYTES = (NP / 2) * RT_BK * 2;       // this CTA's half of one W part
-    static constexpr int STAGE_BYTES = A_BYTES + 3 * P_BYTES;
-    // as many stages as fit (the router is bound by the x bytes in flight)
-    static constexpr int STAGES = (200 * 1024) / STAGE_BYTES < 12 ? (200 * 1024) / STAGE_BYTES : 12;
-    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
     // merged: one MMA of N = 3 NP covers the three W parts and leaves three
     // partial-logit blocks side by side in TMEM; the pair's leader holds W rows
     // [0, 3 NP / 2) of the stacked parts, the peer rows [3 NP / 2, 3 NP).
     // Otherwise each part is its own MMA of N = NP, NP / 2 rows per CTA.
     static constexpr bool MERGED = 3 * NP <= 256;
+    // K boxes (64 deep) per pipeline stage: two when merged (8 MMAs per
+    // barrier round trip), one otherwise (three MMAs per K slice already)
+    static constexpr int KSUB = MERGED ? 2 : 1;
+    static constexpr int A_SUB = RT_BM * RT_BK * 2;             // one x box
+    static constexpr int A_BYTES = A_SUB * KSUB;
+    static constexpr int P_BYTES = (NP / 2) * RT_BK * 2;       // this CTA's half of one W part, one box
     static constexpr int W_BOX = MERGED ? 3 * NP / 2 : NP / 2;   // rows per W load
+    static constexpr int W_SUB = MERGED ? W_BOX * RT_BK * 2 : 3 * P_BYTES;   // W bytes per K box
+    static constexpr int STAGE_BYTES = A_BYTES + KSUB * W_SUB;
+    // as many stages as fit (the router is bound by the x bytes in flight)
+    static constexpr int STAGES = (200 * 1024) / STAGE_BYTES < 12 ? (200 * 1024) / STAGE_BYTES : 12;
+    static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
     static constexpr int ACC_COLS = MERGED ? 3 * NP : NP;      // TMEM columns per K-group accumulator
     static constexpr int TMEM_COLS = 512;                      // buffers x G groups x ACC_COLS
-    static constexpr int MMA_PER_KB = MERGED ? RT_BK / 16 : 3 * (RT_BK / 16);
+    static constexpr int MMA_PER_KB = KSUB * (MERGED ? RT_BK / 16 : 3 * (RT_BK / 16));   // per stage
     static constexpr int KB_PER_GROUP = 64 / MMA_PER_KB;       // <= 64 MMAs per accumulator
     static_assert(STAGE_BYTES % 1024 == 0, "1024-byte aligned stages");
+    static_assert(STAGES >= 2, "double-buffered stages");
     static constexpr int PER_LANE = NP / 32;   // experts whose warp sums of p a lane keeps
 };
 
@@ -217,7 +223,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 
     const uint32_t tmem_base = s_tmem;
     const int ntiles = (int)((p.T + 2 * RT_BM - 1) / (2 * RT_BM));
-    const int nkb = (p.d + RT_BK - 1) / RT_BK;
+    const int nkb = (p.d + S::KSUB * RT_BK - 1) / (S::KSUB * RT_BK);   // stages per tile
     const Waiter w{&s_abort, p.status, p.limit_ns};
 
     if (warp == 0) {
@@ -239,14 +245,19 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     const uint32_t fb_leader = map_to_rank(fb, 0);
                     const uint32_t a_dst = smem_u32(smem + stage * S::STAGE_BYTES);
                     if (leader) mbar_expect_tx(fb, 2 * S::STAGE_BYTES);   // both CTAs' bytes
-                    tma_load_2d_pair(a_dst, &tmX, fb_leader, kb * RT_BK, xrow);
-                    if constexpr (S::MERGED) {
-                        tma_load_2d_pair(a_dst + S::A_BYTES, &tmW, fb_leader, kb * RT_BK, (int)rank * S::W_BOX);
-                    } else {
 #pragma unroll
-                        for (int part = 0; part < 3; ++part)
-                            tma_load_2d_pair(a_dst + S::A_BYTES + part * S::P_BYTES, &tmW, fb_leader, kb * RT_BK,
-                                             part * NP + (int)rank * S::W_BOX);
+                    for (int j = 0; j < S::KSUB; ++j) {
+                        const int k0 = (kb * S::KSUB + j) * RT_BK;
+                        const uint32_t w_dst = a_dst + S::A_BYTES + j * S::W_SUB;
+                        tma_load_2d_pair(a_dst + j * S::A_SUB, &tmX, fb_leader, k0, xrow);
+                        if constexpr (S::MERGED) {
+                            tma_load_2d_pair(w_dst, &tmW, fb_leader, k0, (int)rank * S::W_BOX);
+                        } else {
+#pragma unroll
+                            for (int part = 0; part < 3; ++part)
+                                tma_load_2d_pair(w_dst + part * S::P_BYTES, &tmW, fb_leader, k0,
+                                                 part * NP + (int)rank * S::W_BOX);
+                        }
                     }
                     last_par[stage] = (int)phase;
                     if (++stage == S::STAGES) {
@@ -286,16 +297,20 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                     const uint64_t a_desc = desc0 + (uint64_t)((stage * S::STAGE_BYTES) >> 4);
                     const uint64_t b_desc = a_desc + (uint64_t)(S::A_BYTES >> 4);
 #pragma unroll
-                    for (int kk = 0; kk < RT_BK / 16; ++kk) {
-                        if constexpr (S::MERGED) {
-                            umma_f16_pair(d_tmem, a_desc + 2 * kk, b_desc + 2 * kk, IDESC,
-                                          (!first || kk != 0) ? 1u : 0u);
-                        } else {
+                    for (int j = 0; j < S::KSUB; ++j) {
+                        const uint64_t aj = a_desc + (uint64_t)((j * S::A_SUB) >> 4);
+                        const uint64_t bj = b_desc + (uint64_t)((j * S::W_SUB) >> 4);
 #pragma unroll
-                            for (int part = 0; part < 3; ++part)
-                                umma_f16_pair(d_tmem, a_desc + 2 * kk,
-                                              b_desc + (uint64_t)((part * S::P_BYTES) >> 4) + 2 * kk, IDESC,
-                                              (!first || (kk | part) != 0) ? 1u : 0u);
+                        for (int kk = 0; kk < RT_BK / 16; ++kk) {
+                            if constexpr (S::MERGED) {
+                                umma_f16_pair(d_tmem, aj + 2 * kk, bj + 2 * kk, IDESC,
+                                              (!first || (j | kk) != 0) ? 1u : 0u);
+                            } else {
+#pragma unroll
+                                for (int part = 0; part < 3; ++part)
+                                    umma_f16_pair(d_tmem, aj + 2 * kk, bj + (uint64_t)((part * S::P_BYTES) >> 4) + 2 * kk,
+                                                  IDESC, (!first || (j | kk | part) != 0) ? 1u : 0u);
+                            }
                         }
                     }
                     umma_commit_pair(smem_u32(&empty_bar[stage]), 0x3);   // frees the stage in both CTAs
@@ -484,7 +499,7 @@ cudaError_t run_router_tc(const RouterArgs& a, cudaStream_t s, int sms) {
     if (!make_map_bf16(&mx, a.x, a.T, a.d, RT_BM) || !make_map_bf16(&mw, a.w_split, 3 * NP, a.d, S::W_BOX))
         return cudaErrorInvalidValue;
     RtParams p{};
-    const int nkb = (a.d + RT_BK - 1) / RT_BK;
+    const int nkb = (a.d + S::KSUB * RT_BK - 1) / (S::KSUB * RT_BK);   // stages per tile
     // K groups of at most KB_PER_GROUP k-blocks (<= 64 MMAs per accumulator).
     // Two accumulator buffers (the epilogue overlaps the next tile) when the
     // groups fit in TMEM twice, or when fewer, larger groups of at most 72 MMAs
