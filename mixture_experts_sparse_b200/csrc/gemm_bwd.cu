@@ -22,7 +22,12 @@
 // warps 2-5 epilogue.  Operands:
 //   K-major A (row GEMMs): box 64 K x 128 rows, as in the forward;
 //   MN-major A / B: boxes of 64 MN elements x 64 K rows (128-byte swizzle), two
-//   for A (M = 128), four for B (N = 256), 8 KB apart.
+//   for A (M = 128), four for B (N = 256), 8 KB apart -- one blocked 3-D TMA
+//   load each when the matrix's columns are a multiple of 64.
+// Epilogues: fp32 outputs (dW, compact dx) and the ReLU dU leave through
+// swizzled shared-memory staging rows and TMA tensor stores; scattered dx rows
+// as 128-byte row pieces; the dU epilogue loads its forward values (H or the
+// SwiGLU pre-activations) one 32-column chunk ahead.
 // Every mbarrier wait is bounded (MOE_ERR_TIMEOUT on expiry, then a bounded
 // drain of the copies and MMAs in flight before TMEM is freed).
 #include "tc_common.cuh"
