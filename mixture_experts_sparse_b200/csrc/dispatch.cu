@@ -17,9 +17,9 @@
 //      a decoupled look-back across blocks (dynamic block tickets, bounded
 //      spin) turns the aggregates into exclusive block prefixes.  The last block
 //      to finish derives counts, kept = min(count, C) and the offsets.
-//   2. scatter_kernel: one warp per assignment adds the rank-0 total to rank-1
+//   2. scatter_kernel: per assignment, adds the rank-0 total to rank-1
 //      positions, writes pos/drop and the row map, and copies x[t] into its
-//      compact row with 16-byte vector accesses.
+//      compact row with 16-byte vector accesses (a warp per eight assignments).
 #include "common.cuh"
 
 namespace moe {
@@ -41,10 +41,15 @@ __device__ __forceinline__ void st_relaxed(uint32_t* p, uint32_t v) {
 }
 
 // Decoupled look-back for one counter: publish this block's aggregate, then walk
-// back over predecessors until one with an inclusive prefix is found.  Waiting
-// on a predecessor that has not published is bounded by limit_ns; on expiry the
-// wait latches MOE_ERR_TIMEOUT and this block publishes anyway, so successors
-// never wait on it.
+// back over predecessors until one with an inclusive prefix is found.  The
+// predecessors' states are read kLookWindow at a time (independent loads, one
+// memory round trip per window instead of one per predecessor: all blocks
+// publish their aggregates at about the same time, so a late block would
+// otherwise walk half its predecessors one load after another) and consumed in
+// order.  Waiting on a predecessor that has not published is bounded by
+// limit_ns; on expiry the wait latches MOE_ERR_TIMEOUT and this block publishes
+// anyway, so successors never wait on it.
+constexpr int kLookWindow = 8;
 __device__ uint32_t lookback(uint32_t* state, int bid, int c, int kN, uint32_t agg,
                              long long limit_ns, int32_t* status) {
     if (bid == 0) {
@@ -53,24 +58,37 @@ __device__ uint32_t lookback(uint32_t* state, int bid, int c, int kN, uint32_t a
     }
     st_relaxed(state + (int64_t)bid * kN + c, kFlagAgg | agg);
     uint32_t excl = 0;
-    int p = bid - 1;
+    int p = bid - 1;   // the next predecessor not yet added
     long long t_start = -1;
     unsigned spins = 0;
-    while (p >= 0) {
-        uint32_t v = ld_relaxed(state + (int64_t)p * kN + c);
-        uint32_t fl = v & ~kValMask;
-        if (fl == 0u) {
+    bool found = false;
+    while (!found) {
+        uint32_t v[kLookWindow];
+#pragma unroll
+        for (int j = 0; j < kLookWindow; ++j)   // block 0 always ends the walk, so p - j < 0 is never consumed
+            v[j] = p - j >= 0 ? ld_relaxed(state + (int64_t)(p - j) * kN + c) : kFlagPre;
+        int used = 0;
+#pragma unroll
+        for (int j = 0; j < kLookWindow; ++j) {
+            const uint32_t fl = v[j] & ~kValMask;
+            if (fl == 0u) break;   // not published yet: the next window starts here
+            excl += v[j] & kValMask;
+            ++used;
+            if (fl == kFlagPre) {
+                found = true;
+                break;
+            }
+        }
+        if (found) break;
+        p -= used;
+        if (used == 0) {   // the nearest unread predecessor has not published yet
             if (t_start < 0) t_start = global_ns();
             if ((++spins & 63u) == 0u && global_ns() - t_start > limit_ns) {
                 latch_status(status, MOE_ERR_TIMEOUT);
                 break;
             }
             __nanosleep(64);
-            continue;
         }
-        excl += v & kValMask;
-        if (fl == kFlagPre) break;
-        --p;
     }
     st_relaxed(state + (int64_t)bid * kN + c, kFlagPre | ((excl + agg) & kValMask));
     return excl;
@@ -174,6 +192,54 @@ scan_kernel(const int32_t* __restrict__ idx, int64_t T, int N, int k, int C, int
     }
 }
 
+// Slot bookkeeping of one assignment a (claim order: position q, rank r):
+// writes pos / drop and, when kept, the row map; returns the compact row, or -1
+// when the assignment is dropped.  t receives the token.
+__device__ __forceinline__ int claim_slot(int64_t a, const int32_t* __restrict__ idx, const float* __restrict__ gate,
+                                          int N, int k, int C, const int32_t* __restrict__ claim_base,
+                                          int32_t* __restrict__ pos, uint8_t* __restrict__ drop,
+                                          const int32_t* __restrict__ counts, const int32_t* __restrict__ offsets,
+                                          int32_t* __restrict__ row_token, float* __restrict__ row_gate,
+                                          const int32_t* __restrict__ perm, const int32_t* __restrict__ pos_in,
+                                          int64_t& t) {
+    // Batch priority: the token at position q is perm[q], and the scan's claim
+    // numbers are in pos_in (claim-order layout).
+    const int64_t q = a / k;
+    const int r = (int)(a - q * k);
+    t = perm ? (int64_t)perm[q] : q;
+    const int64_t ao = t * k + r;   // the assignment in token order
+    const int e = idx[ao];
+    const int lp = pos_in ? pos_in[a] : pos[a];   // claim number among this shard's rank-r claims on e
+    int p, row_off;
+    if (r == 0) {
+        p = (claim_base ? claim_base[e] : 0) + lp;
+        row_off = lp;
+    } else {   // every rank-0 claim precedes the rank-1 claims
+        const int base0 = claim_base ? claim_base[e] : 0;
+        p = (claim_base ? claim_base[N + e] : counts[e]) + lp;
+        row_off = kept_after(base0, counts[e], C) + lp;
+    }
+    const bool keep = p < C;
+    pos[ao] = p;
+    drop[ao] = keep ? 0 : 1;
+    if (!keep) return -1;
+    const int row = offsets[e] + row_off;
+    row_token[row] = (int32_t)t;
+    row_gate[row] = gate[ao];
+    return row;
+}
+
+// One warp per kScatterRows consecutive assignments: lanes 0 .. kScatterRows-1
+// do the slot bookkeeping of one assignment each (one dependent chain of loads
+// per warp instead of one per row), then the warp moves the rows two at a
+// time -- a kept row's x[t] into its compact row, a dropped token's output row
+// set to zero when zero_out is given -- with up to 2 x kCopyUnroll 16-byte
+// loads per lane in flight.  The grid is a single wave at Switch-Base sizes
+// (8192 blocks of one assignment per warp, each living about a microsecond,
+// were bound by block launches).
+constexpr int kScatterRows = 8;
+constexpr int kCopyUnroll = 4;
+
 template <typename XT>
 __global__ void __launch_bounds__(256)
 scatter_kernel(const XT* __restrict__ x, const int32_t* __restrict__ idx, const float* __restrict__ gate,
@@ -192,64 +258,63 @@ scatter_kernel(const XT* __restrict__ x, const int32_t* __restrict__ idx, const 
         return;
     }
     const int lane = threadIdx.x & 31;
-    const int64_t a = (int64_t)(blockIdx.x - (aux.G > 0 ? 1 : 0)) * 8 + (threadIdx.x >> 5);
-    if (a >= T * k) return;
-    // a enumerates the assignments in claim order: position q of the claim
-    // order, rank r.  Batch priority: the token at position q is perm[q], and
-    // the scan's claim numbers are in pos_in (claim-order layout).
-    const int64_t q = a / k;
-    const int r = (int)(a - q * k);
-    const int64_t t = perm ? (int64_t)perm[q] : q;
-    const int64_t ao = t * k + r;               // the assignment in token order
-    int row = -1;
-    if (lane == 0) {
-        const int e = idx[ao];
-        const int lp = pos_in ? pos_in[a] : pos[a];   // claim number among this shard's rank-r claims on e
-        int p, row_off;
-        if (r == 0) {
-            p = (claim_base ? claim_base[e] : 0) + lp;
-            row_off = lp;
-        } else {                                // every rank-0 claim precedes the rank-1 claims
-            const int base0 = claim_base ? claim_base[e] : 0;
-            p = (claim_base ? claim_base[N + e] : counts[e]) + lp;
-            row_off = kept_after(base0, counts[e], C) + lp;
-        }
-        const bool keep = p < C;
-        pos[ao] = p;
-        drop[ao] = keep ? 0 : 1;
-        if (keep) {
-            row = offsets[e] + row_off;
-            row_token[row] = (int32_t)t;
-            row_gate[row] = gate[ao];
-        }
+    const int64_t n_assign = T * k;
+    const int64_t a0 = ((int64_t)(blockIdx.x - (aux.G > 0 ? 1 : 0)) * 8 + (threadIdx.x >> 5)) * kScatterRows;
+    if (a0 >= n_assign) return;
+    // per lane i < kScatterRows: what happens to assignment a0 + i's row --
+    // >= 0 copy x[t] to that compact row, -1 zero out[t], -2 nothing
+    int act = -2;
+    int64_t t = 0;
+    if (lane < kScatterRows && a0 + lane < n_assign) {
+        const int row = claim_slot(a0 + lane, idx, gate, N, k, C, claim_base, pos, drop, counts, offsets, row_token,
+                                   row_gate, perm, pos_in, t);
+        act = row >= 0 ? (xe != nullptr ? row : -2) : (zero_out != nullptr ? -1 : -2);
     }
-    row = __shfl_sync(0xffffffffu, row, 0);
     const size_t bytes = (size_t)d * sizeof(XT);
-    if (row >= 0) {
-        if (xe == nullptr) return;
-        const char* src = reinterpret_cast<const char*>(x + t * (int64_t)d);
-        char* dst = reinterpret_cast<char*>(xe + (int64_t)row * d);
+    const uint4 z4 = make_uint4(0, 0, 0, 0);
+#pragma unroll 1
+    for (int i = 0; i < kScatterRows; i += 2) {
+        const int act0 = __shfl_sync(0xffffffffu, act, i), act1 = __shfl_sync(0xffffffffu, act, i + 1);
+        const int64_t t0 = __shfl_sync(0xffffffffu, t, i), t1 = __shfl_sync(0xffffffffu, t, i + 1);
+        if (act0 == -2 && act1 == -2) continue;
+        const XT* s0 = x + t0 * (int64_t)d;
+        const XT* s1 = x + t1 * (int64_t)d;
+        XT* d0 = act0 >= 0 ? xe + (int64_t)act0 * d : (act0 == -1 ? zero_out + t0 * (int64_t)d : nullptr);
+        XT* d1 = act1 >= 0 ? xe + (int64_t)act1 * d : (act1 == -1 ? zero_out + t1 * (int64_t)d : nullptr);
         if (bytes % 16 == 0) {
-            for (size_t o = (size_t)lane * 16; o < bytes; o += 32 * 16)
-                *reinterpret_cast<uint4*>(dst + o) = __ldg(reinterpret_cast<const uint4*>(src + o));
+            const char* c0 = reinterpret_cast<const char*>(s0);
+            const char* c1 = reinterpret_cast<const char*>(s1);
+            char* e0 = reinterpret_cast<char*>(d0);
+            char* e1 = reinterpret_cast<char*>(d1);
+            for (size_t o = (size_t)lane * 16; o < bytes; o += 32 * 16 * kCopyUnroll) {
+                uint4 v0[kCopyUnroll], v1[kCopyUnroll];
+#pragma unroll
+                for (int u = 0; u < kCopyUnroll; ++u) {
+                    const size_t oo = o + (size_t)u * 32 * 16;
+                    v0[u] = (act0 >= 0 && oo < bytes) ? __ldg(reinterpret_cast<const uint4*>(c0 + oo)) : z4;
+                    v1[u] = (act1 >= 0 && oo < bytes) ? __ldg(reinterpret_cast<const uint4*>(c1 + oo)) : z4;
+                }
+#pragma unroll
+                for (int u = 0; u < kCopyUnroll; ++u) {
+                    const size_t oo = o + (size_t)u * 32 * 16;
+                    if (oo < bytes) {
+                        if (e0) *reinterpret_cast<uint4*>(e0 + oo) = v0[u];
+                        if (e1) *reinterpret_cast<uint4*>(e1 + oo) = v1[u];
+                    }
+                }
+            }
         } else {
-            for (int j = lane; j < d; j += 32) xe[(int64_t)row * d + j] = x[t * (int64_t)d + j];
-        }
-    } else if (zero_out != nullptr) {
-        char* dst = reinterpret_cast<char*>(zero_out + t * (int64_t)d);
-        if (bytes % 16 == 0) {
-            for (size_t o = (size_t)lane * 16; o < bytes; o += 32 * 16)
-                *reinterpret_cast<uint4*>(dst + o) = make_uint4(0, 0, 0, 0);
-        } else {
-            for (int j = lane; j < d; j += 32) zero_out[t * (int64_t)d + j] = XT(0.f);
+            for (int j = lane; j < d; j += 32) {
+                if (d0) d0[j] = act0 >= 0 ? s0[j] : XT(0.f);
+                if (d1) d1[j] = act1 >= 0 ? s1[j] : XT(0.f);
+            }
         }
     }
 }
 
 // The same slot bookkeeping without the compact copy and without output rows
 // to zero (moe_dispatch called with no xe): one thread per assignment writes
-// pos, drop, row_token and row_gate -- 32x fewer warps than scatter_kernel,
-// whose warp per assignment exists for the row copy.
+// pos, drop, row_token and row_gate.
 __global__ void __launch_bounds__(256)
 rowmap_kernel(const int32_t* __restrict__ idx, const float* __restrict__ gate, int64_t T, int N, int k, int C,
               const int32_t* __restrict__ claim_base, int32_t* __restrict__ pos, uint8_t* __restrict__ drop,
@@ -265,29 +330,8 @@ rowmap_kernel(const int32_t* __restrict__ idx, const float* __restrict__ gate, i
     }
     const int64_t a = (int64_t)(blockIdx.x - (aux.G > 0 ? 1 : 0)) * 256 + threadIdx.x;
     if (a >= T * k) return;
-    const int64_t q = a / k;
-    const int r = (int)(a - q * k);
-    const int64_t t = perm ? (int64_t)perm[q] : q;
-    const int64_t ao = t * k + r;
-    const int e = idx[ao];
-    const int lp = pos_in ? pos_in[a] : pos[a];
-    int p, row_off;
-    if (r == 0) {
-        p = (claim_base ? claim_base[e] : 0) + lp;
-        row_off = lp;
-    } else {
-        const int base0 = claim_base ? claim_base[e] : 0;
-        p = (claim_base ? claim_base[N + e] : counts[e]) + lp;
-        row_off = kept_after(base0, counts[e], C) + lp;
-    }
-    const bool keep = p < C;
-    pos[ao] = p;
-    drop[ao] = keep ? 0 : 1;
-    if (keep) {
-        const int row = offsets[e] + row_off;
-        row_token[row] = (int32_t)t;
-        row_gate[row] = gate[ao];
-    }
+    int64_t t;
+    claim_slot(a, idx, gate, N, k, C, claim_base, pos, drop, counts, offsets, row_token, row_gate, perm, pos_in, t);
 }
 
 // ---- batch priority: the claim order --------------------------------------
@@ -709,6 +753,11 @@ __global__ void lookback_probe_kernel(uint32_t* state, WsHeader* hdr, long long 
 
 int scan_blocks(int64_t T) { return (int)((T + kScanTokens - 1) / kScanTokens); }
 
+// blocks of scatter_kernel: 8 warps of kScatterRows assignments, plus the aux block
+static unsigned scatter_grid(int64_t n_assign, bool aux_block) {
+    return (unsigned)((n_assign + 8 * kScatterRows - 1) / (8 * kScatterRows)) + (aux_block ? 1u : 0u);
+}
+
 cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
     const int nblk = scan_blocks(a.T);
     if (nblk == 0) return cudaSuccess;
@@ -759,8 +808,7 @@ cudaError_t launch_dispatch(const DispatchArgs& a, cudaStream_t s) {
                         a.claim_base, a.pos, a.drop, a.counts, a.offsets, a.row_token, a.row_gate, a.aux, perm,
                         pos_in);
     }
-    const int64_t warps = a.T * a.k;
-    const unsigned grid = (unsigned)((warps + 7) / 8) + (a.aux.G > 0 ? 1u : 0u);
+    const unsigned grid = scatter_grid(a.T * a.k, a.aux.G > 0);
     if (a.dtype == MOE_BF16)
         return launch_k(scatter_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, 1,
                         reinterpret_cast<const __nv_bfloat16*>(a.x), a.idx, a.gate, a.T, a.d, a.N, a.k, a.C,
@@ -831,7 +879,7 @@ cudaError_t launch_dispatch_ntlb(const NtlbArgs& a, cudaStream_t s) {
                         static_cast<const int32_t*>(a.counts), static_cast<const int32_t*>(a.offsets), a.row_token,
                         a.row_gate, a.aux, none, none);
     }
-    const unsigned grid = (unsigned)((a.T + 7) / 8) + (a.aux.G > 0 ? 1u : 0u);
+    const unsigned grid = scatter_grid(a.T, a.aux.G > 0);
     if (a.dtype == MOE_BF16)
         return launch_k(scatter_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, 1,
                         reinterpret_cast<const __nv_bfloat16*>(a.x), static_cast<const int32_t*>(a.expert),
