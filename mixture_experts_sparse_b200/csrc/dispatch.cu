@@ -49,7 +49,7 @@ __device__ __forceinline__ void st_relaxed(uint32_t* p, uint32_t v) {
 // order.  Waiting on a predecessor that has not published is bounded by
 // limit_ns; on expiry the wait latches MOE_ERR_TIMEOUT and this block publishes
 // anyway, so successors never wait on it.
-constexpr int kLookWindow = 8;
+constexpr int kLookWindow = 16;
 __device__ uint32_t lookback(uint32_t* state, int bid, int c, int kN, uint32_t agg,
                              long long limit_ns, int32_t* status) {
     if (bid == 0) {
@@ -115,7 +115,15 @@ scan_kernel(const int32_t* __restrict__ idx, int64_t T, int N, int k, int C, int
     const int bid = s_bid;
     const int64_t tw0 = (int64_t)bid * kScanTokens + warp * kWarpTokens;
 
-    // 1. in-warp ranks, in token order, per (rank, expert) counter
+    // 1. in-warp ranks, in token order, per (rank, expert) counter; the warp's
+    //    choices are loaded first, all at once (one memory round trip)
+    int keys[kWarpTokens / 32][2];
+#pragma unroll
+    for (int it = 0; it < kWarpTokens / 32; ++it) {
+        const int64_t t = tw0 + it * 32 + lane;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) keys[it][r] = (r < k && t < T) ? r * N + idx[t * k + r] : -1;
+    }
     int rank[kWarpTokens / 32][2];
     const unsigned lt_mask = (1u << lane) - 1u;
 #pragma unroll
@@ -125,7 +133,7 @@ scan_kernel(const int32_t* __restrict__ idx, int64_t T, int N, int k, int C, int
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
             if (r >= k) break;
-            const int key = valid ? r * N + idx[t * k + r] : -1;
+            const int key = keys[it][r];
             const unsigned peers = __match_any_sync(0xffffffffu, key);
             const int before = __popc(peers & lt_mask);
             if (valid) rank[it][r] = s_wcnt[warp][key] + before;
@@ -156,7 +164,7 @@ scan_kernel(const int32_t* __restrict__ idx, int64_t T, int N, int k, int C, int
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
             if (r >= k) break;
-            const int key = r * N + idx[t * k + r];
+            const int key = keys[it][r];
             pos[t * k + r] = (int)s_excl[key] + s_wcnt[warp][key] + rank[it][r];
         }
     }

@@ -13,15 +13,19 @@
 // w1 = bf16(w - w0), w2 = w - w0 - w1).  Every product x * w_p is exact in fp32,
 // and the tensor core accumulates them in fp32, so
 //   h = sum_j x_j w0_j + sum_j x_j w1_j + sum_j x_j w2_j
-// is the fp32 dot product up to accumulation rounding -- three bf16 MMAs per
-// K step.  With 3 NP <= 256 the three parts are adjacent rows of one B tile, so
-// a single MMA of N = 3 NP produces the three partial logits side by side in
-// TMEM (the epilogue adds them in fp32).  The tensor core's fp32 accumulation
-// truncates, so its error grows with the number of MMAs summed into one
-// accumulator; the K loop is therefore cut into G groups of at most 64 MMAs per
-// accumulator, each group in its own TMEM column block, and the epilogue adds
-// the partial logits in fp32 with round-to-nearest in a fixed order.  The router then costs about one read
-// of x from HBM instead of 2 d N FP32-pipe FLOPs per token.
+// is the fp32 dot product up to accumulation rounding -- 3 NP columns of bf16
+// MMA per K step.  With 3 NP <= 256 the three parts are adjacent rows of one B
+// tile, so a single MMA of N = 3 NP produces the three partial logits side by
+// side in TMEM (the epilogue adds them in fp32); with NP = 128, an MMA of
+// N = 256 (parts 0 and 1) and one of N = 128 (part 2, added to part 1's
+// block) -- an MMA costs about the same issue time at N = 128 as at N = 256,
+// so two instructions per K step instead of three.  The tensor core's fp32
+// accumulation truncates, so its error grows with the number of MMAs summed
+// into one accumulator at the logits' scale; the K loop is therefore cut into
+// G groups of at most 64 such MMAs, each group in its own TMEM column block,
+// and the epilogue adds the partial logits in fp32 with round-to-nearest in a
+// fixed order.  The router then costs about one read of x from HBM instead of
+// 2 d N FP32-pipe FLOPs per token.
 //
 // Kernel: persistent CTA pairs (clusters of two), 192 threads per CTA.  A
 // pair owns a 256-token tile and issues cta_group::2 MMAs (M = 256 tokens, 128
@@ -51,7 +55,11 @@ struct RtShape {
     // merged: one MMA of N = 3 NP covers the three W parts and leaves three
     // partial-logit blocks side by side in TMEM; the pair's leader holds W rows
     // [0, 3 NP / 2) of the stacked parts, the peer rows [3 NP / 2, 3 NP).
-    // Otherwise each part is its own MMA of N = NP, NP / 2 rows per CTA.
+    // Otherwise (NP = 128) two MMAs per K slice: one of N = 256 over parts 0
+    // and 1 (the leader holds part 0, the peer part 1) into column blocks 0 and
+    // 1, and one of N = 128 over part 2 (NP / 2 rows per CTA) that accumulates
+    // into block 1 -- parts 1 and 2 are 2^-8 and 2^-16 of w, so their shared
+    // accumulator stays 2^8 below the logits and its truncation error with it.
     static constexpr bool MERGED = 3 * NP <= 256;
     // K boxes (64 deep) per pipeline stage: two when merged (8 MMAs per
     // barrier round trip), one otherwise (three MMAs per K slice already)
@@ -65,10 +73,12 @@ struct RtShape {
     // as many stages as fit (the router is bound by the x bytes in flight)
     static constexpr int STAGES = (200 * 1024) / STAGE_BYTES < 12 ? (200 * 1024) / STAGE_BYTES : 12;
     static constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024;
-    static constexpr int ACC_COLS = MERGED ? 3 * NP : NP;      // TMEM columns per K-group accumulator
+    static constexpr int BLOCKS = MERGED ? 3 : 2;              // partial-logit column blocks per accumulator
+    static constexpr int ACC_COLS = BLOCKS * NP;               // TMEM columns per K-group accumulator
     static constexpr int TMEM_COLS = 512;                      // buffers x G groups x ACC_COLS
-    static constexpr int MMA_PER_KB = KSUB * (MERGED ? RT_BK / 16 : 3 * (RT_BK / 16));   // per stage
-    static constexpr int KB_PER_GROUP = 64 / MMA_PER_KB;       // <= 64 MMAs per accumulator
+    // per stage, MMAs into the full-scale block (part 0's sums)
+    static constexpr int MMA_PER_KB = KSUB * (RT_BK / 16);
+    static constexpr int KB_PER_GROUP = 64 / MMA_PER_KB;       // <= 64 MMAs per full-scale accumulator
     static_assert(STAGE_BYTES % 1024 == 0, "1024-byte aligned stages");
     static_assert(STAGES >= 2, "double-buffered stages");
     static constexpr int PER_LANE = NP / 32;   // experts whose warp sums of p a lane keeps
@@ -171,7 +181,9 @@ template <int NP>
 __global__ void __launch_bounds__(RT_THREADS, 1)
 router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, const RtParams p) {
     using S = RtShape<NP>;
-    constexpr uint32_t IDESC = idesc_bf16_f32(2 * RT_BM, S::ACC_COLS);
+    // merged: N = 3 NP; otherwise N = 256 (parts 0, 1) and N = 128 (part 2)
+    constexpr uint32_t IDESC = idesc_bf16_f32(2 * RT_BM, S::MERGED ? S::ACC_COLS : 2 * NP);
+    constexpr uint32_t IDESC2 = idesc_bf16_f32(2 * RT_BM, NP);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     __shared__ float s_wsum[4][NP];    // per epilogue warp: sums of p over its tokens
@@ -252,11 +264,10 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                         tma_load_2d_pair(a_dst + j * S::A_SUB, &tmX, fb_leader, k0, xrow);
                         if constexpr (S::MERGED) {
                             tma_load_2d_pair(w_dst, &tmW, fb_leader, k0, (int)rank * S::W_BOX);
-                        } else {
-#pragma unroll
-                            for (int part = 0; part < 3; ++part)
-                                tma_load_2d_pair(w_dst + part * S::P_BYTES, &tmW, fb_leader, k0,
-                                                 part * NP + (int)rank * S::W_BOX);
+                        } else {   // this CTA's part (leader 0, peer 1), all NP rows; then its half of part 2
+                            tma_load_2d_pair(w_dst, &tmW, fb_leader, k0, (int)rank * NP);
+                            tma_load_2d_pair(w_dst + S::P_BYTES, &tmW, fb_leader, k0, (int)rank * NP + S::W_BOX);
+                            tma_load_2d_pair(w_dst + 2 * S::P_BYTES, &tmW, fb_leader, k0, 2 * NP + (int)rank * S::W_BOX);
                         }
                     }
                     last_par[stage] = (int)phase;
@@ -305,11 +316,11 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
                             if constexpr (S::MERGED) {
                                 umma_f16_pair(d_tmem, aj + 2 * kk, bj + 2 * kk, IDESC,
                                               (!first || (j | kk) != 0) ? 1u : 0u);
-                            } else {
-#pragma unroll
-                                for (int part = 0; part < 3; ++part)
-                                    umma_f16_pair(d_tmem, aj + 2 * kk, bj + (uint64_t)((part * S::P_BYTES) >> 4) + 2 * kk,
-                                                  IDESC, (!first || (j | kk | part) != 0) ? 1u : 0u);
+                            } else {   // parts 0 | 1 into blocks 0 | 1, then part 2 added to block 1
+                                umma_f16_pair(d_tmem, aj + 2 * kk, bj + 2 * kk, IDESC,
+                                              (!first || (j | kk) != 0) ? 1u : 0u);
+                                umma_f16_pair(d_tmem + NP, aj + 2 * kk, bj + (uint64_t)((2 * S::P_BYTES) >> 4) + 2 * kk,
+                                              IDESC2, 1u);
                             }
                         }
                     }
@@ -367,7 +378,7 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
             for (int g = 0; g < p.groups; ++g) {   // partial logits of the K groups (and W parts), in order
                 constexpr int CH = NP < 64 ? NP : 64;   // columns per TMEM load
 #pragma unroll
-                for (int part = 0; part < (S::MERGED ? 3 : 1); ++part) {
+                for (int part = 0; part < S::BLOCKS; ++part) {
 #pragma unroll
                     for (int c = 0; c < NP / CH; ++c) {
                         const uint32_t col = tbase + g * S::ACC_COLS + part * NP + c * CH;
@@ -500,7 +511,7 @@ cudaError_t run_router_tc(const RouterArgs& a, cudaStream_t s, int sms) {
         return cudaErrorInvalidValue;
     RtParams p{};
     const int nkb = (a.d + S::KSUB * RT_BK - 1) / (S::KSUB * RT_BK);   // stages per tile
-    // K groups of at most KB_PER_GROUP k-blocks (<= 64 MMAs per accumulator).
+    // K groups of at most KB_PER_GROUP k-blocks (<= 64 MMAs per full-scale accumulator).
     // Two accumulator buffers (the epilogue overlaps the next tile) when the
     // groups fit in TMEM twice, or when fewer, larger groups of at most 72 MMAs
     // do; otherwise one buffer with groups of <= 64 MMAs.
