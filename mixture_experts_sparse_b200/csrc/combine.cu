@@ -5,7 +5,7 @@
 // layer, carries it).  "From Switch Transformer to GLaM": y = p_{i*} E_{i*}(x)
 // for top-1 and y = w1 E_{i1}(x) + w2 E_{i2}(x) for top-2, "Expert Capacity and
 // Token Dropping" (an overflowing token skips the expert FFN).
-// One warp per token, 16-byte vector loads/stores: an HBM-bound gather.
+// 16-byte vector loads/stores: an HBM-bound gather.
 //
 // For one shard of a routing group pos holds group-wide claim numbers; the
 // shard's rows of expert e hold its kept rank-0 claims (numbers base0[e] ...)
@@ -17,6 +17,16 @@
 namespace moe {
 namespace {
 
+// One warp per kCombineTokens consecutive tokens: lanes 0 .. kCombineTokens*k-1
+// each locate one assignment's row and gate (one dependent chain of loads per
+// warp instead of one per token), then the warp combines the tokens one after
+// another with all of a token's 16-byte row loads (up to kCombineUnroll
+// chunks per lane per row) in flight before its first store.  With a warp per
+// token, 4096 blocks of 256 threads each lived about a microsecond at top-2
+// sizes and block launches bounded the kernel.
+constexpr int kCombineTokens = 4;
+constexpr int kCombineUnroll = 4;
+
 template <typename XT>
 __global__ void __launch_bounds__(256)
 combine_kernel(const XT* __restrict__ ye, const int32_t* __restrict__ idx, const int32_t* __restrict__ pos,
@@ -27,46 +37,77 @@ combine_kernel(const XT* __restrict__ ye, const int32_t* __restrict__ idx, const
     pdl_wait();
     pdl_launch();
     const int lane = threadIdx.x & 31;
-    const int64_t t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (t >= T) return;
-    int64_t row[2] = {-1, -1};
-    float g[2] = {0.f, 0.f};
-    for (int r = 0; r < k; ++r) {
+    const int64_t t0 = ((int64_t)blockIdx.x * 8 + (threadIdx.x >> 5)) * kCombineTokens;
+    if (t0 >= T) return;
+    int64_t my_row = -1;   // lane i < kCombineTokens * k: token t0 + i / k, rank i % k (-1: dropped)
+    float my_g = 0.f;
+    if (lane < kCombineTokens * k) {
+        const int64_t t = t0 + lane / k;
+        const int r = lane - (lane / k) * k;
         const int64_t a = t * k + r;
-        if (!drop[a]) {
+        if (t < T && !drop[a]) {
             const int e = idx[a];
             int local = pos[a];
             if (claim_base)
                 local = r == 0 ? local - claim_base[e]
                                : kept_after(claim_base[e], counts[e], C) + local - claim_base[N + e];
-            row[r] = (int64_t)offsets[e] + local;
-            g[r] = gate[a];
+            my_row = (int64_t)offsets[e] + local;
+            my_g = gate[a];
         }
     }
-    XT* dst = out + t * (int64_t)d;
-    if (((size_t)d * sizeof(XT)) % 16 == 0) {
-        for (int c = lane * VEC; c < d; c += 32 * VEC) {
-            float acc[VEC];
+#pragma unroll 1
+    for (int i = 0; i < kCombineTokens; ++i) {
+        const int64_t t = t0 + i;
+        if (t >= T) break;   // warp-uniform
+        int64_t row[2];
+        float g[2];
 #pragma unroll
-            for (int j = 0; j < VEC; ++j) acc[j] = 0.f;
-            for (int r = 0; r < k; ++r) {
-                if (row[r] < 0) continue;
-                uint4 v = __ldg(reinterpret_cast<const uint4*>(ye + row[r] * d + c));
-                const XT* xv = reinterpret_cast<const XT*>(&v);
-#pragma unroll
-                for (int j = 0; j < VEC; ++j) acc[j] = fmaf(g[r], Elem<XT>::to_f(xv[j]), acc[j]);
-            }
-            XT o[VEC];
-#pragma unroll
-            for (int j = 0; j < VEC; ++j) o[j] = Elem<XT>::from_f(acc[j]);
-            *reinterpret_cast<uint4*>(dst + c) = *reinterpret_cast<uint4*>(o);
+        for (int r = 0; r < 2; ++r) {
+            const int src = i * k + (r < k ? r : 0);
+            row[r] = __shfl_sync(0xffffffffu, my_row, src);
+            g[r] = __shfl_sync(0xffffffffu, my_g, src);
+            if (r >= k) row[r] = -1;
         }
-    } else {
-        for (int c = lane; c < d; c += 32) {
-            float acc = 0.f;
-            for (int r = 0; r < k; ++r)
-                if (row[r] >= 0) acc = fmaf(g[r], Elem<XT>::to_f(ye[row[r] * d + c]), acc);
-            dst[c] = Elem<XT>::from_f(acc);
+        XT* dst = out + t * (int64_t)d;
+        if (((size_t)d * sizeof(XT)) % 16 == 0) {
+            for (int c0 = lane * VEC; c0 < d; c0 += 32 * VEC * kCombineUnroll) {
+                uint4 v[2][kCombineUnroll];
+#pragma unroll
+                for (int r = 0; r < 2; ++r)
+#pragma unroll
+                    for (int u = 0; u < kCombineUnroll; ++u) {
+                        const int c = c0 + u * 32 * VEC;
+                        v[r][u] = (row[r] >= 0 && c < d)
+                                      ? __ldg(reinterpret_cast<const uint4*>(ye + row[r] * d + c))
+                                      : make_uint4(0, 0, 0, 0);
+                    }
+#pragma unroll
+                for (int u = 0; u < kCombineUnroll; ++u) {
+                    const int c = c0 + u * 32 * VEC;
+                    if (c >= d) break;
+                    float acc[VEC];
+#pragma unroll
+                    for (int j = 0; j < VEC; ++j) acc[j] = 0.f;
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {   // rank order, one rounding at the end
+                        if (row[r] < 0) continue;
+                        const XT* xv = reinterpret_cast<const XT*>(&v[r][u]);
+#pragma unroll
+                        for (int j = 0; j < VEC; ++j) acc[j] = fmaf(g[r], Elem<XT>::to_f(xv[j]), acc[j]);
+                    }
+                    XT o[VEC];
+#pragma unroll
+                    for (int j = 0; j < VEC; ++j) o[j] = Elem<XT>::from_f(acc[j]);
+                    *reinterpret_cast<uint4*>(dst + c) = *reinterpret_cast<uint4*>(o);
+                }
+            }
+        } else {
+            for (int c = lane; c < d; c += 32) {
+                float acc = 0.f;
+                for (int r = 0; r < 2; ++r)
+                    if (row[r] >= 0) acc = fmaf(g[r], Elem<XT>::to_f(ye[row[r] * d + c]), acc);
+                dst[c] = Elem<XT>::from_f(acc);
+            }
         }
     }
 }
@@ -102,7 +143,7 @@ gate_grad_kernel(const XT* __restrict__ dout, const XT* __restrict__ ye, const i
 
 cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
     if (a.T <= 0) return cudaSuccess;
-    const unsigned grid = (unsigned)((a.T + 7) / 8);
+    const unsigned grid = (unsigned)((a.T + 8 * kCombineTokens - 1) / (8 * kCombineTokens));
     if (a.dtype == MOE_BF16)
         return launch_k(combine_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, 1,
                         reinterpret_cast<const __nv_bfloat16*>(a.ye), a.idx, a.pos, a.drop, a.gate, a.offsets,
