@@ -50,8 +50,8 @@ NCU_TRAFFIC = {
     # then the same under ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none
     #     -k regex:grouped_gemm -s 6 -c 2 (first timed forward): stage 1 read 402802944 B (W1 + xe, the
     # compulsory set) and wrote 360883200 B (H, part of it still in L2 when the kernel ends).  Keyed to the
-    # GEMM's sources (gemm_tc.cu, tc_common.cuh) at the capture.
-    "switch_base": {"bytes_per_launch": 402802944 + 360883200, "src_sha": "85fd46671a9f042a"},
+    # GEMM's sources (gemm_tc.cu, tc_common.cuh): those of the capture with one comment corrected since.
+    "switch_base": {"bytes_per_launch": 402802944 + 360883200, "src_sha": "6d1c0c0b0966e2fa"},
 }
 
 

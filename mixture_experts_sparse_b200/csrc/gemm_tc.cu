@@ -235,9 +235,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             // run a wave later: the B lines are loaded evict-last, so the stream
             // of A rows (read by an m-block's n-tiles at about the same time, then
             // dead) does not evict weights that are read again.  Stage-2 DRAM
-            // reads over the compulsory H + W2: Switch-Base 1.052x -> 1.028x,
-            // top-2 1.083x -> 1.035x (A evict-first as well: 1.29x, the n-tiles
-            // then miss each other's rows).
+            // reads over the compulsory H + W2 (ncu, several captures):
+            // Switch-Base 1.052x -> 1.03-1.04x, top-2 1.083x -> 1.04-1.05x (A
+            // evict-first as well: 1.29x, the n-tiles then miss each other's rows).
             const bool hint = ntn <= 4;
             const uint64_t pol_b = l2_evict_last();
             int stage = 0;
