@@ -219,6 +219,29 @@ def test_every_token_to_one_expert():
     assert np.all(got[400:] == 0.0) and np.all(np.abs(got[:400]).sum(1) > 0)
 
 
+@pytest.mark.parametrize("T,C", [(2500, 400), (6000, 50)])
+def test_dropped_rows_zeroed_over_stale_output(T, C):
+    # top-1 bf16: the second GEMM writes only the kept tokens' rows, and the
+    # dispatch zeroes the rows of dropped tokens.  The output starts as NaN
+    # before each of two calls, and every dropped row must come back exactly 0
+    # (most tokens are dropped here), the rest identical to the first call.
+    bias = np.full(8, -20.0, np.float32)
+    bias[3] = 0.0
+    bias[5] = -0.5
+    layer, res, got = _edge(T, 128, 256, 8, 1, C, router_bias=bias)
+    drop = res["disp"]["drop"][:, 0].astype(bool)
+    assert drop.sum() > T // 2
+    x = to_device(inputs.make_layer(T=T, d_model=128, d_ff=256, n_experts=8, top_k=1, seed=3,
+                                    router_bias=bias)["x"])
+    for _ in range(2):
+        layer.out.view(torch.int16).fill_(-1)   # bf16 0xFFFF: NaN
+        nat.check(layer.forward(x))
+        torch.cuda.synchronize()
+        again = widen_out(layer.out)
+        assert np.all(again[drop] == 0.0)
+        np.testing.assert_array_equal(again, got)
+
+
 def test_zero_router_ties_lowest_index():
     layer, res, got = _edge(333, 64, 128, 8, 2, 333, w_r_zero=True)
     assert np.all(res["routing"]["idx"][:, 0] == 0) and np.all(res["routing"]["idx"][:, 1] == 1)
