@@ -242,9 +242,9 @@ __device__ __forceinline__ int claim_slot(int64_t a, const int32_t* __restrict__
 // per warp instead of one per row), then the warp moves the rows two at a
 // time -- a kept row's x[t] into its compact row, a dropped token's output row
 // set to zero when zero_out is given -- with up to 2 x kCopyUnroll 16-byte
-// loads per lane in flight.  The grid is a single wave at Switch-Base sizes
-// (8192 blocks of one assignment per warp, each living about a microsecond,
-// were bound by block launches).
+// loads per lane in flight.  At Switch-Base sizes that is 1024 blocks of 256
+// threads (about two waves); with one assignment per warp, 8192 blocks each
+// living about a microsecond were bound by block launches.
 constexpr int kScatterRows = 8;
 constexpr int kCopyUnroll = 4;
 
