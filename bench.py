@@ -48,10 +48,10 @@ FP32_PEAK_NOTE = "148 SMs x 128 FP32 lanes x 2 flop x SM clock"
 NCU_TRAFFIC = {
     # python bench.py --only --steps 3 --warmup 3 --no-cpu-baseline --no-backward --workload switch_base,
     # then the same under ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none
-    #     -k regex:grouped_gemm -s 6 -c 2 (first timed forward): stage 1 read 402802944 B (W1 + xe, the
-    # compulsory set) and wrote 360883200 B (H, part of it still in L2 when the kernel ends).  Keyed to the
-    # GEMM's sources (gemm_tc.cu, tc_common.cuh): those of the capture with one comment corrected since.
-    "switch_base": {"bytes_per_launch": 402802944 + 360883200, "src_sha": "6d1c0c0b0966e2fa"},
+    #     -k regex:grouped_gemm -s 6 -c 2 (first timed forward): stage 1 read 402801664 B (W1 + xe, the
+    # compulsory set) and wrote 361353728 B (H, part of it still in L2 when the kernel ends).  Keyed to the
+    # GEMM's sources (gemm_tc.cu, tc_common.cuh) at the capture.
+    "switch_base": {"bytes_per_launch": 402801664 + 361353728, "src_sha": "b39b3c9c3aa50846"},
 }
 
 

@@ -96,6 +96,9 @@ struct GemmParams {
     void* const* out_ptrs;        // scatter to several GPUs: row r goes to out_ptrs[row_rank[r]]
     const int32_t* row_rank;
     __nv_bfloat16* pre_out;       // SwiGLU (optional): the pre-activations W1 x + b1 | W3 x + b3, [R, 2 n_dim]
+    // 1: tiles in reverse order.  The second GEMM starts with the last experts,
+    // whose rows of H the first GEMM wrote last and L2 still holds.
+    int reverse;
     int32_t* status;
     long long limit_ns;
 };
@@ -247,7 +250,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             for (int s = 0; s < S::STAGES; ++s) last_par[s] = -1;
             bool ok = true;
             for (int tile = first_tile; tile < total && ok; tile += tile_step) {
-                const TileInfo ti = decode_tile<S::TILE_M>(tile, s_prefix, s_off, N, ntn, BN_OUT);
+                const TileInfo ti = decode_tile<S::TILE_M>(p.reverse ? total - 1 - tile : tile, s_prefix, s_off, N, ntn, BN_OUT);
                 const int arow = ti.row0 + (int)rank * BM;
                 const int brow = ti.e * p.n_dim + ti.n0 + ((PAIR && EPI != EPI_SWIGLU) ? (int)rank * (BN / 2) : 0);
                 const CUtensorMap* bmap = (EPI == EPI_SWIGLU && PAIR && rank == 1) ? &tmB3 : &tmB;
@@ -382,7 +385,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         constexpr int CW = 64;                  // output columns per chunk
         int it = 0;
         for (int tile = first_tile; tile < total; tile += tile_step, ++it) {
-            const TileInfo ti = decode_tile<S::TILE_M>(tile, s_prefix, s_off, N, ntn, BN_OUT);
+            const TileInfo ti = decode_tile<S::TILE_M>(p.reverse ? total - 1 - tile : tile, s_prefix, s_off, N, ntn, BN_OUT);
             const int acc = it & 1;
             const uint32_t acc_par = (uint32_t)((it >> 1) & 1);
             // the row's destination (and, scattering, its token and gate) are
@@ -750,6 +753,7 @@ cudaError_t launch_expert_ffn_tc(const FfnArgs& a, cudaStream_t s) {
     p2.out_ld = a.d;
     p2.bias = reinterpret_cast<const __nv_bfloat16*>(a.b2);
     p2.status = &a.hdr->status;
+    p2.reverse = 1;
     p2.limit_ns = kWaitLimitNs;
     if (a.scatter_out || a.scatter_ptrs) {
         p2.out = reinterpret_cast<__nv_bfloat16*>(a.scatter_out);
