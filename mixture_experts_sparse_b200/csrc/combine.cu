@@ -114,29 +114,62 @@ combine_kernel(const XT* __restrict__ ye, const int32_t* __restrict__ idx, const
 
 // dL/dgate[t, r] = <dout_t, ye[offsets[idx[t,r]] + pos[t,r]]> for a kept
 // assignment, 0 for a dropped one: the gate's gradient for the router backward
-// (out_t = sum_r gate_{t,r} E(x_t), "From Switch Transformer to GLaM").  One
-// warp per assignment, fp32 accumulation, a fixed shuffle tree.
+// (out_t = sum_r gate_{t,r} E(x_t), "From Switch Transformer to GLaM").  A warp
+// per kGradAssign assignments, laid out like the combine: lanes locate the
+// rows together, then per assignment every 16-byte load of both rows is in
+// flight before the fp32 products are summed; a fixed shuffle tree finishes
+// each dot product.
+constexpr int kGradAssign = 4;
+
 template <typename XT>
 __global__ void __launch_bounds__(256)
 gate_grad_kernel(const XT* __restrict__ dout, const XT* __restrict__ ye, const int32_t* __restrict__ idx,
                  const int32_t* __restrict__ pos, const uint8_t* __restrict__ drop,
                  const int32_t* __restrict__ offsets, int64_t T, int d, int k, float* __restrict__ dgate) {
+    constexpr int VEC = 16 / sizeof(XT);
     pdl_wait();
     pdl_launch();
     const int lane = threadIdx.x & 31;
-    const int64_t a = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (a >= T * k) return;
-    const int64_t t = a / k;
-    float acc = 0.f;
-    if (!drop[a]) {
-        const int64_t row = (int64_t)offsets[idx[a]] + pos[a];
-        const XT* g = dout + t * (int64_t)d;
-        const XT* y = ye + row * (int64_t)d;
-        for (int c = lane; c < d; c += 32) acc = fmaf(Elem<XT>::to_f(g[c]), Elem<XT>::to_f(y[c]), acc);
-    }
+    const int64_t n_assign = T * k;
+    const int64_t a0 = ((int64_t)blockIdx.x * 8 + (threadIdx.x >> 5)) * kGradAssign;
+    if (a0 >= n_assign) return;
+    int64_t my_row = -1;   // lane i < kGradAssign: assignment a0 + i's row of ye (-1: dropped)
+    if (lane < kGradAssign && a0 + lane < n_assign && !drop[a0 + lane])
+        my_row = (int64_t)offsets[idx[a0 + lane]] + pos[a0 + lane];
+#pragma unroll 1
+    for (int i = 0; i < kGradAssign; ++i) {
+        const int64_t a = a0 + i;
+        if (a >= n_assign) break;   // warp-uniform
+        const int64_t row = __shfl_sync(0xffffffffu, my_row, i);
+        float acc = 0.f;
+        if (row >= 0) {
+            const XT* g = dout + (a / k) * (int64_t)d;
+            const XT* y = ye + row * (int64_t)d;
+            if (((size_t)d * sizeof(XT)) % 16 == 0) {
+                for (int c0 = lane * VEC; c0 < d; c0 += 32 * VEC * kCombineUnroll) {
+                    uint4 vg[kCombineUnroll], vy[kCombineUnroll];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-    if (lane == 0) dgate[a] = acc;
+                    for (int u = 0; u < kCombineUnroll; ++u) {
+                        const int c = c0 + u * 32 * VEC;
+                        vg[u] = c < d ? __ldg(reinterpret_cast<const uint4*>(g + c)) : make_uint4(0, 0, 0, 0);
+                        vy[u] = c < d ? __ldg(reinterpret_cast<const uint4*>(y + c)) : make_uint4(0, 0, 0, 0);
+                    }
+#pragma unroll
+                    for (int u = 0; u < kCombineUnroll; ++u) {
+                        const XT* xg = reinterpret_cast<const XT*>(&vg[u]);
+                        const XT* xy = reinterpret_cast<const XT*>(&vy[u]);
+#pragma unroll
+                        for (int j = 0; j < VEC; ++j) acc = fmaf(Elem<XT>::to_f(xg[j]), Elem<XT>::to_f(xy[j]), acc);
+                    }
+                }
+            } else {
+                for (int c = lane; c < d; c += 32) acc = fmaf(Elem<XT>::to_f(g[c]), Elem<XT>::to_f(y[c]), acc);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) dgate[a] = acc;
+    }
 }
 
 }  // namespace
@@ -155,7 +188,7 @@ cudaError_t launch_combine(const CombineArgs& a, cudaStream_t s) {
 
 cudaError_t launch_gate_grad(const GateGradArgs& a, cudaStream_t s) {
     if (a.T <= 0) return cudaSuccess;
-    const unsigned grid = (unsigned)((a.T * a.k + 7) / 8);
+    const unsigned grid = (unsigned)((a.T * a.k + 8 * kGradAssign - 1) / (8 * kGradAssign));
     if (a.dtype == MOE_BF16)
         return launch_k(gate_grad_kernel<__nv_bfloat16>, dim3(grid), dim3(256), 0, s, 1,
                         reinterpret_cast<const __nv_bfloat16*>(a.dout), reinterpret_cast<const __nv_bfloat16*>(a.ye),
