@@ -12,7 +12,7 @@
 //  - dW_r = dh^T x, db_r = sum_t dh_t (a contraction over tokens: per
 //    512-token chunk partials, then a fixed-order fp64 sum over chunks), and
 //    dx_t = dh_t W_r.
-// Kernels: router_bwd_dh_kernel (one warp per token); for bf16 x the two
+// Kernels: router_bwd_dh_kernel (a warp per eight tokens); for bf16 x the two
 // contractions run on the tensor cores through exact three-way bf16 splits
 // (rbwd_* kernels, the grouped GEMMs of gemm_bwd.cu); for fp32 x on the FP32
 // pipe: router_bwd_dw_kernel (32 experts x 128 columns per block over one
@@ -26,6 +26,12 @@ namespace {
 
 constexpr int kBwdChunk = 512;   // tokens per dW_r partial
 
+// dL/dh of kDhTokens consecutive tokens per warp (lane: experts lane + 32 q):
+// the load-balancing coefficients a_e are formed once per warp, and every
+// token's probabilities are loaded before the first is used (with a warp per
+// token, 8192 blocks each living about a microsecond bounded the kernel).
+constexpr int kDhTokens = 8;
+
 __global__ void __launch_bounds__(256)
 router_bwd_dh_kernel(const float* __restrict__ probs, const int32_t* __restrict__ idx, const float* __restrict__ gate,
                      const float* __restrict__ dgate, const double* __restrict__ f, float alpha, int64_t T, int N,
@@ -33,46 +39,58 @@ router_bwd_dh_kernel(const float* __restrict__ probs, const int32_t* __restrict_
     pdl_wait();
     pdl_launch();
     const int lane = threadIdx.x & 31;
-    const int64_t t = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
-    if (t >= T) return;
-    const float* p = probs + t * N;
-    float pv[4], av[4];
-    float spa = 0.f;
+    const int64_t t0 = ((int64_t)blockIdx.x * 8 + (threadIdx.x >> 5)) * kDhTokens;
+    if (t0 >= T) return;
+    float av[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const int e = lane + 32 * q;
-        pv[q] = e < N ? p[e] : 0.f;
         av[q] = e < N ? (float)((double)alpha * (double)N * f[e] / (double)T) : 0.f;
-        spa = fmaf(pv[q], av[q], spa);
     }
+    float pv[kDhTokens][4];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) spa += __shfl_xor_sync(0xffffffffu, spa, o);
-    float gv[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) gv[q] = pv[q] * (av[q] - spa);
-    if (k == 1) {
-        const int is = idx[t];
-        const float c = dgate[t] * gate[t];
+    for (int i = 0; i < kDhTokens; ++i)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             const int e = lane + 32 * q;
-            gv[q] += c * ((e == is ? 1.f : 0.f) - pv[q]);
+            pv[i][q] = (t0 + i < T && e < N) ? probs[(t0 + i) * N + e] : 0.f;
         }
-    } else {
-        const int i1 = idx[2 * t], i2 = idx[2 * t + 1];
-        const float g1 = gate[2 * t], g2 = gate[2 * t + 1];
-        const float c = (dgate[2 * t] - dgate[2 * t + 1]) * g1 * g2;
+#pragma unroll
+    for (int i = 0; i < kDhTokens; ++i) {
+        const int64_t t = t0 + i;
+        if (t >= T) break;   // warp-uniform
+        float spa = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) spa = fmaf(pv[i][q], av[q], spa);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) spa += __shfl_xor_sync(0xffffffffu, spa, o);
+        float gv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) gv[q] = pv[i][q] * (av[q] - spa);
+        if (k == 1) {
+            const int is = idx[t];
+            const float c = dgate[t] * gate[t];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int e = lane + 32 * q;
+                gv[q] += c * ((e == is ? 1.f : 0.f) - pv[i][q]);
+            }
+        } else {
+            const int i1 = idx[2 * t], i2 = idx[2 * t + 1];
+            const float g1 = gate[2 * t], g2 = gate[2 * t + 1];
+            const float c = (dgate[2 * t] - dgate[2 * t + 1]) * g1 * g2;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const int e = lane + 32 * q;
+                if (e == i1) gv[q] += c;
+                if (e == i2) gv[q] -= c;
+            }
+        }
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             const int e = lane + 32 * q;
-            if (e == i1) gv[q] += c;
-            if (e == i2) gv[q] -= c;
+            if (e < N) dh[t * N + e] = gv[q];
         }
-    }
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const int e = lane + 32 * q;
-        if (e < N) dh[t * N + e] = gv[q];
     }
 }
 
@@ -227,6 +245,8 @@ __device__ __forceinline__ void split3(float v, __nv_bfloat16& a, __nv_bfloat16&
     c = __float2bfloat16_rn(r1 - __bfloat162float(b));
 }
 
+// A thread splits eight consecutive experts of one token (NP16 is a multiple
+// of 16), so every row segment it writes is one 16-byte store.
 __global__ void __launch_bounds__(256)
 rbwd_split_kernel(const float* __restrict__ dh, int64_t T, int N, int NP16, __nv_bfloat16* __restrict__ adx,
                   __nv_bfloat16* __restrict__ adw, int32_t* __restrict__ offs, int64_t chunk, int nchunk) {
@@ -237,24 +257,36 @@ rbwd_split_kernel(const float* __restrict__ dh, int64_t T, int N, int NP16, __nv
         offs[1] = (int32_t)T;
         for (int i = 0; i <= nchunk; ++i) offs[2 + i] = (int32_t)min((int64_t)i * chunk, T);
     }
-    const int64_t n_el = T * NP16;
+    const int per_row = NP16 / 8;
+    const int64_t n_el = T * per_row;
     for (int64_t q = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; q < n_el; q += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t t = q / NP16;
-        const int e = (int)(q - t * NP16);
-        const float v = e < N ? dh[t * N + e] : 0.f;
-        __nv_bfloat16 h0, h1, h2;
-        split3(v, h0, h1, h2);
-        __nv_bfloat16* rx = adx + t * (6 * NP16) + e;
-        rx[0] = h0;
-        rx[NP16] = h0;
-        rx[2 * NP16] = h1;
-        rx[3 * NP16] = h0;
-        rx[4 * NP16] = h1;
-        rx[5 * NP16] = h2;
-        __nv_bfloat16* rw = adw + t * (3 * NP16) + e;
-        rw[0] = h0;
-        rw[NP16] = h1;
-        rw[2 * NP16] = h2;
+        const int64_t t = q / per_row;
+        const int e0 = (int)(q - t * per_row) * 8;
+        uint32_t p0[4], p1[4], p2[4];   // the eight experts' three parts, packed bf16 pairs
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            __nv_bfloat16 a0, a1, a2, b0, b1, b2;
+            const int e = e0 + 2 * h;
+            split3(e < N ? dh[t * N + e] : 0.f, a0, a1, a2);
+            split3(e + 1 < N ? dh[t * N + e + 1] : 0.f, b0, b1, b2);
+            p0[h] = (uint32_t)__bfloat16_as_ushort(a0) | ((uint32_t)__bfloat16_as_ushort(b0) << 16);
+            p1[h] = (uint32_t)__bfloat16_as_ushort(a1) | ((uint32_t)__bfloat16_as_ushort(b1) << 16);
+            p2[h] = (uint32_t)__bfloat16_as_ushort(a2) | ((uint32_t)__bfloat16_as_ushort(b2) << 16);
+        }
+        const uint4 v0 = make_uint4(p0[0], p0[1], p0[2], p0[3]);
+        const uint4 v1 = make_uint4(p1[0], p1[1], p1[2], p1[3]);
+        const uint4 v2 = make_uint4(p2[0], p2[1], p2[2], p2[3]);
+        __nv_bfloat16* rx = adx + t * (6 * NP16) + e0;   // K segments: parts 0, 0, 1, 0, 1, 2
+        *reinterpret_cast<uint4*>(rx) = v0;
+        *reinterpret_cast<uint4*>(rx + NP16) = v0;
+        *reinterpret_cast<uint4*>(rx + 2 * NP16) = v1;
+        *reinterpret_cast<uint4*>(rx + 3 * NP16) = v0;
+        *reinterpret_cast<uint4*>(rx + 4 * NP16) = v1;
+        *reinterpret_cast<uint4*>(rx + 5 * NP16) = v2;
+        __nv_bfloat16* rw = adw + t * (3 * NP16) + e0;
+        *reinterpret_cast<uint4*>(rw) = v0;
+        *reinterpret_cast<uint4*>(rw + NP16) = v1;
+        *reinterpret_cast<uint4*>(rw + 2 * NP16) = v2;
     }
 }
 
@@ -283,7 +315,16 @@ rbwd_db_kernel(const float* __restrict__ dh, int64_t T, int N, int64_t chunk, fl
     if (e >= N) return;
     const int64_t t0 = (int64_t)blockIdx.x * chunk, t1 = min(T, t0 + chunk);
     float acc = 0.f;
-    for (int64_t t = t0; t < t1; ++t) acc += dh[t * N + e];
+    constexpr int B = 64;   // loads in flight, then added in token order
+    int64_t t = t0;
+    for (; t + B <= t1; t += B) {
+        float v[B];
+#pragma unroll
+        for (int j = 0; j < B; ++j) v[j] = dh[(t + j) * N + e];
+#pragma unroll
+        for (int j = 0; j < B; ++j) acc += v[j];
+    }
+    for (; t < t1; ++t) acc += dh[t * N + e];
     part_db[(int64_t)blockIdx.x * N + e] = acc;
 }
 
@@ -337,7 +378,8 @@ cudaError_t launch_router_backward(const RouterBwdArgs& a, cudaStream_t s) {
         if (e == cudaSuccess && a.db) e = cudaMemsetAsync(a.db, 0, sizeof(float) * a.N, s);
         return e;
     }
-    cudaError_t err = launch_k(router_bwd_dh_kernel, dim3((unsigned)((a.T + 7) / 8)), dim3(256), 0, s, 1, a.probs,
+    cudaError_t err = launch_k(router_bwd_dh_kernel, dim3((unsigned)((a.T + 8 * kDhTokens - 1) / (8 * kDhTokens))),
+                               dim3(256), 0, s, 1, a.probs,
                                a.idx, a.gate, a.dgate, a.f, a.alpha, a.T, a.N, a.k, a.dh);
     if (err != cudaSuccess) return err;
     if (a.dtype == MOE_BF16 && a.tc_adx && (a.dw || a.db || a.dx)) {
@@ -345,7 +387,7 @@ cudaError_t launch_router_backward(const RouterBwdArgs& a, cudaStream_t s) {
         const int NP16 = router_bwd_np16(a.N);
         const int64_t chunk = router_bwd_tc_chunk(a.T);
         const int nchunk = router_bwd_tc_chunks(a.T);
-        const int64_t n_el = a.T * NP16;
+        const int64_t n_el = a.T * (NP16 / 8);   // a thread per eight experts of a token
         const unsigned sg = (unsigned)((n_el + 255) / 256 < 8192 ? (n_el + 255) / 256 : 8192);
         if ((err = launch_k(rbwd_split_kernel, dim3(sg), dim3(256), 0, s, 1, static_cast<const float*>(a.dh), a.T,
                             a.N, NP16, reinterpret_cast<__nv_bfloat16*>(a.tc_adx),
