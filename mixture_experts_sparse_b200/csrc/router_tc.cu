@@ -62,7 +62,7 @@ struct RtShape {
     // accumulator stays 2^8 below the logits and its truncation error with it.
     static constexpr bool MERGED = 3 * NP <= 256;
     // K boxes (64 deep) per pipeline stage: two when merged (8 MMAs per
-    // barrier round trip), one otherwise (three MMAs per K slice already)
+    // barrier round trip), one otherwise (two MMAs per K slice, 8 per stage)
     static constexpr int KSUB = MERGED ? 2 : 1;
     static constexpr int A_SUB = RT_BM * RT_BK * 2;             // one x box
     static constexpr int A_BYTES = A_SUB * KSUB;
